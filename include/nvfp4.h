@@ -1,0 +1,192 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 block quantization, dequantization
+ * and the block-scaled FP4 GEMM on B200 (sm_100a).
+ *
+ * What the calls compute is defined by these pages (cited by title and
+ * section / equation):
+ *   [46] "Four Over Six: more accurate NVFP4 quantization with adaptive block
+ *        scaling" (Chinese translation): §1 (Fig. 1, Table 1), §2.1 Eq. 1-3.
+ *   [NV] Write-up of NVIDIA's "Pretraining LLMs with NVFP4": §一 format,
+ *        §二 the four techniques (2D weight blocks, random Hadamard transform,
+ *        stochastic rounding), §四 Blackwell tensor cores, §六 procedure,
+ *        §七 ablations (SR on gradients only, 1D blocks for activations).
+ *   [Q2] News write-up of Quartet II / MS-EDEN: §一 (MS-EDEN), §二 (recipe).
+ *
+ * Conventions shared by every call
+ *   - All device pointers are caller-owned CUDA device memory; the library
+ *     never allocates.  Scratch memory comes from the caller's workspace.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Nothing synchronises the
+ *     host; the tensor scale alpha stays on the device.
+ *   - Errors the host can see (bad arguments, shapes, alignment, workspace
+ *     too small) return before anything is launched.  Errors found on the
+ *     device (non-finite input, a spin-wait that gave up) are written as a
+ *     negative nvfp4_status_t to the optional device word `status`; that word
+ *     is sticky: the library only ever writes error codes into it, the caller
+ *     zeroes it.  Outputs are unspecified after a device-side error.
+ *   - bf16 tensors are row-major with a row stride `ld` (elements); the base
+ *     pointer must be 16-byte aligned and ld a multiple of 8.
+ *   - Packed FP4 codes: two E2M1 codes per byte, element 2j in the low nibble
+ *     of byte j; a code is sign (bit 3) + magnitude index (bits 0-2) into
+ *     {0, 0.5, 1, 1.5, 2, 3, 4, 6} ([46] §1).
+ *   - Block scales: one unsigned E4M3 byte (bias 7, max 448) per block.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_ARG = -1,        /* bad mode, flag combination or null pointer */
+  NVFP4_ERR_SHAPE = -2,      /* a dimension breaks the block / tile rules   */
+  NVFP4_ERR_ALIGN = -3,      /* a pointer or stride is not 16-byte aligned  */
+  NVFP4_ERR_NONFINITE = -4,  /* device: the input holds a NaN or an Inf     */
+  NVFP4_ERR_LAUNCH = -5,     /* a kernel could not be launched              */
+  NVFP4_ERR_TIMEOUT = -6,    /* device: a bounded spin-wait gave up         */
+  NVFP4_ERR_CUDA = -7,       /* a CUDA runtime call failed                  */
+  NVFP4_ERR_WORKSPACE = -8   /* workspace missing or smaller than required  */
+} nvfp4_status_t;
+
+/* How a 16-element block is encoded. */
+typedef enum {
+  /* Eq. 2 scale rounded to nearest E4M3, Eq. 3 values rounded to nearest
+   * ([46] §2.1, [NV] §六).  Block maximum mapped to 6. */
+  NVFP4_RTN = 0,
+  /* Four Over Six ([46] §1, [Q2] §二): encode the block with its maximum
+   * mapped to 6 and to 4, keep the encoding with the lower squared error
+   * measured after dequantization (ties keep 6). */
+  NVFP4_FOUR_SIX = 1,
+  /* Random Hadamard transform of each 16-block, scale rounded up to E4M3,
+   * values stochastically rounded ([NV] §二, §七: for gradients). */
+  NVFP4_RHT_SR = 2,
+  /* MS-EDEN ([Q2] §一): rotate, round the values to nearest, and put the
+   * randomness only on the E4M3 scale, stochastically rounded from the
+   * unbiasing value ||r||^2 / (alpha <r, q>). */
+  NVFP4_MS_EDEN = 3
+} nvfp4_mode_t;
+
+/* nvfp4_quantize flags */
+#define NVFP4_ROWWISE 0x1u          /* blocks along C (the contiguous axis)      */
+#define NVFP4_COLWISE 0x2u          /* blocks along R; output is the transpose   */
+#define NVFP4_BLOCK2D 0x4u          /* 16x16 blocks (weights, [NV] §二); RTN/4-6 */
+#define NVFP4_SINGLE_PASS 0x8u      /* amax and quantize in one cooperative pass */
+#define NVFP4_ALPHA_PROVIDED 0x10u  /* use *alpha_in instead of Eq. 1            */
+#define NVFP4_GEMM_SCALE_LAYOUT 0x20u /* write scales in nvfp4_gemm's layout     */
+#define NVFP4_RHT 0x40u             /* rotate before RTN / FOUR_SIX encoding     */
+/* nvfp4_dequantize flags (NVFP4_BLOCK2D and NVFP4_GEMM_SCALE_LAYOUT also apply) */
+#define NVFP4_INVERSE_RHT 0x80u     /* undo the rotation after decoding          */
+#define NVFP4_OUT_BF16 0x100u       /* write bf16 instead of fp32                */
+
+/* nvfp4_gemm output types */
+#define NVFP4_OUT_DTYPE_BF16 0
+#define NVFP4_OUT_DTYPE_FP32 1
+
+/* Outputs of nvfp4_quantize.  NULL members are not written; the row members
+ * are required with NVFP4_ROWWISE, the column members with NVFP4_COLWISE.
+ *   codes_row  [R, C/2] bytes            codes_col  [C, R/2] bytes
+ *   scales_row [R, C/16]                 scales_col [C, R/16]
+ *              BLOCK2D: [R/16, C/16]                BLOCK2D: [C/16, R/16]
+ *              GEMM layout: see below               GEMM layout: see below
+ *   alpha_row, alpha_col: one float each (device), the tensor scale of Eq. 1
+ *   amax_out:  optional float[2] (device): amax seen by rows, by columns
+ *   status:    optional sticky device error word (see conventions)
+ * Column outputs hold the transpose: row c of codes_col / scales_col encodes
+ * column c of x, so both outputs are K-major GEMM operands.
+ *
+ * GEMM scale layout (NVFP4_GEMM_SCALE_LAYOUT), for an operand with `rows`
+ * rows and K columns (rows % 128 == 0, K % 64 == 0): the scale of (row m,
+ * K-block j) sits at byte
+ *     ((m / 128) * (K / 64) + j / 4) * 512 + (m % 32) * 16 + ((m / 32) % 4) * 4 + j % 4,
+ * i.e. 512-byte atoms of 128 rows x 4 scales, in the order the tcgen05
+ * block-scaled MMA reads them.  With BLOCK2D the 16x16 scale is written for
+ * every one of its 16 rows (rows x K/16 bytes in total). */
+typedef struct {
+  uint8_t* codes_row;
+  uint8_t* scales_row;
+  float* alpha_row;
+  uint8_t* codes_col;
+  uint8_t* scales_col;
+  float* alpha_col;
+  float* amax_out;
+  int32_t* status;
+} nvfp4_qtensor_t;
+
+/* Bytes of device workspace nvfp4_quantize needs for an R x C tensor and
+ * these flags (0 if none).  The workspace is scratch: its contents on entry
+ * do not matter, and one workspace must not be shared by calls that may run
+ * at the same time. */
+size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
+
+/* Quantize the bf16 tensor x [R, C] (row stride ld) to NVFP4.
+ *
+ * Steps ([46] §2.1 Eq. 1-3; [NV] §六):
+ *   1. amax = max |x| (max over the rotated values in rotating modes,
+ *      separately per orientation); alpha = amax / (6 * 448)        (Eq. 1)
+ *      -- skipped with NVFP4_ALPHA_PROVIDED (alpha = *alpha_in, device).
+ *   2. per block: Delta = E4M3(amax_block / (alpha * M))             (Eq. 2)
+ *   3. per element: q = E2M1(x / (alpha * Delta)), computed as x times the
+ *      correctly rounded reciprocal of alpha * Delta                 (Eq. 3)
+ * with the mode choosing M, the rounding of Delta and q, and the 4/6 choice
+ * (see nvfp4_mode_t).  Rotating modes (RHT_SR, MS_EDEN, or the NVFP4_RHT
+ * flag) first replace each 16-block v by (1/4) H16 D v, D = diag of 16 random
+ * signs drawn from `seed`; the same D serves every block and both
+ * orientations, so two operands quantized with the same seed along their
+ * shared K axis multiply to the unrotated product.
+ *
+ * Random bits come from Philox4x32-10 keyed by `seed`; `stream_id` (< 2^31)
+ * separates the noise of tensors that share a seed.
+ *
+ * Shape rules: R, C >= 0; C % 16 == 0 with NVFP4_ROWWISE, R % 16 == 0 with
+ * NVFP4_COLWISE; both with NVFP4_BLOCK2D (RTN / FOUR_SIX only, no rotation).
+ * Output pointers: 16-byte aligned.  `workspace` must hold
+ * nvfp4_workspace_size(R, C, flags) bytes.  Arithmetic is IEEE binary32
+ * without FMA contraction, so codes and scales are bit-exact with a plain
+ * CPU restatement of these steps. */
+nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld,
+                              nvfp4_mode_t mode, uint32_t flags, uint64_t seed,
+                              uint32_t stream_id, const float* alpha_in,
+                              const nvfp4_qtensor_t* out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Decode packed codes [R, C/2] with scales ([R, C/16]; BLOCK2D [R/16, C/16];
+ * or the GEMM layout with NVFP4_GEMM_SCALE_LAYOUT) and the device tensor
+ * scale *alpha:  y = q * (alpha * Delta)  (the inverse of Eq. 3), optionally
+ * followed by the inverse rotation x = D (1/4) H16 y (NVFP4_INVERSE_RHT, key
+ * `seed`).  y is fp32 [R, C], or bf16 with NVFP4_OUT_BF16 (rounded to
+ * nearest even), row-major, contiguous. */
+nvfp4_status_t nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
+                                const float* alpha, int64_t R, int64_t C,
+                                uint32_t flags, uint64_t seed, void* y,
+                                void* stream);
+
+/* Block-scaled NVFP4 GEMM on the tcgen05 tensor cores ([NV] §四):
+ *     D[m, n] = alphaA * alphaB * sum_k (qA[m,k] DeltaA[m,k/16]) (qB[n,k] DeltaB[n,k/16])
+ * A: codes [M, K/2], B: codes [N, K/2] (both K-major, "TN"); sA, sB: scales
+ * in the GEMM layout above (as written by nvfp4_quantize with
+ * NVFP4_GEMM_SCALE_LAYOUT); alphaA, alphaB: device floats.  Products are
+ * accumulated in FP32; D is bf16 (NVFP4_OUT_DTYPE_BF16) or fp32, row-major
+ * with row stride ldd elements.  M % 128 == 0, N % 128 == 0, K % 128 == 0;
+ * A, B, sA, sB, D 16-byte aligned.  No workspace is needed (pass NULL, 0). */
+nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const float* alphaA,
+                          const uint8_t* B, const uint8_t* sB, const float* alphaB,
+                          int64_t M, int64_t N, int64_t K, void* D, int out_dtype,
+                          int64_t ldd, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Static description of a status code. */
+const char* nvfp4_status_string(nvfp4_status_t status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */
