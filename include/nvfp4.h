@@ -37,6 +37,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -121,7 +127,7 @@ typedef struct {
  * these flags (0 if none).  The workspace is scratch: its contents on entry
  * do not matter, and one workspace must not be shared by calls that may run
  * at the same time. */
-size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
+NVFP4_API size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
 
 /* Quantize the bf16 tensor x [R, C] (row stride ld) to NVFP4.
  *
@@ -142,13 +148,14 @@ size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
  * Random bits come from Philox4x32-10 keyed by `seed`; `stream_id` (< 2^31)
  * separates the noise of tensors that share a seed.
  *
- * Shape rules: R, C >= 0; C % 16 == 0 with NVFP4_ROWWISE, R % 16 == 0 with
- * NVFP4_COLWISE; both with NVFP4_BLOCK2D (RTN / FOUR_SIX only, no rotation).
+ * Shape rules: R, C >= 0; C % 16 == 0; R % 16 == 0 with NVFP4_COLWISE or
+ * NVFP4_BLOCK2D (2D blocks: RTN / FOUR_SIX only, no rotation);
+ * R * C / 16 < 2^31.  An empty tensor (R or C = 0) is a no-op.
  * Output pointers: 16-byte aligned.  `workspace` must hold
  * nvfp4_workspace_size(R, C, flags) bytes.  Arithmetic is IEEE binary32
  * without FMA contraction, so codes and scales are bit-exact with a plain
  * CPU restatement of these steps. */
-nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld,
+NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld,
                               nvfp4_mode_t mode, uint32_t flags, uint64_t seed,
                               uint32_t stream_id, const float* alpha_in,
                               const nvfp4_qtensor_t* out, void* workspace,
@@ -160,7 +167,7 @@ nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld,
  * followed by the inverse rotation x = D (1/4) H16 y (NVFP4_INVERSE_RHT, key
  * `seed`).  y is fp32 [R, C], or bf16 with NVFP4_OUT_BF16 (rounded to
  * nearest even), row-major, contiguous. */
-nvfp4_status_t nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
+NVFP4_API nvfp4_status_t nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
                                 const float* alpha, int64_t R, int64_t C,
                                 uint32_t flags, uint64_t seed, void* y,
                                 void* stream);
@@ -172,18 +179,21 @@ nvfp4_status_t nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
  * NVFP4_GEMM_SCALE_LAYOUT); alphaA, alphaB: device floats.  Products are
  * accumulated in FP32; D is bf16 (NVFP4_OUT_DTYPE_BF16) or fp32, row-major
  * with row stride ldd elements.  M % 128 == 0, N % 128 == 0, K % 128 == 0;
- * A, B, sA, sB, D 16-byte aligned.  No workspace is needed (pass NULL, 0). */
-nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const float* alphaA,
+ * A, B, sA, sB, D 16-byte aligned.  The GEMM needs no scratch memory: the
+ * workspace is optional (NULL, 0); when given (>= 4 bytes) its first int32 is
+ * used as the sticky device status word (NVFP4_ERR_TIMEOUT if a bounded
+ * pipeline wait gave up). */
+NVFP4_API nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const float* alphaA,
                           const uint8_t* B, const uint8_t* sB, const float* alphaB,
                           int64_t M, int64_t N, int64_t K, void* D, int out_dtype,
                           int64_t ldd, void* workspace, size_t workspace_bytes,
                           void* stream);
 
 /* Static description of a status code. */
-const char* nvfp4_status_string(nvfp4_status_t status);
+NVFP4_API const char* nvfp4_status_string(nvfp4_status_t status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
-int nvfp4_version(void);
+NVFP4_API int nvfp4_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,125 @@
+"""torch-facing wrappers of the C ABI: allocate outputs with torch (device
+memory and the current stream are the only things torch supplies) and call
+libnvfp4.so.  Every step of the computation runs in the library's kernels.
+"""
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+from ._lib import (NVFP4_ALPHA_PROVIDED, NVFP4_BLOCK2D, NVFP4_COLWISE, NVFP4_FOUR_SIX,  # noqa: F401
+                   NVFP4_GEMM_SCALE_LAYOUT, NVFP4_INVERSE_RHT, NVFP4_MS_EDEN, NVFP4_OUT_BF16,
+                   NVFP4_OUT_DTYPE_BF16, NVFP4_OUT_DTYPE_FP32, NVFP4_RHT, NVFP4_RHT_SR,
+                   NVFP4_ROWWISE, NVFP4_RTN, NVFP4_SINGLE_PASS)
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {L.nvfp4_status_string(status)} (status {status})")
+        self.status = status
+
+
+def _check(status: int, what: str):
+    if status != L.NVFP4_OK:
+        raise NVFP4Error(status, what)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+@dataclass
+class QTensor:
+    """NVFP4 outputs of one quantize call (device tensors)."""
+    codes_row: Optional[torch.Tensor] = None
+    scales_row: Optional[torch.Tensor] = None
+    alpha_row: Optional[torch.Tensor] = None
+    codes_col: Optional[torch.Tensor] = None
+    scales_col: Optional[torch.Tensor] = None
+    alpha_col: Optional[torch.Tensor] = None
+    amax: Optional[torch.Tensor] = None
+
+
+def scale_shape(rows: int, cols: int, flags: int):
+    """Shape of the scale tensor of an operand [rows, cols] (cols = the
+    blocked axis)."""
+    if flags & NVFP4_GEMM_SCALE_LAYOUT:
+        return (rows * (cols // 16),)
+    if flags & NVFP4_BLOCK2D:
+        return (rows // 16, cols // 16)
+    return (rows, cols // 16)
+
+
+def alloc_outputs(R: int, C: int, flags: int, device) -> QTensor:
+    q = QTensor()
+    u8 = dict(dtype=torch.uint8, device=device)
+    if flags & NVFP4_ROWWISE:
+        q.codes_row = torch.empty((R, C // 2), **u8)
+        q.scales_row = torch.empty(scale_shape(R, C, flags), **u8)
+        q.alpha_row = torch.empty(1, dtype=torch.float32, device=device)
+    if flags & NVFP4_COLWISE:
+        q.codes_col = torch.empty((C, R // 2), **u8)
+        q.scales_col = torch.empty(scale_shape(C, R, flags), **u8)
+        q.alpha_col = torch.empty(1, dtype=torch.float32, device=device)
+    q.amax = torch.zeros(2, dtype=torch.float32, device=device)
+    return q
+
+
+def workspace_for(R: int, C: int, flags: int, device) -> Optional[torch.Tensor]:
+    n = L.nvfp4_workspace_size(R, C, flags)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream_id: int = 0,
+                   alpha: Optional[torch.Tensor] = None, out: Optional[QTensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None) -> QTensor:
+    """Quantize a 2D bf16 CUDA tensor (unit column stride) with the C ABI's
+    nvfp4_quantize; allocates outputs and workspace when not given."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2D bfloat16 CUDA tensor")
+    if x.numel() and x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    R, C = x.shape
+    ld = x.stride(0) if x.numel() else C
+    if alpha is not None:
+        flags |= NVFP4_ALPHA_PROVIDED
+    q = out if out is not None else alloc_outputs(R, C, flags, x.device)
+    ws = workspace if workspace is not None else workspace_for(R, C, flags, x.device)
+    qt = L.nvfp4_qtensor_t(_p(q.codes_row), _p(q.scales_row), _p(q.alpha_row), _p(q.codes_col),
+                           _p(q.scales_col), _p(q.alpha_col), _p(q.amax), _p(status))
+    st = L.nvfp4_quantize(_p(x), R, C, ld, mode, flags, seed, stream_id, _p(alpha), qt, _p(ws),
+                          0 if ws is None else ws.numel(), _stream())
+    _check(st, "nvfp4_quantize")
+    return q
+
+
+def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, alpha: torch.Tensor, R: int, C: int,
+                     flags: int = 0, seed: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Decode [R, C/2] codes to fp32 (or bf16 with NVFP4_OUT_BF16)."""
+    dtype = torch.bfloat16 if flags & NVFP4_OUT_BF16 else torch.float32
+    y = out if out is not None else torch.empty((R, C), dtype=dtype, device=codes.device)
+    st = L.nvfp4_dequantize(_p(codes), _p(scales), _p(alpha), R, C, flags, seed, _p(y), _stream())
+    _check(st, "nvfp4_dequantize")
+    return y
+
+
+def nvfp4_gemm(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch.Tensor,
+               sB: torch.Tensor, alphaB: torch.Tensor, out_dtype: int = NVFP4_OUT_DTYPE_BF16,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """D[M, N] = alphaA alphaB (A dequantized) (B dequantized)^T; A codes
+    [M, K/2], B codes [N, K/2], scales in the GEMM layout."""
+    M, K2 = A.shape
+    N = B.shape[0]
+    K = 2 * K2
+    dt = torch.bfloat16 if out_dtype == NVFP4_OUT_DTYPE_BF16 else torch.float32
+    D = out if out is not None else torch.empty((M, N), dtype=dt, device=A.device)
+    st = L.nvfp4_gemm(_p(A), _p(sA), _p(alphaA), _p(B), _p(sB), _p(alphaB), M, N, K, _p(D), out_dtype,
+                      D.stride(0), None, 0, _stream())
+    _check(st, "nvfp4_gemm")
+    return D

@@ -1,0 +1,344 @@
+// nvfp4_device.cuh -- device-side building blocks of the NVFP4 quantizer.
+//
+// Every floating-point step is one IEEE binary32 operation with round to
+// nearest even, written with the explicit __f*_rn intrinsics so the compiler
+// cannot contract or reorder it; the whole library is also built with
+// -fmad=false.  The encoders follow:
+//   * Four Over Six (Chinese translation), §2.1 Eq. 1-3: tensor scale, block
+//     scale, element rounding; §1 Table 1: the 4/6 selector.
+//   * NVFP4 pretraining write-up, §一 (E2M1 values, E4M3 block scales per 16
+//     values, FP32 tensor scale), §二 (random Hadamard transform, 2D blocks,
+//     stochastic rounding), §四 (hardware conversions with round-to-nearest-even).
+//   * Quartet II / MS-EDEN write-up, §一: rotate, round values to nearest,
+//     randomness on the E4M3 scale only.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3",
+// SC'11).  The ten round keys depend only on the seed, so a thread expands
+// them once and each draw costs ten rounds of two wide multiplies and two
+// three-input XORs.
+// ---------------------------------------------------------------------------
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys K;
+  uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    K.k0[r] = a;
+    K.k1[r] = b;
+    a += 0x9E3779B9u;
+    b += 0xBB67AE85u;
+  }
+  return K;
+}
+
+__device__ __forceinline__ uint4 philox(const PhiloxKeys& K, uint32_t c0, uint32_t c1,
+                                        uint32_t c2, uint32_t c3) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    c0 = hi1 ^ c1 ^ K.k0[r];
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ K.k1[r];
+    c3 = lo0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// Counter words of the quantizer's draws: (unit_lo, unit_hi, c2, tag).
+constexpr uint32_t kTagValueSR = 1u;   // 16-bit fields for element rounding
+constexpr uint32_t kTagScaleSR = 2u;   // 24-bit field for the E4M3 scale
+constexpr uint32_t kTagSigns = 3u;     // the sign diagonal of the rotation
+
+// ---------------------------------------------------------------------------
+// bf16 <-> f32
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 8 bf16 packed in a uint4 -> 8 floats
+__device__ __forceinline__ void unpack8(const uint4 u, float* v) {
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x);
+  v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z);
+  v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 block scales (OCP E4M3FN, non-negative): 127 finite codes, max 448.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = b >> 3, m = b & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
+           : __fmul_rn(static_cast<float>(m), 0.001953125f);  // m * 2^-9, exact
+}
+
+// Round to nearest even, saturating at 448 (hardware conversion; PTX
+// cvt.rn.satfinite.e4m3x2.f32).  v >= 0.
+__device__ __forceinline__ uint32_t e4m3_rne(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return r & 0xFFu;
+}
+
+// Smallest E4M3 value not below v (saturating at 448).  v >= 0.
+__device__ __forceinline__ uint32_t e4m3_ceil(float v) {
+  uint32_t b = e4m3_rne(v);
+  if (b < 0x7Eu && e4m3_value(b) < v) ++b;
+  return b;
+}
+
+// Stochastic rounding to E4M3 with a 24-bit uniform: up iff u24 < f * 2^24,
+// f the position of v between its neighbours.  v >= 0.
+__device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t u24) {
+  if (!(v < 448.0f)) return 0x7Eu;
+  uint32_t lo = e4m3_rne(v);
+  if (e4m3_value(lo) > v) --lo;
+  const float vlo = e4m3_value(lo);
+  if (vlo == v) return lo;
+  const float gap = __fsub_rn(e4m3_value(lo + 1), vlo);        // a power of two
+  const float f = __fdiv_rn(__fsub_rn(v, vlo), gap);           // exact
+  return (static_cast<float>(u24) < __fmul_rn(f, 16777216.0f)) ? lo + 1 : lo;
+}
+
+// ---------------------------------------------------------------------------
+// E2M1 values: codes sign | index into {0, .5, 1, 1.5, 2, 3, 4, 6}.
+// ---------------------------------------------------------------------------
+// Two values -> one byte (lo in bits 0-3, hi in bits 4-7), round to nearest
+// even with saturation at +-6 (PTX cvt.rn.satfinite.e2m1x2.f32).
+__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte of two codes -> their two signed grid values (PTX cvt.rn.f16x2.e2m1x2,
+// exact), widened to float.
+__device__ __forceinline__ void e2m1x2_values(uint32_t byte, float& lo, float& hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2) : "r"(byte));
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// Stochastic rounding of y to the grid with a 16-bit uniform u16: with the
+// grid step 1/m on |y|'s segment ([0,2): 0.5, [2,4): 1, [4,6]: 2), t = |y| m
+// is exact, f = t - floor(t) is the position between the neighbours, and the
+// magnitude rounds up iff u16 < f * 65536.  |y| >= 6 -> 6.  Returns the
+// signed grid value (exactly representable, so its encoding is exact).
+__device__ __forceinline__ float e2m1_sr_value(float y, uint32_t u16) {
+  const float a = fabsf(y);
+  float q;
+  if (a >= 6.0f) {
+    q = 6.0f;
+  } else {
+    const float m = (a < 2.0f) ? 2.0f : ((a < 4.0f) ? 1.0f : 0.5f);
+    const float t = __fmul_rn(a, m);
+    const float fl = floorf(t);
+    const float f = __fsub_rn(t, fl);
+    const float up = (static_cast<float>(u16) < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
+    q = __fdiv_rn(__fadd_rn(fl, up), m);  // m is a power of two: exact
+  }
+  return copysignf(q, y);
+}
+
+// ---------------------------------------------------------------------------
+// 16-wide Hadamard butterfly, natural (Sylvester) order, strides 1, 2, 4, 8.
+// r = (1/4) H16 D v where D flips the signs selected by `signs`.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void rht16(float* v, uint32_t signs) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((signs >> i) & 1u) << 31));
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+}
+
+// Inverse: x = D (1/4) H16 r.
+__device__ __forceinline__ void irht16(float* v, uint32_t signs) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    v[i] = __uint_as_float(__float_as_uint(__fmul_rn(v[i], 0.25f)) ^ (((signs >> i) & 1u) << 31));
+}
+
+// Pairwise sum with strides 8, 4, 2, 1 (the stated summation order).
+__device__ __forceinline__ float sum16(const float* e) {
+  float t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = __fadd_rn(e[i], e[i + 8]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t[i] = __fadd_rn(t[i], t[i + 4]);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) t[i] = __fadd_rn(t[i], t[i + 2]);
+  return __fadd_rn(t[0], t[1]);
+}
+
+__device__ __forceinline__ float max_abs16(const float* v) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+  return m;
+}
+
+// ---------------------------------------------------------------------------
+// Block encoding (one 16-vector).  Codes come back packed: byte j of `lo`
+// (j < 4) holds elements 2j, 2j+1; `hi` holds elements 8..15.
+// ---------------------------------------------------------------------------
+struct Packed16 {
+  uint32_t lo, hi;
+};
+
+// Eq. 2: Delta_raw = amax_b / (alpha * M); the E4M3 rounding is chosen by the
+// caller.  A zero denominator gives 0.
+__device__ __forceinline__ float scale_raw(float amax_b, float alpha, float M) {
+  const float den = __fmul_rn(alpha, M);
+  return (den == 0.0f) ? 0.0f : __fdiv_rn(amax_b, den);
+}
+
+// Eq. 3 with round to nearest: codes of v under stored scale byte sb.  When
+// s = alpha * Delta is 0, or 1/s overflows, the magnitudes are 0 and the
+// codes keep the signs of v.
+__device__ __forceinline__ Packed16 encode_rne(const float* v, float alpha, uint32_t sb) {
+  const float s = __fmul_rn(alpha, e4m3_value(sb));
+  const float rinv = __frcp_rn(s);
+  Packed16 p{0u, 0u};
+  if (isinf(rinv)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t sign = (__float_as_uint(v[i]) >> 31) << 3;
+      if (i < 8) p.lo |= sign << (4 * i);
+      else p.hi |= sign << (4 * (i - 8));
+    }
+    return p;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t b = e2m1x2_rne(__fmul_rn(v[2 * j], rinv), __fmul_rn(v[2 * j + 1], rinv));
+    if (j < 4) p.lo |= b << (8 * j);
+    else p.hi |= b << (8 * (j - 4));
+  }
+  return p;
+}
+
+// Eq. 3 with stochastic rounding of the values; u16[i] are the element's
+// 16-bit uniforms.
+__device__ __forceinline__ Packed16 encode_sr(const float* v, float alpha, uint32_t sb,
+                                              const uint32_t* words /* 8 words */) {
+  const float s = __fmul_rn(alpha, e4m3_value(sb));
+  const float rinv = __frcp_rn(s);
+  Packed16 p{0u, 0u};
+  if (isinf(rinv)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t sign = (__float_as_uint(v[i]) >> 31) << 3;
+      if (i < 8) p.lo |= sign << (4 * i);
+      else p.hi |= sign << (4 * (i - 8));
+    }
+    return p;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // elements 2j, 2j+1 share word (j & 3) of draw (j >> 2): low / high half
+    const uint32_t w = words[((j >> 2) << 2) | (j & 3)];
+    const float q0 = e2m1_sr_value(__fmul_rn(v[2 * j], rinv), w & 0xFFFFu);
+    const float q1 = e2m1_sr_value(__fmul_rn(v[2 * j + 1], rinv), w >> 16);
+    const uint32_t b = e2m1x2_rne(q0, q1);
+    if (j < 4) p.lo |= b << (8 * j);
+    else p.hi |= b << (8 * (j - 4));
+  }
+  return p;
+}
+
+// Signed grid values of the 16 codes.
+__device__ __forceinline__ void decode16(const Packed16& p, float* q) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t b = ((j < 4) ? (p.lo >> (8 * j)) : (p.hi >> (8 * (j - 4)))) & 0xFFu;
+    e2m1x2_values(b, q[2 * j], q[2 * j + 1]);
+  }
+}
+
+// Squared error of an encoding in the original domain, summed with sum16:
+// e_i = (v_i - q_i s)^2.
+__device__ __forceinline__ float sq_error(const float* v, float alpha, uint32_t sb,
+                                          const Packed16& p) {
+  const float s = __fmul_rn(alpha, e4m3_value(sb));
+  float q[16], e[16];
+  decode16(p, q);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float d = __fsub_rn(v[i], __fmul_rn(q[i], s));
+    e[i] = __fmul_rn(d, d);
+  }
+  return sum16(e);
+}
+
+// Unsigned division by a runtime constant d >= 1 for n < 2^32:
+// q = (n * mul) >> (32 + shift), mul = ceil(2^(32+shift) / d) (33 bits),
+// shift = ceil(log2 d).  The rounding error of mul is below d <= 2^shift, so
+// the quotient is exact for every 32-bit n.
+struct FastDiv {
+  uint32_t d, shift;
+  uint64_t mul;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  f.shift = s;
+  f.mul = ((1ull << (32 + s)) + d - 1) / d;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+  // n * mul < 2^32 * 2^33 would overflow 64 bits only if mul >= 2^32 and n is
+  // large; split mul into its high bit and low word.
+  const uint64_t lo = static_cast<uint64_t>(n) * static_cast<uint32_t>(f.mul);
+  const uint64_t hi = (f.mul >> 32) ? static_cast<uint64_t>(n) : 0ull;  // n * 2^32 / 2^32
+  // (n * mul) >> 32 = hi + (lo >> 32)
+  const uint64_t t = hi + (lo >> 32);
+  return static_cast<uint32_t>(t >> f.shift);
+}
+
+}  // namespace nvfp4

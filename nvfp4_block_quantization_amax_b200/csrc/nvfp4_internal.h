@@ -1,0 +1,56 @@
+// nvfp4_internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+constexpr int kModeRTN = NVFP4_RTN;
+constexpr int kModeFourSix = NVFP4_FOUR_SIX;
+constexpr int kModeRhtSR = NVFP4_RHT_SR;
+constexpr int kModeMsEden = NVFP4_MS_EDEN;
+
+constexpr uint32_t kRowwise = NVFP4_ROWWISE;
+constexpr uint32_t kColwise = NVFP4_COLWISE;
+constexpr uint32_t kBlock2D = NVFP4_BLOCK2D;
+constexpr uint32_t kSinglePass = NVFP4_SINGLE_PASS;
+constexpr uint32_t kAlphaProvided = NVFP4_ALPHA_PROVIDED;
+constexpr uint32_t kGemmScaleLayout = NVFP4_GEMM_SCALE_LAYOUT;
+constexpr uint32_t kRht = NVFP4_RHT;
+constexpr uint32_t kInverseRht = NVFP4_INVERSE_RHT;
+constexpr uint32_t kOutBf16 = NVFP4_OUT_BF16;
+
+constexpr int32_t kStatusArg = NVFP4_ERR_ARG;
+constexpr int32_t kStatusNonFinite = NVFP4_ERR_NONFINITE;
+constexpr int32_t kStatusTimeout = NVFP4_ERR_TIMEOUT;
+
+struct QuantOutputs {
+  uint8_t* codes_row;
+  uint8_t* scales_row;
+  float* alpha_row;
+  uint8_t* codes_col;
+  uint8_t* scales_col;
+  float* alpha_col;
+  float* amax_out;
+  int32_t* status;
+};
+
+int sm_count();
+size_t quant_workspace_bytes(int64_t R, int64_t C, uint32_t flags);
+
+cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int mode,
+                            uint32_t flags, uint64_t seed, uint32_t stream_id,
+                            const float* alpha_in, const QuantOutputs& out, void* workspace,
+                            cudaStream_t st);
+
+cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* scales, const float* alpha,
+                              int64_t R, int64_t C, uint32_t flags, uint64_t seed, void* y,
+                              cudaStream_t st);
+
+cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                        const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K,
+                        void* D, int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st);
+
+}  // namespace nvfp4

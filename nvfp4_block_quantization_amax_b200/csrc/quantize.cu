@@ -1,0 +1,638 @@
+// quantize.cu -- NVFP4 quantization kernels for sm_100a.
+//
+// Two-pass path (Four Over Six §2.1 Eq. 1 needs the tensor amax before any
+// block can be scaled; the NVFP4 pretraining write-up §九 notes this extra
+// pass over memory):
+//   1. an amax kernel reads the bf16 tensor once and leaves one partial
+//      maximum per CTA in the workspace (no atomics, no zero-fill needed);
+//   2. a quantize kernel reduces those partials to amax and alpha in its
+//      prologue, then encodes every block.
+// Rowwise-only work streams straight from HBM into registers (128-bit loads,
+// one 16-element block per thread).  Column, dual (row + column from one
+// read) and 2D 16x16 work stage a 64 x 128 tile in shared memory with
+// cp.async, so that both orientations are read conflict-free and the
+// transposed outputs are written in full 32-byte sectors.
+#include <cuda_runtime.h>
+#include <algorithm>
+#include <cstdint>
+
+#include "nvfp4_device.cuh"
+#include "nvfp4_internal.h"
+
+namespace nvfp4 {
+
+// ---------------------------------------------------------------------------
+// Shared parameter block of the quantize kernels.
+// ---------------------------------------------------------------------------
+struct QuantArgs {
+  const uint16_t* x;
+  int64_t R, C, ld;
+  uint64_t seed;
+  uint32_t stream_id;
+  uint32_t flags;
+  const float* alpha_in;          // device, used with NVFP4_ALPHA_PROVIDED
+  const uint32_t* partials;       // row-orientation maxima (float bits), one per amax CTA
+  const uint32_t* partials_col;   // column-orientation maxima (== partials when not rotated)
+  int npart;
+  uint8_t* codes_row;
+  uint8_t* scales_row;
+  float* alpha_row;
+  uint8_t* codes_col;
+  uint8_t* scales_col;
+  float* alpha_col;
+  float* amax_out;
+  int32_t* status;
+  FastDiv nb_row;                 // C / 16
+  int64_t tiles_r, tiles_c;       // tile grid (tile kernels)
+};
+
+constexpr uint32_t kNonFinite = 0xFFFFFFFFu;   // partial marker: a NaN / Inf was read
+
+__device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+// Block-wide max of a uint32 (all threads get the result).
+template <int NT>
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < NT / 32) ? red[l] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// Reduce the amax partials of one orientation (all threads of the CTA).
+template <int NT>
+__device__ __forceinline__ uint32_t reduce_partials(const uint32_t* p, int n, uint32_t* red) {
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < n; i += NT) m = max(m, __ldcg(p + i));
+  return block_max_u32<NT>(m, red);
+}
+
+// Tensor scales of both orientations from the partials (or the caller's
+// alpha).  need_* select what is computed, pub_* what is published; CTA 0
+// publishes alpha, amax and a device-side error.
+template <int NT>
+__device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, bool need_c,
+                                              bool pub_r, bool pub_c, float& alpha_r,
+                                              float& alpha_c, uint32_t* red) {
+  if (a.flags & kAlphaProvided) {
+    const float al = __ldg(a.alpha_in);
+    alpha_r = alpha_c = al;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      if (!(al >= 0.0f && al <= 3.402823466e38f) && a.status) *a.status = kStatusArg;
+      if (pub_r && a.alpha_row) *a.alpha_row = al;
+      if (pub_c && a.alpha_col) *a.alpha_col = al;
+    }
+    return;
+  }
+  uint32_t mr = 0, mc = 0;
+  if (need_r) mr = reduce_partials<NT>(a.partials, a.npart, red);
+  if (need_c) mc = reduce_partials<NT>(a.partials_col, a.npart, red);
+  // Eq. 1: alpha = amax / (6 * 448)
+  const float amax_r = __uint_as_float(mr == kNonFinite ? 0u : mr);
+  const float amax_c = __uint_as_float(mc == kNonFinite ? 0u : mc);
+  alpha_r = __fdiv_rn(amax_r, 2688.0f);
+  alpha_c = __fdiv_rn(amax_c, 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if ((mr == kNonFinite || mc == kNonFinite) && a.status) *a.status = kStatusNonFinite;
+    if (pub_r && a.alpha_row) *a.alpha_row = alpha_r;
+    if (pub_c && a.alpha_col) *a.alpha_col = alpha_c;
+    if (a.amax_out) {
+      if (pub_r) a.amax_out[0] = amax_r;
+      if (pub_c) a.amax_out[1] = amax_c;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t sign_bits(const PhiloxKeys& K) {
+  return philox(K, 0u, 0u, 0u, kTagSigns).x & 0xFFFFu;
+}
+
+// Byte offset of the scale of (row m, K-block j) in the tcgen05 block-scale
+// layout: 512-byte atoms of 128 rows x 4 K-blocks, K-atoms fastest; inside an
+// atom, row m % 32 selects a 16-byte line and (m / 32) % 4 a 4-byte word.
+__device__ __forceinline__ int64_t gemm_scale_offset(int64_t m, int64_t j, int64_t kblocks) {
+  return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
+}
+
+// ---------------------------------------------------------------------------
+// One 16-element block in a mode.  v holds the (rotated) values; the block's
+// random streams are keyed by (seed, c2 = 2 stream_id + orientation, blk).
+// ---------------------------------------------------------------------------
+template <int MODE>
+__device__ __forceinline__ Packed16 quantize_block(const float* v, float alpha,
+                                                   const PhiloxKeys& K, uint32_t c2,
+                                                   uint64_t blk, uint32_t& sb) {
+  const float amax_b = max_abs16(v);
+  if constexpr (MODE == kModeRTN) {
+    sb = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
+    return encode_rne(v, alpha, sb);
+  } else if constexpr (MODE == kModeFourSix) {
+    const uint32_t sb6 = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
+    const uint32_t sb4 = e4m3_rne(scale_raw(amax_b, alpha, 4.0f));
+    const Packed16 p6 = encode_rne(v, alpha, sb6);
+    const Packed16 p4 = encode_rne(v, alpha, sb4);
+    const float e6 = sq_error(v, alpha, sb6, p6);
+    const float e4 = sq_error(v, alpha, sb4, p4);
+    const bool take4 = e4 < e6;
+    sb = take4 ? sb4 : sb6;
+    return take4 ? p4 : p6;
+  } else if constexpr (MODE == kModeRhtSR) {
+    sb = e4m3_ceil(scale_raw(amax_b, alpha, 6.0f));
+    const uint64_t u0 = 2 * blk, u1 = 2 * blk + 1;
+    const uint4 w0 = philox(K, static_cast<uint32_t>(u0), static_cast<uint32_t>(u0 >> 32), c2, kTagValueSR);
+    const uint4 w1 = philox(K, static_cast<uint32_t>(u1), static_cast<uint32_t>(u1 >> 32), c2, kTagValueSR);
+    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    return encode_sr(v, alpha, sb, words);
+  } else {  // MS-EDEN
+    const uint32_t prov = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
+    const Packed16 p = encode_rne(v, alpha, prov);
+    float q[16], rr[16], rq[16];
+    decode16(p, q);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      rr[i] = __fmul_rn(v[i], v[i]);
+      rq[i] = __fmul_rn(v[i], q[i]);
+    }
+    const float num = sum16(rr);
+    const float den = __fmul_rn(alpha, sum16(rq));
+    if (den == 0.0f) {
+      sb = 0u;
+    } else {
+      const float dstar = __fdiv_rn(num, den);
+      const uint64_t unit = blk >> 2;
+      const uint4 w = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
+      const uint32_t sel = static_cast<uint32_t>(blk & 3);
+      const uint32_t word = sel == 0 ? w.x : (sel == 1 ? w.y : (sel == 2 ? w.z : w.w));
+      sb = e4m3_sr(dstar, word >> 8);
+    }
+    return p;
+  }
+}
+
+// ===========================================================================
+// amax kernels
+// ===========================================================================
+// Rows of 16-blocks, streamed: max |x| (or max |rotated block|).  Also the
+// plain amax for any orientation.  One partial per CTA.
+template <bool ROT, int NT>
+__global__ void __launch_bounds__(NT) amax_rows_kernel(const uint16_t* __restrict__ x, int64_t R,
+                                                       int64_t ld, FastDiv nb, uint64_t seed,
+                                                       uint32_t* __restrict__ partial) {
+  __shared__ uint32_t red[NT / 32];
+  uint32_t signs = 0;
+  if constexpr (ROT) signs = sign_bits(philox_keys(seed));
+  const uint32_t total = static_cast<uint32_t>(R) * nb.d;
+  uint32_t m = 0;
+  bool bad = false;
+  for (uint32_t k = blockIdx.x * NT + threadIdx.x; k < total; k += gridDim.x * NT) {
+    const uint32_t r = fastdiv(k, nb), cb = k - r * nb.d;
+    const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld + 16 * cb);
+    const uint4 a = __ldcs(p), b = __ldcs(p + 1);
+    float v[16];
+    unpack8(a, v);
+    unpack8(b, v + 8);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) bad |= abs_bits(v[i]) >= 0x7F800000u;
+    if constexpr (ROT) rht16(v, signs);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = max(m, abs_bits(v[i]));
+  }
+  if (bad) m = kNonFinite;
+  m = block_max_u32<NT>(m, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+}
+
+// Column-rotated amax: 16-row stripes; each thread owns two adjacent columns
+// of a stripe, so a warp reads 128 contiguous bytes per row.
+template <int NT>
+__global__ void __launch_bounds__(NT) amax_cols_kernel(const uint16_t* __restrict__ x, int64_t R,
+                                                       int64_t C, int64_t ld, uint64_t seed,
+                                                       uint32_t* __restrict__ partial) {
+  __shared__ uint32_t red[NT / 32];
+  const uint32_t signs = sign_bits(philox_keys(seed));
+  const int64_t pairs = C / 2, stripes = R / 16;
+  const int64_t total = pairs * stripes;
+  uint32_t m = 0;
+  bool bad = false;
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x; k < total;
+       k += static_cast<int64_t>(gridDim.x) * NT) {
+    const int64_t st = k / pairs, pr = k - st * pairs;
+    const uint32_t* base = reinterpret_cast<const uint32_t*>(x + 16 * st * ld) + pr;
+    float c0[16], c1[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t w = __ldcs(base + i * (ld / 2));
+      c0[i] = bf16lo(w);
+      c1[i] = bf16hi(w);
+      bad |= abs_bits(c0[i]) >= 0x7F800000u || abs_bits(c1[i]) >= 0x7F800000u;
+    }
+    rht16(c0, signs);
+    rht16(c1, signs);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = max(m, max(abs_bits(c0[i]), abs_bits(c1[i])));
+  }
+  if (bad) m = kNonFinite;
+  m = block_max_u32<NT>(m, red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+}
+
+// ===========================================================================
+// Rowwise quantization, streamed: one thread per 16-element block.
+// ===========================================================================
+template <int MODE, bool ROT, int NT>
+__global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
+  __shared__ uint32_t red[NT / 32];
+  float alpha, alpha_unused;
+  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red);
+  const PhiloxKeys K = philox_keys(a.seed);
+  uint32_t signs = 0;
+  if constexpr (ROT) signs = sign_bits(K);
+  const uint32_t c2 = a.stream_id * 2u;
+  const uint32_t nb = a.nb_row.d;
+  const uint32_t total = static_cast<uint32_t>(a.R) * nb;
+  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
+  const bool check = (a.flags & kAlphaProvided) != 0;
+  for (uint32_t k = blockIdx.x * NT + threadIdx.x; k < total; k += gridDim.x * NT) {
+    const uint32_t r = fastdiv(k, a.nb_row), cb = k - r * nb;
+    const uint4* p = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(r) * a.ld + 16 * cb);
+    const uint4 u0 = __ldcs(p), u1 = __ldcs(p + 1);
+    float v[16];
+    unpack8(u0, v);
+    unpack8(u1, v + 8);
+    if (check) {
+      bool bad = false;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) bad |= abs_bits(v[i]) >= 0x7F800000u;
+      if (bad && a.status) *a.status = kStatusNonFinite;
+    }
+    if constexpr (ROT) rht16(v, signs);
+    uint32_t sb;
+    const Packed16 q = quantize_block<MODE>(v, alpha, K, c2, k, sb);
+    *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(r) * (a.C / 2) + 8 * cb) =
+        make_uint2(q.lo, q.hi);
+    if (a.scales_row) {
+      const int64_t off = gemm ? gemm_scale_offset(r, cb, nb) : static_cast<int64_t>(k);
+      a.scales_row[off] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
+// ===========================================================================
+// Tiled quantization: columns, dual rows + columns, and 2D 16x16 blocks.
+// Tile: 64 rows x 128 columns of bf16 (16 KB) in shared memory.
+// ===========================================================================
+constexpr int TR = 64, TC = 128, TNT = 256;
+constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
+
+struct TileSmem {
+  uint4 tile[TR][TC / 8];                   // 64 x 256 B
+  uint8_t colcodes[TC][kColPitch];          // transposed codes, 32 B per column
+  uint8_t colscale[TC][TR / 16];            // column scales of the tile
+  uint8_t scale2d[TR / 16][TC / 16];        // chosen 2D scales
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// 16 bf16 of row `row`, column block `cb` of the smem tile, read as two
+// 16-byte halves in a lane-dependent order so eight lanes hit eight distinct
+// bank groups.
+__device__ __forceinline__ void tile_row_block(const TileSmem& s, int row, int cb, float* v) {
+  const int first = (cb >> 2) & 1;
+  const uint4 h0 = s.tile[row][2 * cb + first];
+  const uint4 h1 = s.tile[row][2 * cb + (first ^ 1)];
+  if (first) {
+    unpack8(h1, v);
+    unpack8(h0, v + 8);
+  } else {
+    unpack8(h0, v);
+    unpack8(h1, v + 8);
+  }
+}
+
+template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
+__global__ void __launch_bounds__(TNT) quant_tile_kernel(const QuantArgs a) {
+  __shared__ TileSmem s;
+  __shared__ uint32_t red[TNT / 32];
+  float alpha_r, alpha_c;
+  // 2D tiles share one tensor scale (the plain amax, which both orientations
+  // read from the same partials) between orientations.
+  resolve_alpha<TNT>(a, ROW || TWO_D, COL, ROW, COL, alpha_r, alpha_c, red);
+  if constexpr (TWO_D) alpha_c = alpha_r;
+  const PhiloxKeys K = philox_keys(a.seed);
+  uint32_t signs = 0;
+  if constexpr (ROT) signs = sign_bits(K);
+  const uint32_t c2r = a.stream_id * 2u, c2c = a.stream_id * 2u + 1u;
+  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
+  const bool check = (a.flags & kAlphaProvided) != 0;
+  const int t = threadIdx.x;
+  const int64_t R = a.R, C = a.C;
+  const int64_t ntiles = a.tiles_r * a.tiles_c;
+
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);   // multiple of 16
+    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);   // multiple of 16
+
+    // ---- load the tile (16-byte async copies, 4 per thread) ----
+    __syncthreads();  // previous tile fully consumed
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int ch = t + TNT * i;
+      const int row = ch >> 4, cc = ch & 15;
+      if (row < rows && 8 * cc < cols)
+        cp_async16(&s.tile[row][cc], a.x + (r0 + row) * a.ld + c0 + 8 * cc);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    if (check) {
+      bool bad = false;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ch = t + TNT * i;
+        const int row = ch >> 4, cc = ch & 15;
+        if (row < rows && 8 * cc < cols) {
+          float v[8];
+          unpack8(s.tile[row][cc], v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) bad |= abs_bits(v[j]) >= 0x7F800000u;
+        }
+      }
+      if (bad && a.status) *a.status = kStatusNonFinite;
+    }
+
+    if constexpr (TWO_D) {
+      // ---- 2D blocks: 16 lanes per 16x16 block, one row each ----
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int task = t + TNT * i;
+        const int bb = task >> 4, lr = task & 15;
+        const int rb = bb >> 3, cbb = bb & 7;
+        const bool valid = (16 * rb < rows) && (16 * cbb < cols);  // uniform per half-warp
+        float v[16];
+        if (valid) tile_row_block(s, 16 * rb + lr, cbb, v);
+        else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        }
+        float m = max_abs16(v);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        const uint32_t sb6 = e4m3_rne(scale_raw(m, alpha_r, 6.0f));
+        Packed16 p = encode_rne(v, alpha_r, sb6);
+        uint32_t sb = sb6;
+        if constexpr (MODE == kModeFourSix) {
+          const uint32_t sb4 = e4m3_rne(scale_raw(m, alpha_r, 4.0f));
+          const Packed16 p4 = encode_rne(v, alpha_r, sb4);
+          float e6 = sq_error(v, alpha_r, sb6, p);
+          float e4 = sq_error(v, alpha_r, sb4, p4);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) {
+            e6 = __fadd_rn(e6, __shfl_xor_sync(0xFFFFFFFFu, e6, o));
+            e4 = __fadd_rn(e4, __shfl_xor_sync(0xFFFFFFFFu, e4, o));
+          }
+          if (e4 < e6) {
+            sb = sb4;
+            p = p4;
+          }
+        }
+        if (valid) {
+          const int64_t grow = r0 + 16 * rb + lr;
+          const int64_t gcb = c0 / 16 + cbb;
+          if (lr == 0) s.scale2d[rb][cbb] = static_cast<uint8_t>(sb);
+          if constexpr (ROW) {
+            *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(p.lo, p.hi);
+            if (a.scales_row) {
+              if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sb);
+              else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sb);
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
+
+    if constexpr (ROW && !TWO_D) {
+      // ---- row blocks: 64 rows x 8 blocks, two per thread ----
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int task = t + TNT * i;
+        const int row = task >> 3, cb = task & 7;
+        if (row < rows && 16 * cb < cols) {
+          float v[16];
+          tile_row_block(s, row, cb, v);
+          if constexpr (ROT) rht16(v, signs);
+          const int64_t grow = r0 + row, gcb = c0 / 16 + cb;
+          const uint64_t blk = static_cast<uint64_t>(grow) * (C / 16) + gcb;
+          uint32_t sb;
+          const Packed16 q = quantize_block<MODE>(v, alpha_r, K, c2r, blk, sb);
+          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(q.lo, q.hi);
+          if (a.scales_row)
+            a.scales_row[gemm ? gemm_scale_offset(grow, gcb, C / 16) : static_cast<int64_t>(blk)] =
+                static_cast<uint8_t>(sb);
+        }
+      }
+    }
+
+    if constexpr (COL) {
+      // ---- column blocks: 4 row-blocks x 128 columns; a thread owns a
+      //      column pair of one row-block ----
+      const int cp = t & 63, rb = t >> 6;
+      if (16 * rb < rows && 2 * cp < cols) {
+        float v0[16], v1[16];
+        const uint32_t* base = reinterpret_cast<const uint32_t*>(&s.tile[16 * rb][0]) + cp;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = base[i * (TC / 2)];
+          v0[i] = bf16lo(w);
+          v1[i] = bf16hi(w);
+        }
+        uint32_t sb0, sb1;
+        Packed16 q0, q1;
+        if constexpr (TWO_D) {
+          sb0 = sb1 = s.scale2d[rb][cp >> 3];
+          q0 = encode_rne(v0, alpha_c, sb0);
+          q1 = encode_rne(v1, alpha_c, sb1);
+        } else {
+          if constexpr (ROT) {
+            rht16(v0, signs);
+            rht16(v1, signs);
+          }
+          const int64_t nbc = R / 16;
+          const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
+          q0 = quantize_block<MODE>(v0, alpha_c, K, c2c, static_cast<uint64_t>(gc) * nbc + grb, sb0);
+          q1 = quantize_block<MODE>(v1, alpha_c, K, c2c, static_cast<uint64_t>(gc + 1) * nbc + grb, sb1);
+        }
+        *reinterpret_cast<uint2*>(&s.colcodes[2 * cp][8 * rb]) = make_uint2(q0.lo, q0.hi);
+        *reinterpret_cast<uint2*>(&s.colcodes[2 * cp + 1][8 * rb]) = make_uint2(q1.lo, q1.hi);
+        s.colscale[2 * cp][rb] = static_cast<uint8_t>(sb0);
+        s.colscale[2 * cp + 1][rb] = static_cast<uint8_t>(sb1);
+      }
+      __syncthreads();
+      // ---- write the transposed codes: column c of the tile is 32 bytes
+      //      (rows/2 valid) of output row c0 + c ----
+      {
+        const int c = t >> 1, h = t & 1;
+        const int nbytes = rows / 2;
+        if (c < cols && 16 * h < nbytes) {
+          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
+          const uint2* src = reinterpret_cast<const uint2*>(&s.colcodes[c][16 * h]);
+          const uint2 lo = src[0];
+          reinterpret_cast<uint2*>(dst)[0] = lo;
+          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+        }
+      }
+      if (a.scales_col) {
+        const int c = t >> 1;
+        if (c < cols) {
+          for (int rb = (t & 1); rb < rows / 16; rb += 2) {
+            const int64_t gc = c0 + c, grb = r0 / 16 + rb;
+            const uint8_t sb = s.colscale[c][rb];
+            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sb;
+            else if (TWO_D) {
+              if ((c & 15) == 0) a.scales_col[(gc / 16) * (R / 16) + grb] = sb;
+            } else {
+              a.scales_col[gc * (R / 16) + grb] = sb;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// ===========================================================================
+// Host-side launchers
+// ===========================================================================
+static int g_sm_count[64] = {0};
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+int amax_partial_count() { return 4 * 148; }
+
+size_t quant_workspace_bytes(int64_t, int64_t, uint32_t flags) {
+  if (flags & kAlphaProvided) return 0;
+  return static_cast<size_t>(2 * amax_partial_count()) * sizeof(uint32_t);
+}
+
+template <int MODE, bool ROT>
+static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
+  const uint32_t total = static_cast<uint32_t>(a.R) * a.nb_row.d;
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
+  quant_rows_kernel<MODE, ROT, 256><<<std::max(blocks, 1), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
+static cudaError_t launch_tile(const QuantArgs& a, cudaStream_t st) {
+  const int64_t ntiles = a.tiles_r * a.tiles_c;
+  const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 6));
+  quant_tile_kernel<MODE, ROT, ROW, COL, TWO_D><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int MODE, bool ROT>
+static cudaError_t dispatch_1d(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
+  if (row && !col) return launch_rows<MODE, ROT>(a, st);
+  if (row && col) return launch_tile<MODE, ROT, true, true, false>(a, st);
+  return launch_tile<MODE, ROT, false, true, false>(a, st);
+}
+
+// Launch the amax pass: rows into partials[0, npart), columns (rotated
+// only) into partials[npart, 2 npart).  Plain amax is shared by both
+// orientations.
+static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot, cudaStream_t st) {
+  const int np = a.npart;
+  uint32_t* pr = const_cast<uint32_t*>(a.partials);
+  uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
+  if (!rot) {
+    amax_rows_kernel<false, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr);
+    return cudaGetLastError();
+  }
+  if (row) amax_rows_kernel<true, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr);
+  if (col) amax_cols_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.C, a.ld, a.seed, pc);
+  return cudaGetLastError();
+}
+
+cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int mode, uint32_t flags,
+                            uint64_t seed, uint32_t stream_id, const float* alpha_in,
+                            const QuantOutputs& o, void* workspace, cudaStream_t st) {
+  QuantArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.R = R;
+  a.C = C;
+  a.ld = ld;
+  a.seed = seed;
+  a.stream_id = stream_id;
+  a.flags = flags;
+  a.alpha_in = alpha_in;
+  a.npart = amax_partial_count();
+  a.partials = static_cast<const uint32_t*>(workspace);
+  a.partials_col = a.partials;
+  a.codes_row = o.codes_row;
+  a.scales_row = o.scales_row;
+  a.alpha_row = o.alpha_row;
+  a.codes_col = o.codes_col;
+  a.scales_col = o.scales_col;
+  a.alpha_col = o.alpha_col;
+  a.amax_out = o.amax_out;
+  a.status = o.status;
+  a.nb_row = make_fastdiv(static_cast<uint32_t>(C / 16));
+  a.tiles_r = (R + TR - 1) / TR;
+  a.tiles_c = (C + TC - 1) / TC;
+  const bool row = flags & kRowwise, col = flags & kColwise, two_d = flags & kBlock2D;
+  const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || (flags & kRht)) && !two_d;
+  if (rot) a.partials_col = a.partials + a.npart;
+  if (R == 0 || C == 0) return cudaSuccess;
+
+  if (!(flags & kAlphaProvided)) {
+    cudaError_t e = launch_amax(a, row || two_d, col && !two_d, rot, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (two_d) {
+    if (mode == kModeRTN) {
+      if (row && col) return launch_tile<kModeRTN, false, true, true, true>(a, st);
+      if (row) return launch_tile<kModeRTN, false, true, false, true>(a, st);
+      return launch_tile<kModeRTN, false, false, true, true>(a, st);
+    }
+    if (row && col) return launch_tile<kModeFourSix, false, true, true, true>(a, st);
+    if (row) return launch_tile<kModeFourSix, false, true, false, true>(a, st);
+    return launch_tile<kModeFourSix, false, false, true, true>(a, st);
+  }
+  switch (mode) {
+    case kModeRTN:
+      return rot ? dispatch_1d<kModeRTN, true>(a, row, col, st) : dispatch_1d<kModeRTN, false>(a, row, col, st);
+    case kModeFourSix:
+      return rot ? dispatch_1d<kModeFourSix, true>(a, row, col, st)
+                 : dispatch_1d<kModeFourSix, false>(a, row, col, st);
+    case kModeRhtSR:
+      return dispatch_1d<kModeRhtSR, true>(a, row, col, st);
+    default:
+      return dispatch_1d<kModeMsEden, true>(a, row, col, st);
+  }
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,80 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/nvfp4.h declares; host-side argument checks run without a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_block_quantization_amax_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_workspace_size",
+            "nvfp4_status_string", "nvfp4_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_binding_names_match_header():
+    from nvfp4_block_quantization_amax_b200 import _lib
+    for name in declared_functions():
+        assert hasattr(_lib, name), name
+    assert set(_lib.EXPORTED) == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    from nvfp4_block_quantization_amax_b200 import _lib
+    assert _lib.nvfp4_status_string(0) == "ok"
+    assert "NaN" in _lib.nvfp4_status_string(-4)
+    assert _lib.nvfp4_version() >= 10000
+
+
+def test_host_argument_checks_need_no_gpu(lib):
+    from nvfp4_block_quantization_amax_b200 import _lib as L
+    out = L.nvfp4_qtensor_t()
+    fake = 0x10000  # never dereferenced: every call below fails its checks first
+    # bad mode, bad flags, no orientation
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 7, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, 0x8000, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, 0, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_ARG
+    # missing outputs
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_ARG
+    out = L.nvfp4_qtensor_t(fake, fake, fake, fake, fake, fake, None, None)
+    # C not a multiple of 16; R not a multiple of 16 for columns
+    assert L.nvfp4_quantize(fake, 16, 24, 24, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_quantize(fake, 20, 32, 32, 0, L.NVFP4_COLWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_SHAPE
+    # 2D blocks only for RTN / FOUR_SIX
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 2, L.NVFP4_ROWWISE | L.NVFP4_BLOCK2D, 0, 0, None, out, None, 0,
+                            None) == L.NVFP4_ERR_ARG
+    # misaligned input, then missing workspace
+    assert L.nvfp4_quantize(fake + 2, 16, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_ALIGN
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_WORKSPACE
+    assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE) > 0
+    assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE | L.NVFP4_ALPHA_PROVIDED) == 0
+    # empty tensors are a no-op
+    assert L.nvfp4_quantize(None, 0, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_OK
+    # dequantize / gemm checks
+    assert L.nvfp4_dequantize(fake, fake, fake, 16, 24, 0, 0, fake, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_dequantize(fake, fake, fake, 16, 16, 0x8000, 0, fake, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_gemm(fake, fake, fake, fake, fake, fake, 100, 128, 128, fake, 0, 128, None, 0, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_gemm(fake, fake, fake, fake, fake, fake, 128, 128, 128, fake, 5, 128, None, 0, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_gemm(None, fake, fake, fake, fake, fake, 128, 128, 128, fake, 0, 128, None, 0, None) == L.NVFP4_ERR_ARG
