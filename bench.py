@@ -1,0 +1,526 @@
+"""Benchmark of the NVFP4 hot path: one linear layer's forward + backward
+step at the 8B-shaped workload, every quantization and all three GEMMs on the
+device through the C ABI.
+
+A step (one batch, one rank):
+  1. X  [8192, 4096]  -> Four Over Six, 1D row blocks          (fprop A)
+  2. W  [14336, 4096] -> Four Over Six, 16x16 2D blocks        (fprop B)
+  3. fprop  Y  = X W^T            8192 x 14336, K = 4096, bf16 out
+  4. dY [8192, 14336] -> MS-EDEN (or RHT+SR), rows and columns (dgrad A, wgrad A)
+  5. W  -> rotated RTN along the output features (columns)     (dgrad B)
+  6. dgrad  dX = dY W             8192 x 4096,  K = 14336
+  7. X  -> rotated RTN along the tokens (columns)              (wgrad B)
+  8. wgrad  dW = dY^T X           14336 x 4096, K = 8192
+The rotated operands of a backward GEMM share one seed, so the Hadamard
+rotations cancel in the product.
+
+`value` = the three GEMMs' algorithmic FLOPs / device time of the whole step
+(quantization included), summed over ranks (weak scaling: every rank runs its
+own batch; no data-path collective).  Rank 0 prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--bwd-mode eden|sr]
+  python bench.py --impl reference ...   # the CPU oracle, bounded sample
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 quantize Gelem/s & % HBM roofline; NVFP4 GEMM TFLOPS & % FP4 peak"
+TOKENS, HIDDEN, OUT = 8192, 4096, 14336
+WORKLOAD = ("linear fwd+bwd, 8B-shaped: X 8192x4096 (4/6 1D), W 14336x4096 (4/6 2D), "
+            "dY 8192x14336 (MS-EDEN rows+cols), fprop/dgrad/wgrad NVFP4 GEMMs, bf16 out")
+FP4_PER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+ROW, COL, B2D, RHT, GEMM = 0x1, 0x2, 0x4, 0x40, 0x20
+RTN, FOUR_SIX, RHT_SR, MS_EDEN = 0, 1, 2, 3
+
+
+def gemm_flops():
+    return 2.0 * TOKENS * OUT * HIDDEN * 3
+
+
+# (name, elements, algorithmic bytes per element) of the step's quantize calls
+def quant_calls():
+    return [("X 4/6 rows", TOKENS * HIDDEN, 2 + 0.5 + 1 / 16),
+            ("W 4/6 2D", OUT * HIDDEN, 2 + 0.5 + 1 / 16),
+            ("dY rows+cols", TOKENS * OUT, 2 + 2 * (0.5 + 1 / 16)),
+            ("W rotated cols", OUT * HIDDEN, 2 + 0.5 + 1 / 16),
+            ("X rotated cols", TOKENS * HIDDEN, 2 + 0.5 + 1 / 16)]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; CPU tests drive it with gloo)
+# --------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x, device=None):
+    """Max of a host float over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, device=None):
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[4:8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, _, r in rows for n, v in zip(names, r) if v.lower().startswith("active")})
+        loaded = [c for c, _, _ in rows if c > 0.5 * rows[0][1]] or [c for c, _, _ in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": rows[0][1], "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# the step
+# --------------------------------------------------------------------------
+class LayerStep:
+    """Pre-allocated buffers and the C-ABI call sequence of one step."""
+
+    def __init__(self, x, w, dy, bwd_mode, device):
+        import torch
+        from nvfp4_block_quantization_amax_b200 import api
+        self.api = api
+        self.x, self.w, self.dy = x, w, dy
+        self.bwd = bwd_mode
+        T, H = x.shape
+        O = w.shape[0]
+        self.plan = [  # (tensor, mode, flags)
+            ("x", FOUR_SIX, ROW | GEMM),
+            ("w", FOUR_SIX, ROW | B2D | GEMM),
+            ("dy", bwd_mode, ROW | COL | GEMM),
+            ("w_rot", RTN, COL | RHT | GEMM),
+            ("x_rot", RTN, COL | RHT | GEMM),
+        ]
+        src = {"x": x, "w": w, "dy": dy, "w_rot": w, "x_rot": x}
+        self.src = src
+        self.out = {}
+        self.ws = {}
+        for name, mode, flags in self.plan:
+            t = src[name]
+            self.out[name] = api.alloc_outputs(t.shape[0], t.shape[1], flags, device)
+            self.ws[name] = api.workspace_for(t.shape[0], t.shape[1], flags, device)
+        self.y = torch.empty((T, O), dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        self.dw = torch.empty((O, H), dtype=torch.bfloat16, device=device)
+        self.ev = None
+
+    def quantize(self, name, mode, flags, seed, sid):
+        self.api.nvfp4_quantize(self.src[name], mode, flags, seed=seed, stream_id=sid, out=self.out[name],
+                                workspace=self.ws[name])
+
+    def run(self, step, timers=None):
+        """One step.  timers: dict name -> list of (start, end) CUDA events."""
+        api = self.api
+        seed = 1000 * (step + 1)   # a new rotation and noise per step
+        mark = (lambda k: _Mark(timers, k)) if timers is not None else (lambda k: _NoMark())
+        with mark("quantize"):
+            self.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0)
+            self.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1)
+        qx, qw = self.out["x"], self.out["w"]
+        with mark("gemm"):
+            api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row, qw.scales_row, qw.alpha_row,
+                           out=self.y)
+        with mark("quantize"):
+            self.quantize("dy", self.bwd, ROW | COL | GEMM, seed, 0)
+            self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1)
+        qd, qwr = self.out["dy"], self.out["w_rot"]
+        with mark("gemm"):
+            api.nvfp4_gemm(qd.codes_row, qd.scales_row, qd.alpha_row, qwr.codes_col, qwr.scales_col,
+                           qwr.alpha_col, out=self.dx)
+        with mark("quantize"):
+            self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2)
+        qxr = self.out["x_rot"]
+        with mark("gemm"):
+            api.nvfp4_gemm(qd.codes_col, qd.scales_col, qd.alpha_col, qxr.codes_col, qxr.scales_col,
+                           qxr.alpha_col, out=self.dw)
+
+
+class _NoMark:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+class _Mark:
+    def __init__(self, timers, key):
+        self.timers, self.key = timers, key
+
+    def __enter__(self):
+        import torch
+        self.s = torch.cuda.Event(enable_timing=True)
+        self.s.record()
+        return self
+
+    def __exit__(self, *a):
+        import torch
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.timers.setdefault(self.key, []).append((self.s, e))
+        return False
+
+
+def gemm_traffic_record():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = os.path.join(ROOT, "nvfp4_block_quantization_amax_b200", "csrc", "gemm.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    g = d.get("gemm", {})
+    return g.get("dram_bytes_per_launch") if g.get("source_sha256_16") == h else None
+
+
+def run_device(args, rank, world, local_rank):
+    import torch
+    from nvfp4_block_quantization_amax_b200 import _lib, synthetic
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    _lib.load()
+    layer = synthetic.fwd_bwd_8b(seed=17 * rank)
+    x, w, dy = (layer[k].to(device) for k in ("x", "w", "dy"))
+    bwd = MS_EDEN if args.bwd_mode == "eden" else RHT_SR
+    step = LayerStep(x, w, dy, bwd, device)
+
+    # --- device-resident timing ---
+    for i in range(args.warmup):
+        step.run(i)
+    torch.cuda.synchronize()
+    barrier(device)
+    timers = {}
+    launches0 = _lib.nvfp4_launch_count()
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize()
+        barrier(device)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record()
+        for i in range(args.steps):
+            step.run(args.warmup + i, timers)
+        end.record()
+        torch.cuda.synchronize()
+        barrier(device)
+    launches = _lib.nvfp4_launch_count() - launches0
+    ms_local = start.elapsed_time(end) / args.steps
+    clocks = clk.summary()
+    ms = max_over_ranks(ms_local, device)
+    gemm_ms = sum(s.elapsed_time(e) for s, e in timers["gemm"]) / (3 * args.steps)
+    quant_ms = sum(s.elapsed_time(e) for s, e in timers["quantize"]) / args.steps
+
+    # --- end to end: pinned host inputs in, results back to pinned host ---
+    hx, hw, hdy = (t.cpu().pin_memory() for t in (x, w, dy))
+    hy = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
+    hdx = torch.empty(step.dx.shape, dtype=torch.bfloat16).pin_memory()
+    hdw = torch.empty(step.dw.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_once(i):
+        x.copy_(hx, non_blocking=True)
+        w.copy_(hw, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        step.run(i)
+        hy.copy_(step.y, non_blocking=True)
+        hdx.copy_(step.dx, non_blocking=True)
+        hdw.copy_(step.dw, non_blocking=True)
+
+    e2e_once(0)
+    torch.cuda.synchronize()
+    barrier(device)
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for i in range(e2e_steps):
+        e2e_once(i)
+    e2.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2) / e2e_steps, device)
+    barrier(device)
+
+    total_flops = sum_over_ranks(gemm_flops(), device)
+    peaks, src = load_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    gemm_tflops = 2.0 * TOKENS * OUT * HIDDEN / (gemm_ms * 1e-3) / 1e12
+    q_elems = sum(n for _, n, _ in quant_calls())
+    q_bytes = sum(n * b for _, n, b in quant_calls())
+    q_gelem = q_elems / (quant_ms * 1e-3) / 1e9
+    q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
+    traffic = gemm_traffic_record()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
+    result = {
+        "metric": METRIC,
+        "value": total_flops / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1 x e2m1 -> f32 (GEMM), f32 (quantizer)",
+        "data": "synthetic (seeded; shapes and distributions of the pages' 8B workload)",
+        "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN, "out_features": OUT,
+                   "bwd_mode": args.bwd_mode, "parallelism": f"replicas x{world} (weak)",
+                   "l2": "inputs larger than L2: 419 MB of bf16 per step"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+                     "kernel": "nvfp4_gemm_kernel (avg of fprop, dgrad, wgrad)",
+                     "peak_source": f"{src} bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)"},
+        "quantize": {"gelem_s": q_gelem, "alg_gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
+                     "ms_per_step": quant_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
+                     "note": "algorithmic bytes: bf16 read once + codes + scales per orientation"},
+        "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak, "ms_per_gemm": gemm_ms},
+        "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    return result
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle on a bounded sample of the same step
+# --------------------------------------------------------------------------
+def oracle_sample(budget_rows=64, gemm_rows=16, gemm_cols=16, bwd_mode="eden"):
+    """Time the oracle on a sample of every part of the step and extrapolate
+    to one full step.  Returns (step_seconds_extrapolated, sample description,
+    threads)."""
+    import numpy as np
+    import oracle
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    rng = np.random.default_rng(0)
+    xb = synthetic.bf16_bits(synthetic.normal_with_channel_outliers(budget_rows * 16, HIDDEN, seed=0))
+    wb = synthetic.bf16_bits(synthetic.weight(budget_rows * 16, HIDDEN, seed=1))
+    dyb = synthetic.bf16_bits(synthetic.laplace_with_spikes(budget_rows * 16, OUT, seed=2))
+    bwd = MS_EDEN if bwd_mode == "eden" else RHT_SR
+    t_total = 0.0
+    parts = []
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        r = fn()
+        return time.perf_counter() - t0, r
+
+    # quantize parts: sample tensors of (budget_rows*16) rows, scaled by rows
+    for name, bits, mode, flags, full_rows in [
+            ("X 4/6 rows", xb, FOUR_SIX, ROW, TOKENS), ("W 4/6 2D", wb, FOUR_SIX, ROW | B2D, OUT),
+            ("dY rows+cols", dyb, bwd, ROW | COL, TOKENS), ("W rot cols", wb, RTN, COL | RHT, OUT),
+            ("X rot cols", xb, RTN, COL | RHT, TOKENS)]:
+        dt, _ = timed(lambda: oracle.quantize(bits, mode, flags, seed=1))
+        scale = full_rows / bits.shape[0]
+        t_total += dt * scale
+        parts.append(f"{name}: {bits.shape[0]}x{bits.shape[1]}")
+    # GEMM parts: FP64 reference on gemm_rows x gemm_cols outputs at full K
+    for (M, N, K) in [(TOKENS, OUT, HIDDEN), (TOKENS, HIDDEN, OUT), (OUT, HIDDEN, TOKENS)]:
+        A = rng.integers(0, 256, (gemm_rows, K // 2), dtype=np.uint8)
+        B = rng.integers(0, 256, (gemm_cols, K // 2), dtype=np.uint8)
+        sA = rng.integers(0x28, 0x48, (gemm_rows, K // 16), dtype=np.uint8)
+        sB = rng.integers(0x28, 0x48, (gemm_cols, K // 16), dtype=np.uint8)
+        dt, _ = timed(lambda: oracle.gemm_f64(A, sA, 1.0, B, sB, 1.0, gemm_rows, gemm_cols, K))
+        t_total += dt * (M * N) / (gemm_rows * gemm_cols)
+        parts.append(f"GEMM {gemm_rows}x{gemm_cols} of {M}x{N}, K={K}")
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = ("oracle timed on " + "; ".join(parts) + "; each part scaled to the full step by its element count")
+    return t_total, desc, threads
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    t_step = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        dt, desc, threads = oracle_sample(bwd_mode=args.bwd_mode)
+        if i >= args.warmup:
+            t_step.append(dt)
+    s = statistics.mean(t_step)
+    v = gemm_flops() / s / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer, f64 GEMM (CPU oracle)",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "bwd_mode": args.bwd_mode},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline_line(bwd_mode):
+    dt, desc, threads = oracle_sample(bwd_mode=bwd_mode)
+    return {"value": gemm_flops() / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": desc, "step_seconds_extrapolated": dt}
+
+
+KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_w_rot",
+                "quant_x_rot")
+
+
+def run_kernel_case(name, iters=3):
+    """Run one C-ABI call of the step a few times on its full-size inputs
+    (the small, single-kernel command that profiler captures use)."""
+    import torch
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    layer = synthetic.fwd_bwd_8b(seed=0)
+    x, w, dy = (layer[k].to(device) for k in ("x", "w", "dy"))
+    step = LayerStep(x, w, dy, MS_EDEN, device)
+    step.run(0)  # produce every operand once
+    torch.cuda.synchronize()
+    api = step.api
+    qx, qw, qd, qwr, qxr = (step.out[k] for k in ("x", "w", "dy", "w_rot", "x_rot"))
+    calls = {
+        "gemm_fprop": lambda: api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row,
+                                             qw.scales_row, qw.alpha_row, out=step.y),
+        "gemm_dgrad": lambda: api.nvfp4_gemm(qd.codes_row, qd.scales_row, qd.alpha_row, qwr.codes_col,
+                                             qwr.scales_col, qwr.alpha_col, out=step.dx),
+        "gemm_wgrad": lambda: api.nvfp4_gemm(qd.codes_col, qd.scales_col, qd.alpha_col, qxr.codes_col,
+                                             qxr.scales_col, qxr.alpha_col, out=step.dw),
+        "quant_x": lambda: step.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0),
+        "quant_w2d": lambda: step.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1),
+        "quant_dy": lambda: step.quantize("dy", MS_EDEN, ROW | COL | GEMM, 7, 0),
+        "quant_w_rot": lambda: step.quantize("w_rot", RTN, COL | RHT | GEMM, 7, 1),
+        "quant_x_rot": lambda: step.quantize("x_rot", RTN, COL | RHT | GEMM, 7, 2),
+    }
+    for _ in range(iters):
+        calls[name]()
+    torch.cuda.synchronize()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--bwd-mode", choices=["eden", "sr"], default="eden")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=KERNEL_CASES,
+                    help="run one call of the step a few times and exit (for profiler captures)")
+    args = ap.parse_args(argv)
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case)
+        return 0
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        r = run_reference(args)
+        if r is not None:
+            print(json.dumps(r), flush=True)
+        return 0
+    rank, world, local_rank = dist_env()
+    init_dist("nccl" if world > 1 else "gloo")
+    res = run_device(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_line(args.bwd_mode)
+        print(json.dumps(res), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

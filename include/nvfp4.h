@@ -189,6 +189,11 @@ NVFP4_API nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const f
                           int64_t ldd, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Number of kernels this library has launched in the calling process since
+ * it was loaded (all devices, all streams).  Instrumentation for callers that
+ * account for their launches; not a page-defined operation. */
+NVFP4_API uint64_t nvfp4_launch_count(void);
+
 /* Static description of a status code. */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status_t status);
 

@@ -30,7 +30,7 @@ NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
 EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm",
-            "nvfp4_status_string", "nvfp4_version")
+            "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
 
 
 class nvfp4_qtensor_t(ctypes.Structure):
@@ -66,6 +66,8 @@ def load(path=LIB_PATH):
     L.nvfp4_status_string.restype = ctypes.c_char_p
     L.nvfp4_version.argtypes = []
     L.nvfp4_version.restype = ctypes.c_int
+    L.nvfp4_launch_count.argtypes = []
+    L.nvfp4_launch_count.restype = ctypes.c_uint64
     _lib = L
     return L
 
@@ -92,6 +94,10 @@ def nvfp4_gemm(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, workspa
 
 def nvfp4_status_string(status):
     return load().nvfp4_status_string(status).decode()
+
+
+def nvfp4_launch_count():
+    return int(load().nvfp4_launch_count())
 
 
 def nvfp4_version():

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libnvfp4.so: argument checks, workspace sizing and
 // dispatch.  Host-detectable errors return before anything is launched.
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "nvfp4.h"
@@ -23,9 +24,17 @@ nvfp4_status_t launch_status(cudaError_t e) {
              : NVFP4_ERR_CUDA;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
 }  // namespace
 
+namespace nvfp4 {
+void note_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+}  // namespace nvfp4
+
 extern "C" {
+
+uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int nvfp4_version(void) { return 10000; }
 

@@ -64,9 +64,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 template <bool INV, bool BF16>
 static void launch_dq(int sc, dim3 g, const uint8_t* codes, const uint8_t* scales, const float* alpha,
                       int64_t R, int64_t C, FastDiv nb, uint64_t seed, void* y, cudaStream_t st) {
-  if (sc == 0) dequant_kernel<INV, BF16, 0><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y);
-  else if (sc == 1) dequant_kernel<INV, BF16, 1><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y);
-  else dequant_kernel<INV, BF16, 2><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y);
+  if (sc == 0) { dequant_kernel<INV, BF16, 0><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
+  else if (sc == 1) { dequant_kernel<INV, BF16, 1><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
+  else { dequant_kernel<INV, BF16, 2><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
 }
 
 cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* scales, const float* alpha,

@@ -360,6 +360,7 @@ cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, con
                                                             static_cast<int>(M), static_cast<int>(N),
                                                             static_cast<int>(K), out_dtype == NVFP4_OUT_DTYPE_FP32,
                                                             status);
+  note_launch();
   return cudaGetLastError();
 }
 

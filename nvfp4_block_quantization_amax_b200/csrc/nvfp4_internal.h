@@ -38,6 +38,7 @@ struct QuantOutputs {
 };
 
 int sm_count();
+void note_launch(int n = 1);  // count kernels launched by the library
 size_t quant_workspace_bytes(int64_t R, int64_t C, uint32_t flags);
 
 cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int mode,

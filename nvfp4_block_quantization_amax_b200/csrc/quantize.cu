@@ -543,6 +543,7 @@ static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
   const uint32_t total = static_cast<uint32_t>(a.R) * a.nb_row.d;
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
   quant_rows_kernel<MODE, ROT, 256><<<std::max(blocks, 1), 256, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -551,6 +552,7 @@ static cudaError_t launch_tile(const QuantArgs& a, cudaStream_t st) {
   const int64_t ntiles = a.tiles_r * a.tiles_c;
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 6));
   quant_tile_kernel<MODE, ROT, ROW, COL, TWO_D><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -570,10 +572,11 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
   if (!rot) {
     amax_rows_kernel<false, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr);
+    note_launch();
     return cudaGetLastError();
   }
-  if (row) amax_rows_kernel<true, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr);
-  if (col) amax_cols_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.C, a.ld, a.seed, pc);
+  if (row) { amax_rows_kernel<true, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr); note_launch(); }
+  if (col) { amax_cols_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.C, a.ld, a.seed, pc); note_launch(); }
   return cudaGetLastError();
 }
 

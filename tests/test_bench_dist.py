@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py's multi-rank path, on CPU with gloo
+(world size 2): max / sum over ranks, rank-0-only reference arm, and the
+command-line contract."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w = bench.init_dist("gloo")
+    bench.barrier()
+    mx = bench.max_over_ranks(1.5 + rank)
+    sm = bench.sum_over_ranks(10.0 * (rank + 1))
+    ref = bench.run_reference(type("A", (), {"warmup": 0, "steps": 0, "bwd_mode": "eden"})()) if rank else None
+    q.put((rank, r, w, mx, sm, ref))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(i, 2, port, q)) for i in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, r, w, mx, sm, ref in out:
+        assert (r, w) == (rank, 2)
+        assert mx == 2.5          # max over ranks of 1.5 + rank
+        assert sm == 30.0         # 10 + 20
+        if rank == 1:
+            assert ref is None    # the reference arm runs on rank 0 only
+
+
+def test_single_rank_reductions_are_identity():
+    assert bench.max_over_ranks(3.25) == 3.25
+    assert bench.sum_over_ranks(2.0) == 2.0
+
+
+def test_cli_rejects_short_warmup():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
+
+
+def test_step_accounting():
+    flops = bench.gemm_flops()
+    assert flops == 3 * 2 * 8192 * 14336 * 4096
+    calls = bench.quant_calls()
+    assert [n for _, n, _ in calls] == [8192 * 4096, 14336 * 4096, 8192 * 14336, 14336 * 4096, 8192 * 4096]
