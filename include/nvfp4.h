@@ -161,6 +161,24 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int
                               const nvfp4_qtensor_t* out, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* nvfp4_quantize for callers that may not allocate device memory while they
+ * run (no page defines this; it has no counterpart in the method): a plugin
+ * inside another runtime that owns all device memory, or a program whose
+ * memory plan is fixed at start-up.  Same arguments and results as
+ * nvfp4_quantize, minus the workspace: the scratch of the amax pass lives in
+ * an 8192-byte array compiled into the library, which every GPU that loads
+ * the library holds until the process exits.  A call that would need more
+ * scratch than that returns NVFP4_ERR_WORKSPACE.  The first call on each
+ * device (with that device current) looks up the array's device address;
+ * make it before any stream capture starts.  All calls on a device share the
+ * array, so calls whose kernels may overlap on the GPU race and can give wrong
+ * results: order them on one stream.  Nothing in the array must start at
+ * zero.  The function itself allocates nothing. */
+NVFP4_API nvfp4_status_t nvfp4_quantize_noalloc(const void* x, int64_t R, int64_t C, int64_t ld,
+                                                nvfp4_mode_t mode, uint32_t flags, uint64_t seed,
+                                                uint32_t stream_id, const float* alpha_in,
+                                                const nvfp4_qtensor_t* out, void* stream);
+
 /* Decode packed codes [R, C/2] with scales ([R, C/16]; BLOCK2D [R/16, C/16];
  * or the GEMM layout with NVFP4_GEMM_SCALE_LAYOUT) and the device tensor
  * scale *alpha:  y = q * (alpha * Delta)  (the inverse of Eq. 3), optionally

@@ -29,8 +29,8 @@ NVFP4_OUT_BF16 = 0x100
 NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
-EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm",
-            "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
+EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
+            "nvfp4_gemm", "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
 
 
 class nvfp4_qtensor_t(ctypes.Structure):
@@ -58,6 +58,9 @@ def load(path=LIB_PATH):
     L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, ctypes.c_int, u32, u64, u32, vp,
                                  ctypes.POINTER(nvfp4_qtensor_t), vp, sz, vp]
     L.nvfp4_quantize.restype = ctypes.c_int
+    L.nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, i64, ctypes.c_int, u32, u64, u32, vp,
+                                         ctypes.POINTER(nvfp4_qtensor_t), vp]
+    L.nvfp4_quantize_noalloc.restype = ctypes.c_int
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, u32, u64, vp, vp]
     L.nvfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
@@ -80,6 +83,15 @@ def nvfp4_quantize(x, R, C, ld, mode, flags, seed, stream_id, alpha_in, out, wor
                    workspace_bytes, stream):
     return int(load().nvfp4_quantize(x, R, C, ld, mode, flags, seed, stream_id, alpha_in,
                                      ctypes.byref(out), workspace, workspace_bytes, stream))
+
+
+def nvfp4_quantize_noalloc(x, R, C, ld, mode, flags, seed, stream_id, alpha_in, out, stream):
+    """nvfp4_quantize without a workspace, for callers that may not allocate
+    device memory while they run; its scratch is a fixed array inside the
+    library shared by every call on a device (order such calls on one
+    stream)."""
+    return int(load().nvfp4_quantize_noalloc(x, R, C, ld, mode, flags, seed, stream_id, alpha_in,
+                                             ctypes.byref(out), stream))
 
 
 def nvfp4_dequantize(codes, scales, alpha, R, C, flags, seed, y, stream):
