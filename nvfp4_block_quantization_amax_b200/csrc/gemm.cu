@@ -15,8 +15,13 @@
 //     tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128, N=BN, K=64),
 //     accumulating in TMEM, then commits the stage back to the producer.
 //   * warps 2-5: epilogue.  Each reads its 32-lane quarter of the FP32
-//     accumulator with tcgen05.ld, multiplies by alphaA * alphaB, converts to
-//     bf16 (or keeps fp32) and stores.
+//     accumulator with tcgen05.ld, multiplies by alphaA * alphaB and converts
+//     to bf16 into registers (the whole row), hands the accumulator back, then
+//     writes 16-row x 128-byte boxes into swizzled shared memory and stores
+//     them with TMA.
+// The kernel is persistent (one CTA per SM, tiles round-robin): the producer
+// runs ahead into the next tile while the epilogue drains the accumulator,
+// and the MMA warp starts the next tile as soon as the accumulator is read.
 // Every wait is bounded (about two seconds of %globaltimer); a wait that
 // gives up raises an abort flag that every role checks, the kernel records
 // NVFP4_ERR_TIMEOUT in the optional status word and still frees its TMEM.
@@ -33,8 +38,10 @@ namespace nvfp4 {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK_BYTES = 128;  // 256 FP4 values per row per stage
-constexpr int STAGES = 4;
+constexpr int BK_BYTES = 128;  // 256 FP4 values per row per stage: four MMA K blocks
+constexpr int KB_PER_STAGE = 4;
+constexpr int kOutStaging = 4 * 2048;  // epilogue: one 16-row x 128-byte box per warp
+constexpr int kSfSlots = 2 * KB_PER_STAGE;  // TMEM scale slots: two sets of one stage's K blocks
 constexpr int NUM_THREADS = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
@@ -42,13 +49,18 @@ template <int BN>
 struct Cfg {
   static constexpr int A_STAGE = BM * BK_BYTES;
   static constexpr int B_STAGE = BN * BK_BYTES;
-  static constexpr int SFA_STAGE = 4 * 512;
-  static constexpr int SFB_STAGE = (BN / 128) * 4 * 512;
+  static constexpr int SFA_STAGE = KB_PER_STAGE * 512;
+  static constexpr int SFB_STAGE = (BN / 128) * KB_PER_STAGE * 512;
   static constexpr int STAGE = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
-  static constexpr int SMEM = STAGES * STAGE + 1024 /* alignment */ + 256 /* barriers */;
-  static constexpr uint32_t TMEM_COLS = (BN + 16 + 4 * 4 * (BN / 128)) <= 256 ? 256 : 512;
-  static constexpr uint32_t SFA_COL = BN;            // 4 columns per MMA k-block
-  static constexpr uint32_t SFB_COL = BN + 16;       // 4 * (BN/128) columns per MMA k-block
+  // as many stages as fit: loads take about a microsecond to land, so the
+  // ring must hold that much MMA work
+  static constexpr int STAGES = (232448 - kOutStaging - 1024 - 512) / STAGE;
+  static constexpr int SMEM = STAGES * STAGE + kOutStaging + 1024 /* alignment */ + 512 /* barriers */;
+  // Scales of one 64-wide K block in TMEM: SFA 4 columns, then SFB
+  // 4 * (BN / 128) columns.
+  static constexpr uint32_t SF_W = 4 + 4 * (BN / 128);
+  static constexpr uint32_t TMEM_COLS = (BN + kSfSlots * SF_W) <= 256 ? 256 : 512;
+  static constexpr uint32_t SF_COL = BN;
   // Instruction descriptor (kind::mxf4nvf4): A and B are E2M1 (format 1),
   // K-major, scales E4M3, N >> 3 at bit 17, M >> 4 at bit 24.
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BM) >> 4) << 24);
@@ -114,7 +126,8 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 
 // Shared-memory matrix descriptor, K-major operand with 128-byte swizzle:
 // start >> 4, leading offset 1 (unused when swizzled), stride 1024 B between
-// 8-row groups, descriptor version 1, layout SWIZZLE_128B (2) in bits 61-63.
+// 8-row groups (8 rows x 128 B), descriptor version 1, layout SWIZZLE_128B
+// (2) in bits 61-63.
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
   return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (1ull << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) |
          (1ull << 46) | (2ull << 61);
@@ -147,8 +160,9 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 lanes x 32 columns of 32-bit accumulators: thread t gets lane t's row.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+// 32 lanes x 32 columns of 32-bit accumulators: thread t gets lane t's row
+// (the caller waits with tmem_ld_wait before using r).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -157,34 +171,120 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// TMA tile store from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+
+// ---- cluster / CTA-pair helpers (2-SM MMA) ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// an mbarrier that may live in the peer CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t accumulate, uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Arrive on the mbarrier at this shared-memory offset in both CTAs of the pair
+// once every tcgen05 operation issued so far has completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
 }
 
 template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
-                      const float* __restrict__ alpha_a, const float* __restrict__ alpha_b, void* __restrict__ d,
-                      int64_t ldd, int M, int N, int K, int out_fp32, int32_t* status) {
+                      const __grid_constant__ CUtensorMap tmap_d, const uint8_t* __restrict__ sfa,
+                      const uint8_t* __restrict__ sfb, const float* __restrict__ alpha_a,
+                      const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status) {
   using G = Cfg<BN>;
+  constexpr int STAGES = G::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * G::A_STAGE;
   uint8_t* sSFA = sB + STAGES * G::B_STAGE;
   uint8_t* sSFB = sSFA + STAGES * G::SFA_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + STAGES * G::SFB_STAGE);
+  uint8_t* sOut = sSFB + STAGES * G::SFB_STAGE;  // 4 warps x one 2 KB box, 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kOutStaging);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  uint64_t* acc_empty = bars + 2 * STAGES + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = M / BM;
-  const int tile_m = blockIdx.x % m_tiles, tile_n = blockIdx.x / m_tiles;
-  const int kblocks64 = K / 64;           // scale atoms along K
-  const int kstages = (K + 255) / 256;
+  const int num_tiles = m_tiles * (N / BN);
+  const int kblocks64 = K / 64;  // scale atoms along K
+  const int kstages = (K + 255) / 256;  // K % 128 == 0: the last stage may hold 2 K blocks
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -192,6 +292,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_empty), 4);  // one arrival per epilogue warp
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -208,31 +309,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- producer ----------------
-      int issued = 0;
-      for (int kt = 0; kt < kstages; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = (kt / STAGES) & 1;
-        if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) break;
-        ++issued;
-        const int nk = min(4, kblocks64 - 4 * kt);  // 64-wide K blocks in this stage
-        const uint32_t bytes = G::A_STAGE + G::B_STAGE + nk * 512 * (1 + BN / 128);
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_expect_tx(fb, bytes);
-        tma_load_2d(smem_u32(sA + s * G::A_STAGE), &tmap_a, kt * BK_BYTES, tile_m * BM, fb);
-        tma_load_2d(smem_u32(sB + s * G::B_STAGE), &tmap_b, kt * BK_BYTES, tile_n * BN, fb);
-        bulk_load(smem_u32(sSFA + s * G::SFA_STAGE),
-                  sfa + (static_cast<int64_t>(tile_m) * kblocks64 + 4 * kt) * 512, nk * 512, fb);
+      // ---------------- producer: runs ahead across tiles ----------------
+      int it = 0;  // global stage counter
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+        const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+        for (int kt = 0; kt < kstages; ++kt, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);  // K blocks in this stage
+          const uint32_t bytes = G::A_STAGE + G::B_STAGE + nk * 512 * (1 + BN / 128);
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_expect_tx(fb, bytes);
+          tma_load_2d(smem_u32(sA + s * G::A_STAGE), &tmap_a, kt * BK_BYTES, tile_m * BM, fb);
+          tma_load_2d(smem_u32(sB + s * G::B_STAGE), &tmap_b, kt * BK_BYTES, tile_n * BN, fb);
+          bulk_load(smem_u32(sSFA + s * G::SFA_STAGE),
+                    sfa + (static_cast<int64_t>(tile_m) * kblocks64 + KB_PER_STAGE * kt) * 512, nk * 512, fb);
 #pragma unroll
-        for (int g = 0; g < BN / 128; ++g)
-          bulk_load(smem_u32(sSFB + s * G::SFB_STAGE + g * 2048),
-                    sfb + (static_cast<int64_t>(tile_n * (BN / 128) + g) * kblocks64 + 4 * kt) * 512, nk * 512, fb);
+          for (int g = 0; g < BN / 128; ++g)
+            bulk_load(smem_u32(sSFB + s * G::SFB_STAGE + g * KB_PER_STAGE * 512),
+                      sfb + (static_cast<int64_t>(tile_n * (BN / 128) + g) * kblocks64 + KB_PER_STAGE * kt) * 512,
+                      nk * 512, fb);
+        }
       }
       if (*abort_flag) {
         // A wait gave up somewhere: let the copies this thread issued land
         // before the CTA exits (each wait again bounded).
-        for (int kt = (issued > STAGES ? issued - STAGES : 0); kt < issued; ++kt) {
-          const uint32_t bar = smem_u32(&full[kt % STAGES]), ph = (kt / STAGES) & 1;
+        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i) {
+          const uint32_t bar = smem_u32(&full[i % STAGES]), ph = (i / STAGES) & 1;
           const uint64_t t0 = globaltimer();
           while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
           }
@@ -242,65 +350,138 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      for (int kt = 0; kt < kstages; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = (kt / STAGES) & 1;
-        if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) break;
+      // Per stage: wait for its data, copy its scales (one TMEM slot per K
+      // block, two slot sets used alternately so the copies never overwrite
+      // scales an earlier, still-running MMA reads), issue its MMAs, release
+      // the stage.  No wait on later stages sits between a stage's MMAs and
+      // its release.
+      const int my_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                           static_cast<int>(gridDim.x);
+      const int total = my_tiles * kstages;
+      for (int g = 0; g < total; ++g) {
+        const int kt = g % kstages, ti = g / kstages, s = g % STAGES;
+        if (kt == 0) {
+          // the epilogue must have drained the previous tile's accumulator
+          if (!mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag)) break;
+          fence_after();
+        }
+        if (!mbar_wait(smem_u32(&full[s]), (g / STAGES) & 1, abort_flag)) break;
         fence_after();
-        const int nk = min(4, kblocks64 - 4 * kt);
         const uint32_t sfa_s = smem_u32(sSFA + s * G::SFA_STAGE);
         const uint32_t sfb_s = smem_u32(sSFB + s * G::SFB_STAGE);
+        const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
+        const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
         for (int kk = 0; kk < nk; ++kk) {
-          tmem_cp_sf(tmem + G::SFA_COL + 4 * kk, desc_sf(sfa_s + 512 * kk));
+          const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
+          tmem_cp_sf(col, desc_sf(sfa_s + 512 * kk));
 #pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-            tmem_cp_sf(tmem + G::SFB_COL + 4 * (BN / 128) * kk + 4 * g, desc_sf(sfb_s + g * 2048 + 512 * kk));
+          for (int gg = 0; gg < BN / 128; ++gg)
+            tmem_cp_sf(col + 4 + 4 * gg, desc_sf(sfb_s + gg * KB_PER_STAGE * 512 + 512 * kk));
         }
         const uint64_t adesc = desc_sw128(smem_u32(sA + s * G::A_STAGE));
         const uint64_t bdesc = desc_sw128(smem_u32(sB + s * G::B_STAGE));
         for (int kk = 0; kk < nk; ++kk) {
+          const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
           // K = 64 FP4 values = 32 bytes: advance the start address by 2 x 16 B
-          mma_mxf4nvf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, G::IDESC, (kt > 0 || kk > 0) ? 1u : 0u,
-                       tmem + G::SFA_COL + 4 * kk, tmem + G::SFB_COL + 4 * (BN / 128) * kk);
+          mma_mxf4nvf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, G::IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col, col + 4);
         }
         umma_commit(smem_u32(&empty[s]));
+        if (kt == kstages - 1) umma_commit(smem_u32(acc_full));
       }
-      umma_commit(smem_u32(acc_full));
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const bool ok = mbar_wait(smem_u32(acc_full), 0, abort_flag);
-    fence_after();
-    if (ok && !*abort_flag) {
-      const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
-      const int64_t row = static_cast<int64_t>(tile_m) * BM + 32 * q + lane;
-      const int64_t col0 = static_cast<int64_t>(tile_n) * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c, r);
-        if (out_fp32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(d) + row * ldd + col0 + c);
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31 = output rows of the tile.
+    // bf16: the whole 256-column row goes to registers as packed bf16 first,
+    // so the accumulator is handed back to the MMA warp before any store;
+    // then 16-row x 128-byte boxes go out through one swizzled staging
+    // buffer per warp with TMA stores.
+    const int q = warp & 3;
+    uint8_t* buf = sOut + (warp - 2) * 2048;
+    const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
+    int ti = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+      if (!mbar_wait(smem_u32(acc_full), ti & 1, abort_flag)) break;
+      fence_after();
+      const int row0 = tile_m * BM + 32 * q;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      if (!out_fp32) {
+        uint32_t packed[BN / 2];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), ab), __fmul_rn(__uint_as_float(r[4 * j + 1]), ab),
-                                 __fmul_rn(__uint_as_float(r[4 * j + 2]), ab),
-                                 __fmul_rn(__uint_as_float(r[4 * j + 3]), ab));
-        } else {
-          uint32_t w[16];
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_nowait(taddr + c, r);
+          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), ab),
-                                                           __fmul_rn(__uint_as_float(r[2 * j + 1]), ab));
-            w[j] = *reinterpret_cast<const uint32_t*>(&h);
+          for (int h = 0; h < 16; ++h) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * h]), ab),
+                                                            __fmul_rn(__uint_as_float(r[2 * h + 1]), ab));
+            packed[c / 2 + h] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(acc_empty));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        for (int p = 0; p < BN / 64; ++p) {      // 64-column pieces
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {  // rows 0-15, 16-31 of the warp
+            if (lane == 0) bulk_wait_read<0>();  // the previous box has been read
+            __syncwarp();
+            if ((lane >> 4) == half) {
+              uint8_t* rowp = buf + (lane & 15) * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(packed[32 * p + 4 * j], packed[32 * p + 4 * j + 1], packed[32 * p + 4 * j + 2],
+                               packed[32 * p + 4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * BN + 64 * p, row0 + 16 * half);
+              bulk_commit();
+            }
+          }
+        }
+      } else {
+        // fp32: 32-column pieces straight from TMEM
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_nowait(taddr + c, r);
+          tmem_ld_wait();
+          if (c + 32 == BN) {
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            if ((lane >> 4) == half) {
+              uint8_t* rowp = buf + (lane & 15) * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(__float_as_uint(__fmul_rn(__uint_as_float(r[4 * j]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 1]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 2]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 3]), ab)));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * BN + c, row0 + 16 * half);
+              bulk_commit();
+            }
+          }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   fence_before();
   __syncthreads();
@@ -308,6 +489,257 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(G::TMEM_COLS) : "memory");
+  }
+}
+
+// ===========================================================================
+// 2-SM variant: a CTA pair (cluster of 2) computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64).  Each CTA loads its own
+// 128 rows of A and its own 128 rows of B, so per SM the operand traffic per
+// FLOP is 2/3 of the single-CTA 128 x 256 tile; each CTA holds its 128 rows x
+// 256 columns of the accumulator.  Scales: each CTA loads the scales of its A
+// rows and of all 256 B rows (the MMA reads them from its own TMEM).
+// Protocol (same shared-memory offsets in both CTAs):
+//   full[s]    -- in the leader (rank 0) only: the leader's producer arms it
+//                 with both CTAs' bytes; both CTAs' loads complete on it.
+//   empty[s]   -- in both: the leader's MMA commit arrives on both.
+//   acc_full   -- in both: the leader's commit at the end of a tile.
+//   acc_empty  -- in the leader: 4 epilogue warps of each CTA arrive.
+// ===========================================================================
+constexpr int P_STAGE_A = 128 * BK_BYTES;        // own A rows
+constexpr int P_STAGE_B = 128 * BK_BYTES;        // own B rows
+constexpr int P_STAGE_SFA = KB_PER_STAGE * 512;  // own A rows' scales
+constexpr int P_STAGE_SFB = 2 * KB_PER_STAGE * 512;  // all 256 B rows' scales
+constexpr int P_STAGE = P_STAGE_A + P_STAGE_B + P_STAGE_SFA + P_STAGE_SFB;
+constexpr int P_STAGES = (232448 - kOutStaging - 1024 - 512) / P_STAGE;
+constexpr int P_SMEM = P_STAGES * P_STAGE + kOutStaging + 1024 + 512;
+constexpr uint32_t P_SF_W = 4 + 8;               // SFA 4 + SFB (256 rows) 8 columns per K block
+constexpr uint32_t P_SF_COL = 256;
+constexpr uint32_t P_TMEM_COLS = 512;            // 256 accumulator + 2 x 4 K blocks x 12 scale columns
+// M = 256 (>> 4 = 16 at bit 24), N = 256 (>> 3 = 32 at bit 17), E2M1 x E2M1, E4M3 scales
+constexpr uint32_t P_IDESC = (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                           const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
+                           const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
+                           const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + P_STAGES * P_STAGE_A;
+  uint8_t* sSFA = sB + P_STAGES * P_STAGE_B;
+  uint8_t* sSFB = sSFA + P_STAGES * P_STAGE_SFA;
+  uint8_t* sOut = sSFB + P_STAGES * P_STAGE_SFB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kOutStaging);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + P_STAGES;
+  uint64_t* acc_full = bars + 2 * P_STAGES;
+  uint64_t* acc_empty = bars + 2 * P_STAGES + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P_STAGES + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x) >> 1, num_pairs = static_cast<int>(gridDim.x) >> 1;
+  const int m_tiles = M / 256;
+  const int num_tiles = m_tiles * (N / 256);
+  const int kblocks64 = K / 64;
+  const int kstages = (K + 255) / 256;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_empty), 8);  // 4 epilogue warps in each CTA
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(P_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncwarp();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer (both CTAs) ----------------
+      int it = 0;
+      bool stop = false;
+      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
+        const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+        for (int kt = 0; kt < kstages; ++kt, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          const uint32_t fb_leader = map_to_rank(smem_u32(&full[s]), 0);
+          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * P_STAGE);
+          tma_load_2d_pair(smem_u32(sA + s * P_STAGE_A), &tmap_a, kt * BK_BYTES, tile_m * 256 + 128 * rank,
+                           fb_leader);
+          tma_load_2d_pair(smem_u32(sB + s * P_STAGE_B), &tmap_b, kt * BK_BYTES, tile_n * 256 + 128 * rank,
+                           fb_leader);
+          // scale atoms viewed as rows of 256 bytes: a stage is 8 rows per 128 operand rows
+          tma_load_2d_pair(smem_u32(sSFA + s * P_STAGE_SFA), &tmap_sfa, 0,
+                           ((tile_m * 2 + static_cast<int>(rank)) * kblocks64 + KB_PER_STAGE * kt) * 2, fb_leader);
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+            tma_load_2d_pair(smem_u32(sSFB + s * P_STAGE_SFB + g * P_STAGE_SFA), &tmap_sfb, 0,
+                             ((tile_n * 2 + g) * kblocks64 + KB_PER_STAGE * kt) * 2, fb_leader);
+        }
+      }
+      if (*abort_flag && leader) {
+        for (int i = (it > P_STAGES ? it - P_STAGES : 0); i < it; ++i) {
+          const uint32_t bar = smem_u32(&full[i % P_STAGES]), ph = (i / P_STAGES) & 1;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      // ---------------- MMA issuer (leader only) ----------------
+      const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
+      const int total = my_tiles * kstages;
+      for (int g = 0; g < total; ++g) {
+        const int kt = g % kstages, ti = g / kstages, s = g % P_STAGES;
+        if (kt == 0) {
+          if (!mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag)) break;
+          fence_after();
+        }
+        if (!mbar_wait(smem_u32(&full[s]), (g / P_STAGES) & 1, abort_flag)) break;
+        fence_after();
+        const uint32_t sfa_s = smem_u32(sSFA + s * P_STAGE_SFA);
+        const uint32_t sfb_s = smem_u32(sSFB + s * P_STAGE_SFB);
+        const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
+        const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
+          tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * kk));
+          tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * kk));
+          tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + P_STAGE_SFA + 512 * kk));
+        }
+        const uint64_t adesc = desc_sw128(smem_u32(sA + s * P_STAGE_A));
+        const uint64_t bdesc = desc_sw128(smem_u32(sB + s * P_STAGE_B));
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
+          mma_mxf4nvf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col,
+                            col + 4);
+        }
+        umma_commit_pair(smem_u32(&empty[s]));
+        if (kt == kstages - 1) umma_commit_pair(smem_u32(acc_full));
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int q = warp & 3;
+    uint8_t* buf = sOut + (warp - 2) * 2048;
+    const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
+    const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+    int ti = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++ti) {
+      const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+      if (!mbar_wait(smem_u32(acc_full), ti & 1, abort_flag)) break;
+      fence_after();
+      const int row0 = tile_m * 256 + 128 * static_cast<int>(rank) + 32 * q;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      if (!out_fp32) {
+        uint32_t packed[128];
+#pragma unroll
+        for (int c = 0; c < 256; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_nowait(taddr + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * h]), ab),
+                                                            __fmul_rn(__uint_as_float(r[2 * h + 1]), ab));
+            packed[c / 2 + h] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+        }
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            if ((lane >> 4) == half) {
+              uint8_t* rowp = buf + (lane & 15) * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(packed[32 * p + 4 * j], packed[32 * p + 4 * j + 1], packed[32 * p + 4 * j + 2],
+                               packed[32 * p + 4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * 256 + 64 * p, row0 + 16 * half);
+              bulk_commit();
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          uint32_t r[32];
+          tmem_ld32_nowait(taddr + c, r);
+          tmem_ld_wait();
+          if (c + 32 == 256) {
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            if ((lane >> 4) == half) {
+              uint8_t* rowp = buf + (lane & 15) * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(__float_as_uint(__fmul_rn(__uint_as_float(r[4 * j]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 1]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 2]), ab)),
+                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 3]), ab)));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * 256 + c, row0 + 16 * half);
+              bulk_commit();
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  fence_before();
+  __syncwarp();
+  // neither CTA may leave (or free TMEM) while its peer can still touch its
+  // shared memory or its TMEM
+  cluster_sync();
+  if (threadIdx.x == 0 && *abort_flag && status) *status = kStatusTimeout;
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(P_TMEM_COLS) : "memory");
   }
 }
 
@@ -340,13 +772,30 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t kbytes, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D map over the output D [M, N] (row stride ldd elements): boxes of 16 rows
+// x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle, for TMA stores.
+bool make_out_map(CUtensorMap* map, void* base, int64_t M, int64_t N, int64_t ldd, bool fp32) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t esize = fp32 ? 4 : 2;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd) * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN>
 cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                    const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
                    int32_t* status, cudaStream_t st) {
   using G = Cfg<BN>;
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, A, M, K / 2, BM) || !make_map(&mb, B, N, K / 2, BN)) return cudaErrorInvalidValue;
+  const bool fp32 = out_dtype == NVFP4_OUT_DTYPE_FP32;
+  CUtensorMap ma, mb, md;
+  if (!make_map(&ma, A, M, K / 2, BM) || !make_map(&mb, B, N, K / 2, BN) || !make_out_map(&md, D, M, N, ldd, fp32))
+    return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -355,13 +804,64 @@ cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, con
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int grid = static_cast<int>((M / BM) * (N / BN));
-  nvfp4_gemm_kernel<BN><<<grid, NUM_THREADS, G::SMEM, st>>>(ma, mb, sA, sB, alphaA, alphaB, D, ldd,
-                                                            static_cast<int>(M), static_cast<int>(N),
-                                                            static_cast<int>(K), out_dtype == NVFP4_OUT_DTYPE_FP32,
-                                                            status);
+  const int64_t tiles = (M / BM) * (N / BN);
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());  // persistent: one CTA per SM
+  nvfp4_gemm_kernel<BN><<<grid, NUM_THREADS, G::SMEM, st>>>(ma, mb, md, sA, sB, alphaA, alphaB, static_cast<int>(M),
+                                                            static_cast<int>(N), static_cast<int>(K), fp32, status);
   note_launch();
   return cudaGetLastError();
+}
+
+// Scale array of an operand (GEMM layout) viewed as rows of 256 bytes:
+// 512-byte atoms -> two rows each; one stage of 4 atoms = 8 rows.
+bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int64_t bytes = (rows / 128) * (K / 64) * 512;
+  const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, 8};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
+                        const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
+                        int32_t* status, cudaStream_t st) {
+  const bool fp32 = out_dtype == NVFP4_OUT_DTYPE_FP32;
+  CUtensorMap ma, mb, md, msa, msb;
+  if (!make_map(&ma, A, M, K / 2, 128) || !make_map(&mb, B, N, K / 2, 128) ||
+      !make_out_map(&md, D, M, N, ldd, fp32) || !make_sf_map(&msa, sA, M, K) || !make_sf_map(&msb, sB, N, K))
+    return cudaErrorInvalidValue;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t tiles = (M / 256) * (N / 256);
+  const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;  // persistent: one pair per TPC
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = P_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel, ma, mb, md, msa, msb, alphaA, alphaB,
+                                     static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                                     static_cast<int>(fp32), status);
+  note_launch();
+  return e;
 }
 
 }  // namespace
@@ -369,6 +869,8 @@ cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, con
 cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                         const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
                         int32_t* status, cudaStream_t st) {
+  if (M % 256 == 0 && N % 256 == 0)
+    return launch_pair(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
   if (N % 256 == 0) return launch<256>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
   return launch<128>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
 }

@@ -73,7 +73,8 @@ def run_gemm(api, A, sA, aA, B, sB, aB, out_dtype):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 128), (128, 256, 256), (256, 384, 384), (384, 512, 1024),
-                                   (256, 256, 4096), (128, 128, 2048 + 128)])
+                                   (256, 256, 4096), (128, 128, 2048 + 128), (512, 512, 384),
+                                   (768, 1024, 2048), (2048, 1536, 256)])
 def test_random_operands(api, M, N, K):
     rng = np.random.default_rng(M * 7 + N * 13 + K)
     A, sA = rand_operand(rng, M, K)
