@@ -70,6 +70,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// One lane of a converged warp (elect.sync): the warp computes every operand
+// together so they stay warp-uniform, and this lane issues the single-thread
+// tcgen05 / TMA instruction.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -308,69 +321,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- producer: runs ahead across tiles ----------------
-      int it = 0;  // global stage counter
-      bool stop = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
-        const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
-        for (int kt = 0; kt < kstages; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) {
-            stop = true;
-            break;
-          }
-          const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);  // K blocks in this stage
-          const uint32_t bytes = G::A_STAGE + G::B_STAGE + nk * 512 * (1 + BN / 128);
-          const uint32_t fb = smem_u32(&full[s]);
+    // ---------------- producer: runs ahead across tiles ----------------
+    // The whole warp walks the loop (operands stay warp-uniform); lane 0
+    // waits, one elected lane issues the copies.
+    int it = 0;  // global stage counter
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+      const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+      for (int kt = 0; kt < kstages; ++kt, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag);
+        if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);  // K blocks in this stage
+        const uint32_t bytes = G::A_STAGE + G::B_STAGE + nk * 512 * (1 + BN / 128);
+        const uint32_t fb = smem_u32(&full[s]);
+        const uint32_t dA = smem_u32(sA + s * G::A_STAGE), dB = smem_u32(sB + s * G::B_STAGE);
+        const uint32_t dSA = smem_u32(sSFA + s * G::SFA_STAGE), dSB = smem_u32(sSFB + s * G::SFB_STAGE);
+        const uint8_t* gSA = sfa + (static_cast<int64_t>(tile_m) * kblocks64 + KB_PER_STAGE * kt) * 512;
+        if (elect_one()) {
           mbar_expect_tx(fb, bytes);
-          tma_load_2d(smem_u32(sA + s * G::A_STAGE), &tmap_a, kt * BK_BYTES, tile_m * BM, fb);
-          tma_load_2d(smem_u32(sB + s * G::B_STAGE), &tmap_b, kt * BK_BYTES, tile_n * BN, fb);
-          bulk_load(smem_u32(sSFA + s * G::SFA_STAGE),
-                    sfa + (static_cast<int64_t>(tile_m) * kblocks64 + KB_PER_STAGE * kt) * 512, nk * 512, fb);
+          tma_load_2d(dA, &tmap_a, kt * BK_BYTES, tile_m * BM, fb);
+          tma_load_2d(dB, &tmap_b, kt * BK_BYTES, tile_n * BN, fb);
+          bulk_load(dSA, gSA, nk * 512, fb);
 #pragma unroll
           for (int g = 0; g < BN / 128; ++g)
-            bulk_load(smem_u32(sSFB + s * G::SFB_STAGE + g * KB_PER_STAGE * 512),
+            bulk_load(dSB + g * KB_PER_STAGE * 512,
                       sfb + (static_cast<int64_t>(tile_n * (BN / 128) + g) * kblocks64 + KB_PER_STAGE * kt) * 512,
                       nk * 512, fb);
         }
+        __syncwarp();
       }
-      if (*abort_flag) {
-        // A wait gave up somewhere: let the copies this thread issued land
-        // before the CTA exits (each wait again bounded).
-        for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i) {
-          const uint32_t bar = smem_u32(&full[i % STAGES]), ph = (i / STAGES) & 1;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
-          }
+    }
+    if (lane == 0 && *abort_flag) {
+      // A wait gave up somewhere: let the copies already issued land before
+      // the CTA exits (each wait again bounded).
+      for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i) {
+        const uint32_t bar = smem_u32(&full[i % STAGES]), ph = (i / STAGES) & 1;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      // Per stage: wait for its data, copy its scales (one TMEM slot per K
-      // block, two slot sets used alternately so the copies never overwrite
-      // scales an earlier, still-running MMA reads), issue its MMAs, release
-      // the stage.  No wait on later stages sits between a stage's MMAs and
-      // its release.
-      const int my_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                           static_cast<int>(gridDim.x);
-      const int total = my_tiles * kstages;
-      for (int g = 0; g < total; ++g) {
-        const int kt = g % kstages, ti = g / kstages, s = g % STAGES;
-        if (kt == 0) {
-          // the epilogue must have drained the previous tile's accumulator
-          if (!mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag)) break;
-          fence_after();
-        }
-        if (!mbar_wait(smem_u32(&full[s]), (g / STAGES) & 1, abort_flag)) break;
+    // ---------------- MMA issuer ----------------
+    // Per stage: wait for its data, copy its scales (one TMEM slot per K
+    // block, two slot sets used alternately so the copies never overwrite
+    // scales an earlier, still-running MMA reads), issue its MMAs, release
+    // the stage.  The whole warp computes the operands; one elected lane
+    // issues the tcgen05 instructions.
+    const int my_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                         static_cast<int>(gridDim.x);
+    const int total = my_tiles * kstages;
+    for (int g = 0; g < total; ++g) {
+      const int kt = g % kstages, ti = g / kstages, s = g % STAGES;
+      bool ok = true;
+      if (kt == 0) {
+        // the epilogue must have drained the previous tile's accumulator
+        if (lane == 0) ok = mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag);
+        if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
         fence_after();
-        const uint32_t sfa_s = smem_u32(sSFA + s * G::SFA_STAGE);
-        const uint32_t sfb_s = smem_u32(sSFB + s * G::SFB_STAGE);
-        const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
-        const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
+      }
+      if (lane == 0) ok = mbar_wait(smem_u32(&full[s]), (g / STAGES) & 1, abort_flag);
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
+      fence_after();
+      const uint32_t sfa_s = smem_u32(sSFA + s * G::SFA_STAGE);
+      const uint32_t sfb_s = smem_u32(sSFB + s * G::SFB_STAGE);
+      const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
+      const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
+      const uint64_t adesc = desc_sw128(smem_u32(sA + s * G::A_STAGE));
+      const uint64_t bdesc = desc_sw128(smem_u32(sB + s * G::B_STAGE));
+      if (elect_one()) {
         for (int kk = 0; kk < nk; ++kk) {
           const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
           tmem_cp_sf(col, desc_sf(sfa_s + 512 * kk));
@@ -378,8 +403,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int gg = 0; gg < BN / 128; ++gg)
             tmem_cp_sf(col + 4 + 4 * gg, desc_sf(sfb_s + gg * KB_PER_STAGE * 512 + 512 * kk));
         }
-        const uint64_t adesc = desc_sw128(smem_u32(sA + s * G::A_STAGE));
-        const uint64_t bdesc = desc_sw128(smem_u32(sB + s * G::B_STAGE));
         for (int kk = 0; kk < nk; ++kk) {
           const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
           // K = 64 FP4 values = 32 bytes: advance the start address by 2 x 16 B
@@ -388,6 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(smem_u32(&empty[s]));
         if (kt == kstages - 1) umma_commit(smem_u32(acc_full));
       }
+      __syncwarp();
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
@@ -571,75 +595,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- producer (both CTAs) ----------------
-      int it = 0;
-      bool stop = false;
-      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
-        const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
-        for (int kt = 0; kt < kstages; ++kt, ++it) {
-          const int s = it % P_STAGES;
-          const uint32_t ph = (it / P_STAGES) & 1;
-          if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag)) {
-            stop = true;
-            break;
-          }
-          const uint32_t fb_leader = map_to_rank(smem_u32(&full[s]), 0);
-          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * P_STAGE);
-          tma_load_2d_pair(smem_u32(sA + s * P_STAGE_A), &tmap_a, kt * BK_BYTES, tile_m * 256 + 128 * rank,
-                           fb_leader);
-          tma_load_2d_pair(smem_u32(sB + s * P_STAGE_B), &tmap_b, kt * BK_BYTES, tile_n * 256 + 128 * rank,
-                           fb_leader);
-          // scale atoms viewed as rows of 256 bytes: a stage is 8 rows per 128 operand rows
-          tma_load_2d_pair(smem_u32(sSFA + s * P_STAGE_SFA), &tmap_sfa, 0,
-                           ((tile_m * 2 + static_cast<int>(rank)) * kblocks64 + KB_PER_STAGE * kt) * 2, fb_leader);
-#pragma unroll
-          for (int g = 0; g < 2; ++g)
-            tma_load_2d_pair(smem_u32(sSFB + s * P_STAGE_SFB + g * P_STAGE_SFA), &tmap_sfb, 0,
-                             ((tile_n * 2 + g) * kblocks64 + KB_PER_STAGE * kt) * 2, fb_leader);
+    // ---------------- producer (both CTAs; whole warp, one lane issues) ----------------
+    int it = 0;
+    bool stop = false;
+    for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
+      const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+      for (int kt = 0; kt < kstages; ++kt, ++it) {
+        const int s = it % P_STAGES;
+        const uint32_t ph = (it / P_STAGES) & 1;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag);
+        if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+          stop = true;
+          break;
         }
+        const uint32_t fb_leader = map_to_rank(smem_u32(&full[s]), 0);
+        const uint32_t dA = smem_u32(sA + s * P_STAGE_A), dB = smem_u32(sB + s * P_STAGE_B);
+        const uint32_t dSA = smem_u32(sSFA + s * P_STAGE_SFA), dSB = smem_u32(sSFB + s * P_STAGE_SFB);
+        // scale atoms viewed as rows of 256 bytes: a stage is 8 rows per 128 operand rows
+        const int ysa = ((tile_m * 2 + static_cast<int>(rank)) * kblocks64 + KB_PER_STAGE * kt) * 2;
+        const int ysb = ((tile_n * 2) * kblocks64 + KB_PER_STAGE * kt) * 2;
+        if (elect_one()) {
+          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * P_STAGE);
+          tma_load_2d_pair(dA, &tmap_a, kt * BK_BYTES, tile_m * 256 + 128 * rank, fb_leader);
+          tma_load_2d_pair(dB, &tmap_b, kt * BK_BYTES, tile_n * 256 + 128 * rank, fb_leader);
+          tma_load_2d_pair(dSA, &tmap_sfa, 0, ysa, fb_leader);
+          tma_load_2d_pair(dSB, &tmap_sfb, 0, ysb, fb_leader);
+          tma_load_2d_pair(dSB + P_STAGE_SFA, &tmap_sfb, 0, ysb + 2 * kblocks64, fb_leader);
+        }
+        __syncwarp();
       }
-      if (*abort_flag && leader) {
-        for (int i = (it > P_STAGES ? it - P_STAGES : 0); i < it; ++i) {
-          const uint32_t bar = smem_u32(&full[i % P_STAGES]), ph = (i / P_STAGES) & 1;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
-          }
+    }
+    if (lane == 0 && *abort_flag && leader) {
+      for (int i = (it > P_STAGES ? it - P_STAGES : 0); i < it; ++i) {
+        const uint32_t bar = smem_u32(&full[i % P_STAGES]), ph = (i / P_STAGES) & 1;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
         }
       }
     }
   } else if (warp == 1) {
-    if (leader && lane == 0) {
-      // ---------------- MMA issuer (leader only) ----------------
+    if (leader) {
+      // ---------------- MMA issuer (leader only; whole warp, one lane issues) ----------------
       const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
       const int total = my_tiles * kstages;
       for (int g = 0; g < total; ++g) {
         const int kt = g % kstages, ti = g / kstages, s = g % P_STAGES;
+        bool ok = true;
         if (kt == 0) {
-          if (!mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag)) break;
+          if (lane == 0) ok = mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag);
+          if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
           fence_after();
         }
-        if (!mbar_wait(smem_u32(&full[s]), (g / P_STAGES) & 1, abort_flag)) break;
+        if (lane == 0) ok = mbar_wait(smem_u32(&full[s]), (g / P_STAGES) & 1, abort_flag);
+        if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
         fence_after();
         const uint32_t sfa_s = smem_u32(sSFA + s * P_STAGE_SFA);
         const uint32_t sfb_s = smem_u32(sSFB + s * P_STAGE_SFB);
         const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
         const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
-          tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * kk));
-          tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * kk));
-          tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + P_STAGE_SFA + 512 * kk));
-        }
         const uint64_t adesc = desc_sw128(smem_u32(sA + s * P_STAGE_A));
         const uint64_t bdesc = desc_sw128(smem_u32(sB + s * P_STAGE_B));
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
-          mma_mxf4nvf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col,
-                            col + 4);
+        if (elect_one()) {
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
+            tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * kk));
+            tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * kk));
+            tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + P_STAGE_SFA + 512 * kk));
+          }
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
+            mma_mxf4nvf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col,
+                              col + 4);
+          }
+          umma_commit_pair(smem_u32(&empty[s]));
+          if (kt == kstages - 1) umma_commit_pair(smem_u32(acc_full));
         }
-        umma_commit_pair(smem_u32(&empty[s]));
-        if (kt == kstages - 1) umma_commit_pair(smem_u32(acc_full));
+        __syncwarp();
       }
     }
   } else {
