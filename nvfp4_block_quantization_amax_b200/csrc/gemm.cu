@@ -535,15 +535,18 @@ constexpr int P_STAGE_B = 128 * BK_BYTES;        // own B rows
 constexpr int P_STAGE_SFA = KB_PER_STAGE * 512;  // own A rows' scales
 constexpr int P_STAGE_SFB = 2 * KB_PER_STAGE * 512;  // all 256 B rows' scales
 constexpr int P_STAGE = P_STAGE_A + P_STAGE_B + P_STAGE_SFA + P_STAGE_SFB;
-constexpr int P_STAGES = (232448 - kOutStaging - 1024 - 512) / P_STAGE;
-constexpr int P_SMEM = P_STAGES * P_STAGE + kOutStaging + 1024 + 512;
+constexpr int P_EPI_WARPS = 8;                   // two per TMEM lane quarter, 128 columns each
+constexpr int P_THREADS = 64 + 32 * P_EPI_WARPS;
+constexpr int P_OUT_STAGING = P_EPI_WARPS * 2048;
+constexpr int P_STAGES = (232448 - P_OUT_STAGING - 1024 - 512) / P_STAGE;
+constexpr int P_SMEM = P_STAGES * P_STAGE + P_OUT_STAGING + 1024 + 512;
 constexpr uint32_t P_SF_W = 4 + 8;               // SFA 4 + SFB (256 rows) 8 columns per K block
 constexpr uint32_t P_SF_COL = 256;
 constexpr uint32_t P_TMEM_COLS = 512;            // 256 accumulator + 2 x 4 K blocks x 12 scale columns
 // M = 256 (>> 4 = 16 at bit 24), N = 256 (>> 3 = 32 at bit 17), E2M1 x E2M1, E4M3 scales
 constexpr uint32_t P_IDESC = (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(P_THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
                            const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
@@ -555,7 +558,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sSFA = sB + P_STAGES * P_STAGE_B;
   uint8_t* sSFB = sSFA + P_STAGES * P_STAGE_SFA;
   uint8_t* sOut = sSFB + P_STAGES * P_STAGE_SFB;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kOutStaging);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + P_OUT_STAGING);
   uint64_t* full = bars;
   uint64_t* empty = bars + P_STAGES;
   uint64_t* acc_full = bars + 2 * P_STAGES;
@@ -578,7 +581,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
-    mbar_init(smem_u32(acc_empty), 8);  // 4 epilogue warps in each CTA
+    mbar_init(smem_u32(acc_empty), 2 * P_EPI_WARPS);  // every epilogue warp of both CTAs
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -671,12 +674,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           umma_commit_pair(smem_u32(&empty[s]));
           if (kt == kstages - 1) umma_commit_pair(smem_u32(acc_full));
         }
-        __syncwarp();
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
-    const int q = warp & 3;
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31 and columns 128 h .. + 127
+    // (h = 0 for warps 2-5, 1 for warps 6-9): two warps share each lane
+    // quarter, each converting and storing half of the tile's columns.
+    const int q = warp & 3, h = (warp - 2) >> 2;
     uint8_t* buf = sOut + (warp - 2) * 2048;
     const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
@@ -686,26 +691,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(smem_u32(acc_full), ti & 1, abort_flag)) break;
       fence_after();
       const int row0 = tile_m * 256 + 128 * static_cast<int>(rank) + 32 * q;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      const int col0 = tile_n * 256 + 128 * h;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + 128 * h;
       if (!out_fp32) {
-        uint32_t packed[128];
+        uint32_t packed[64];
 #pragma unroll
-        for (int c = 0; c < 256; c += 32) {
-          uint32_t r[32];
+        for (int c = 0; c < 128; c += 64) {
+          uint32_t r[64];
           tmem_ld32_nowait(taddr + c, r);
+          tmem_ld32_nowait(taddr + c + 32, r + 32);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * h]), ab),
-                                                            __fmul_rn(__uint_as_float(r[2 * h + 1]), ab));
-            packed[c / 2 + h] = *reinterpret_cast<const uint32_t*>(&b2);
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), ab),
+                                                            __fmul_rn(__uint_as_float(r[2 * j + 1]), ab));
+            packed[c / 2 + j] = *reinterpret_cast<const uint32_t*>(&b2);
           }
         }
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < 2; ++p) {        // 64-column pieces
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             if (lane == 0) bulk_wait_read<0>();
@@ -721,18 +728,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * 256 + 64 * p, row0 + 16 * half);
+              tma_store_2d(&tmap_d, smem_u32(buf), col0 + 64 * p, row0 + 16 * half);
               bulk_commit();
             }
           }
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < 128; c += 32) {
           uint32_t r[32];
           tmem_ld32_nowait(taddr + c, r);
           tmem_ld_wait();
-          if (c + 32 == 256) {
+          if (c + 32 == 128) {
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
@@ -754,7 +761,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmap_d, smem_u32(buf), tile_n * 256 + c, row0 + 16 * half);
+              tma_store_2d(&tmap_d, smem_u32(buf), col0 + c, row0 + 16 * half);
               bulk_commit();
             }
           }
@@ -879,7 +886,7 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;  // persistent: one pair per TPC
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.blockDim = dim3(P_THREADS);
   cfg.dynamicSmemBytes = P_SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

@@ -201,6 +201,65 @@ __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
     v[i] = __uint_as_float(__float_as_uint(__fmul_rn(v[i], 0.25f)) ^ (((signs >> i) & 1u) << 31));
 }
 
+// ---------------------------------------------------------------------------
+// Lane-paired arithmetic: two independent blocks share each float2 (x = the
+// first block's element, y = the second's), so one packed sm_100 instruction
+// does the work of two.  Each component is rounded exactly as the scalar
+// __f*_rn operation; a - b is a + (-b), which IEEE defines to be the same.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// Sign masks of the rotation's diagonal: bit 31 set where element i flips.
+struct SignMasks {
+  uint32_t m[16];
+};
+__device__ __forceinline__ SignMasks sign_masks(uint32_t signs) {
+  SignMasks s;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) s.m[i] = ((signs >> i) & 1u) << 31;
+  return s;
+}
+
+// Two blocks of 16 bf16 (a0/a1: first block's halves, b0/b1: second's) ->
+// lane-paired floats with the diagonal's signs applied.
+__device__ __forceinline__ void unpack16x2_signed(const uint4 a0, const uint4 a1, const uint4 b0, const uint4 b1,
+                                                  const SignMasks& sm, float2* v) {
+  const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = make_float2(__uint_as_float((wa[j] << 16) ^ sm.m[2 * j]), __uint_as_float((wb[j] << 16) ^ sm.m[2 * j]));
+    v[2 * j + 1] = make_float2(__uint_as_float((wa[j] & 0xFFFF0000u) ^ sm.m[2 * j + 1]),
+                               __uint_as_float((wb[j] & 0xFFFF0000u) ^ sm.m[2 * j + 1]));
+  }
+}
+
+// H16 v for two lane-paired blocks (signs already applied): the butterfly of
+// rht16 without its final 1/4.
+__device__ __forceinline__ void hadamard16x2(float2* v) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const float2 a = v[i], b = v[i + h];
+        v[i] = add2(a, b);
+        v[i + h] = sub2(a, b);
+      }
+    }
+  }
+}
+
+// rht16 of two lane-paired blocks whose signs are already applied.
+__device__ __forceinline__ void rht16x2_presigned(float2* v) {
+  hadamard16x2(v);
+  const float2 q = make_float2(0.25f, 0.25f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = mul2(v[i], q);
+}
+
 // Pairwise sum with strides 8, 4, 2, 1 (the stated summation order).
 __device__ __forceinline__ float sum16(const float* e) {
   float t[8];

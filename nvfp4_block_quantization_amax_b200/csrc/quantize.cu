@@ -176,70 +176,177 @@ __device__ __forceinline__ Packed16 quantize_block(const float* v, float alpha,
 }
 
 // ===========================================================================
-// amax kernels
+// amax kernels.  Each CTA leaves one partial maximum (float bits, or
+// kNonFinite) per orientation; the quantize kernels reduce them.
 // ===========================================================================
-// Rows of 16-blocks, streamed: max |x| (or max |rotated block|).  Also the
-// plain amax for any orientation.  One partial per CTA.
-template <bool ROT, int NT>
-__global__ void __launch_bounds__(NT) amax_rows_kernel(const uint16_t* __restrict__ x, int64_t R,
-                                                       int64_t ld, FastDiv nb, uint64_t seed,
-                                                       uint32_t* __restrict__ partial) {
+// Plain amax: max |x| over the tensor in 16-byte chunks, four loads in
+// flight per thread.  bf16 magnitudes order like their bit patterns with the
+// sign cleared, so two are compared at once with a per-halfword unsigned
+// max; a pattern >= 0x7F80 is an Inf or a NaN.
+template <int NT>
+__global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t ld,
+                                                        FastDiv cpr, uint32_t* __restrict__ partial) {
   __shared__ uint32_t red[NT / 32];
-  uint32_t signs = 0;
-  if constexpr (ROT) signs = sign_bits(philox_keys(seed));
-  const uint32_t total = static_cast<uint32_t>(R) * nb.d;
-  uint32_t m = 0;
-  bool bad = false;
-  for (uint32_t k = blockIdx.x * NT + threadIdx.x; k < total; k += gridDim.x * NT) {
-    const uint32_t r = fastdiv(k, nb), cb = k - r * nb.d;
-    const uint4* p = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld + 16 * cb);
-    const uint4 a = __ldcs(p), b = __ldcs(p + 1);
-    float v[16];
-    unpack8(a, v);
-    unpack8(b, v + 8);
+  const uint32_t total = static_cast<uint32_t>(R) * cpr.d;   // chunks of 8 values
+  const uint32_t stride = gridDim.x * NT;
+  uint32_t hm = 0;
+  auto chunk = [&](uint32_t k) {
+    const uint32_t r = fastdiv(k, cpr), c = k - r * cpr.d;
+    return __ldcs(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld) + c);
+  };
+  uint32_t k = blockIdx.x * NT + threadIdx.x;
+  for (; k + 3 * stride < total; k += 4 * stride) {
+    uint4 u[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) bad |= abs_bits(v[i]) >= 0x7F800000u;
-    if constexpr (ROT) rht16(v, signs);
+    for (int j = 0; j < 4; ++j) u[j] = chunk(k + j * stride);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = max(m, abs_bits(v[i]));
+    for (int j = 0; j < 4; ++j) {
+      hm = __vmaxu2(hm, u[j].x & 0x7FFF7FFFu);
+      hm = __vmaxu2(hm, u[j].y & 0x7FFF7FFFu);
+      hm = __vmaxu2(hm, u[j].z & 0x7FFF7FFFu);
+      hm = __vmaxu2(hm, u[j].w & 0x7FFF7FFFu);
+    }
   }
-  if (bad) m = kNonFinite;
+  for (; k < total; k += stride) {
+    const uint4 u = chunk(k);
+    hm = __vmaxu2(hm, u.x & 0x7FFF7FFFu);
+    hm = __vmaxu2(hm, u.y & 0x7FFF7FFFu);
+    hm = __vmaxu2(hm, u.z & 0x7FFF7FFFu);
+    hm = __vmaxu2(hm, u.w & 0x7FFF7FFFu);
+  }
+  const uint32_t h = max(hm & 0xFFFFu, hm >> 16);
+  uint32_t m = (h >= 0x7F80u) ? kNonFinite : (h << 16);
   m = block_max_u32<NT>(m, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = m;
 }
 
-// Column-rotated amax: 16-row stripes; each thread owns two adjacent columns
-// of a stripe, so a warp reads 128 contiguous bytes per row.
-template <int NT>
-__global__ void __launch_bounds__(NT) amax_cols_kernel(const uint16_t* __restrict__ x, int64_t R,
-                                                       int64_t C, int64_t ld, uint64_t seed,
-                                                       uint32_t* __restrict__ partial) {
-  __shared__ uint32_t red[NT / 32];
-  const uint32_t signs = sign_bits(philox_keys(seed));
-  const int64_t pairs = C / 2, stripes = R / 16;
-  const int64_t total = pairs * stripes;
-  uint32_t m = 0;
-  bool bad = false;
-  for (int64_t k = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x; k < total;
-       k += static_cast<int64_t>(gridDim.x) * NT) {
-    const int64_t st = k / pairs, pr = k - st * pairs;
-    const uint32_t* base = reinterpret_cast<const uint32_t*>(x + 16 * st * ld) + pr;
-    float c0[16], c1[16];
+// Tiles of 64 x 128 bf16 staged in shared memory, two buffers so the next
+// tile streams in while this one is reduced.  The 16-byte chunks of a tile
+// row are stored with chunk c at c ^ ((c >> 3) & 1): the eight lanes that read
+// one row's eight 32-byte blocks then hit 32 distinct banks, and the lanes
+// reading a column word still see a permutation of one row's words.
+constexpr int TR = 64, TC = 128, TNT = 256;
+
+__device__ __forceinline__ int tile_chunk(int c) { return c ^ ((c >> 3) & 1); }
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// Issue the copies of tile `tile` (row-major tile grid) into buf.
+__device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
+                                                int64_t ld, int64_t tiles_c, int64_t tile) {
+  const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+  const int64_t r0 = tr * TR, c0 = tc * TC;
+  const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
+  const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t w = __ldcs(base + i * (ld / 2));
-      c0[i] = bf16lo(w);
-      c1[i] = bf16hi(w);
-      bad |= abs_bits(c0[i]) >= 0x7F800000u || abs_bits(c1[i]) >= 0x7F800000u;
-    }
-    rht16(c0, signs);
-    rht16(c1, signs);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) m = max(m, max(abs_bits(c0[i]), abs_bits(c1[i])));
+  for (int i = 0; i < 4; ++i) {
+    const int ch = threadIdx.x + TNT * i;
+    const int row = ch >> 4, cc = ch & 15;
+    if (row < rows && 8 * cc < cols) cp_async16(&buf[row][tile_chunk(cc)], x + (r0 + row) * ld + c0 + 8 * cc);
   }
-  if (bad) m = kNonFinite;
-  m = block_max_u32<NT>(m, red);
-  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+  cp_async_commit();
+}
+
+// Rotated maxima: rows (16-element blocks along a row) and / or columns
+// (16-element blocks down a column), from one read of the tensor.  The
+// butterfly runs on two blocks at once (lane-paired) and without its final
+// 1/4: round-to-nearest multiplication is monotone, so the maximum of the
+// scaled magnitudes is the scaled maximum, applied once per CTA.
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                        int64_t ld, int64_t tiles_c, int64_t ntiles, uint64_t seed,
+                                                        uint32_t* __restrict__ part_r,
+                                                        uint32_t* __restrict__ part_c) {
+  __shared__ __align__(16) uint4 tiles[2][TR][TC / 8];
+  __shared__ uint32_t red[TNT / 32];
+  const SignMasks sm = sign_masks(sign_bits(philox_keys(seed)));
+  const int t = threadIdx.x;
+  float mr = 0.0f, mc = 0.0f;
+  uint32_t hin = 0;   // per-halfword max of the input magnitudes (Inf / NaN check)
+  int64_t tile = blockIdx.x;
+  int buf = 0;
+  if (tile < ntiles) load_tile_async(tiles[0], x, R, C, ld, tiles_c, tile);
+  for (; tile < ntiles; tile += gridDim.x, buf ^= 1) {
+    const int64_t next = tile + gridDim.x;
+    if (next < ntiles) {
+      load_tile_async(tiles[buf ^ 1], x, R, C, ld, tiles_c, next);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint4 (*s)[TC / 8] = tiles[buf];
+    const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+    const int rows = static_cast<int>(R - tr * TR < TR ? R - tr * TR : TR);
+    const int cols = static_cast<int>(C - tc * TC < TC ? C - tc * TC : TC);
+    if constexpr (ROW) {
+      // blocks (row, cb) and (row + 32, cb)
+      const int row = t >> 3, cb = t & 7;
+      const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
+      const uint4 a0 = s[row][tile_chunk(2 * cb)], a1 = s[row][tile_chunk(2 * cb + 1)];
+      const uint4 b0 = s[row + 32][tile_chunk(2 * cb)], b1 = s[row + 32][tile_chunk(2 * cb + 1)];
+      if (va) {
+        hin = __vmaxu2(hin, a0.x & 0x7FFF7FFFu); hin = __vmaxu2(hin, a0.y & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, a0.z & 0x7FFF7FFFu); hin = __vmaxu2(hin, a0.w & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, a1.x & 0x7FFF7FFFu); hin = __vmaxu2(hin, a1.y & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, a1.z & 0x7FFF7FFFu); hin = __vmaxu2(hin, a1.w & 0x7FFF7FFFu);
+      }
+      if (vb) {
+        hin = __vmaxu2(hin, b0.x & 0x7FFF7FFFu); hin = __vmaxu2(hin, b0.y & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, b0.z & 0x7FFF7FFFu); hin = __vmaxu2(hin, b0.w & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, b1.x & 0x7FFF7FFFu); hin = __vmaxu2(hin, b1.y & 0x7FFF7FFFu);
+        hin = __vmaxu2(hin, b1.z & 0x7FFF7FFFu); hin = __vmaxu2(hin, b1.w & 0x7FFF7FFFu);
+      }
+      float2 v[16];
+      unpack16x2_signed(a0, a1, b0, b1, sm, v);
+      hadamard16x2(v);
+      float ma = 0.0f, mb = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        ma = fmaxf(ma, fabsf(v[i].x));
+        mb = fmaxf(mb, fabsf(v[i].y));
+      }
+      if (va) mr = fmaxf(mr, ma);
+      if (vb) mr = fmaxf(mr, mb);
+    }
+    if constexpr (COL) {
+      // columns (2 cp, 2 cp + 1) of row block rb: one 32-bit word per row
+      const int cp = t & 63, rb = t >> 6;
+      if (16 * rb < rows && 2 * cp < cols) {
+        const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
+        const int wofs = (tile_chunk(cp >> 2) << 2) | (cp & 3);
+        float2 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = base[i * (TC / 2) + wofs];
+          if constexpr (!ROW) hin = __vmaxu2(hin, w & 0x7FFF7FFFu);
+          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+        }
+        hadamard16x2(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mc = fmaxf(mc, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      }
+    }
+    __syncthreads();   // buf is refilled two iterations from now
+  }
+  const uint32_t h = max(hin & 0xFFFFu, hin >> 16);
+  const bool bad = h >= 0x7F80u;
+  if constexpr (ROW) {
+    uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mr, 0.25f));
+    m = block_max_u32<TNT>(m, red);
+    if (t == 0) part_r[blockIdx.x] = m;
+  }
+  if constexpr (COL) {
+    uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mc, 0.25f));
+    m = block_max_u32<TNT>(m, red);
+    if (t == 0) part_c[blockIdx.x] = m;
+  }
 }
 
 // ===========================================================================
@@ -287,7 +394,6 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
 // Tiled quantization: columns, dual rows + columns, and 2D 16x16 blocks.
 // Tile: 64 rows x 128 columns of bf16 (16 KB) in shared memory.
 // ===========================================================================
-constexpr int TR = 64, TC = 128, TNT = 256;
 constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
 
 struct TileSmem {
@@ -297,10 +403,6 @@ struct TileSmem {
   uint8_t scale2d[TR / 16][TC / 16];        // chosen 2D scales
 };
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
 }
@@ -571,12 +673,17 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   uint32_t* pr = const_cast<uint32_t*>(a.partials);
   uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
   if (!rot) {
-    amax_rows_kernel<false, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr);
-    note_launch();
-    return cudaGetLastError();
+    amax_plain_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, make_fastdiv(static_cast<uint32_t>(a.C / 8)), pr);
+  } else {
+    const int64_t ntiles = a.tiles_r * a.tiles_c;
+    if (row && col)
+      amax_tile_kernel<true, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
+    else if (row)
+      amax_tile_kernel<true, false><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
+    else
+      amax_tile_kernel<false, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
   }
-  if (row) { amax_rows_kernel<true, 256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.nb_row, a.seed, pr); note_launch(); }
-  if (col) { amax_cols_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.C, a.ld, a.seed, pc); note_launch(); }
+  note_launch();
   return cudaGetLastError();
 }
 
