@@ -108,8 +108,10 @@ __device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t u24) {
   if (e4m3_value(lo) > v) --lo;
   const float vlo = e4m3_value(lo);
   if (vlo == v) return lo;
-  const float gap = __fsub_rn(e4m3_value(lo + 1), vlo);        // a power of two
-  const float f = __fdiv_rn(__fsub_rn(v, vlo), gap);           // exact
+  // gap is a normal power of two, so 1/gap is exact (exponent 254 - e) and
+  // the product below equals the exact quotient (v - vlo) / gap.
+  const float gap = __fsub_rn(e4m3_value(lo + 1), vlo);
+  const float f = __fmul_rn(__fsub_rn(v, vlo), __uint_as_float(0x7F000000u - __float_as_uint(gap)));
   return (static_cast<float>(u24) < __fmul_rn(f, 16777216.0f)) ? lo + 1 : lo;
 }
 
@@ -205,10 +207,11 @@ __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
 // Lane-paired arithmetic: two independent blocks share each float2 (x = the
 // first block's element, y = the second's), so one packed sm_100 instruction
 // does the work of two.  Each component is rounded exactly as the scalar
-// __f*_rn operation; a - b is a + (-b), which IEEE defines to be the same.
+// __f*_rn operation.  a - b is formed as fma(b, -1, a): the product b * -1 is
+// exact, so the single rounding gives RN(a - b), signed zeros included.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // Sign masks of the rotation's diagonal: bit 31 set where element i flips.
@@ -370,6 +373,111 @@ __device__ __forceinline__ float sq_error(const float* v, float alpha, uint32_t 
     e[i] = __fmul_rn(d, d);
   }
   return sum16(e);
+}
+
+// ---------------------------------------------------------------------------
+// Eight values <-> one word of eight E2M1 codes (element k in bits 4k..4k+3).
+// Same conversions as e2m1x2_rne / e2m1x2_values, four at a time.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1x8_rne(float y0, float y1, float y2, float y3, float y4, float y5,
+                                               float y6, float y7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+  return r;
+}
+
+__device__ __forceinline__ void e2m1x8_values(uint32_t w, float* q) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+      ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %8;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+      "mov.b32 {l0, u0}, h0;\n\t"
+      "mov.b32 {l1, u1}, h1;\n\t"
+      "mov.b32 {l2, u2}, h2;\n\t"
+      "mov.b32 {l3, u3}, h3;\n\t"
+      "cvt.f32.f16 %0, l0;\n\tcvt.f32.f16 %1, u0;\n\t"
+      "cvt.f32.f16 %2, l1;\n\tcvt.f32.f16 %3, u1;\n\t"
+      "cvt.f32.f16 %4, l2;\n\tcvt.f32.f16 %5, u2;\n\t"
+      "cvt.f32.f16 %6, l3;\n\tcvt.f32.f16 %7, u3;\n\t}"
+      : "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]), "=f"(q[6]), "=f"(q[7])
+      : "r"(w));
+}
+
+// Sign-only codes (magnitude 0) of one lane of sixteen pairs.
+template <bool Y>
+__device__ __forceinline__ Packed16 sign_codes16(const float2* v) {
+  Packed16 p{0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t sign = (__float_as_uint(Y ? v[i].y : v[i].x) >> 31) << 3;
+    if (i < 8) p.lo |= sign << (4 * i);
+    else p.hi |= sign << (4 * (i - 8));
+  }
+  return p;
+}
+
+// encode_rne for two lane-paired blocks with scale bytes sba (x) and sbb (y).
+__device__ __forceinline__ void encode_rne_x2(const float2* v, float alpha, uint32_t sba, uint32_t sbb,
+                                              Packed16& pa, Packed16& pb) {
+  const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
+  const float rb = __frcp_rn(__fmul_rn(alpha, e4m3_value(sbb)));
+  const float2 r2 = make_float2(ra, rb);
+  float2 y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = mul2(v[i], r2);
+  pa.lo = e2m1x8_rne(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
+  pa.hi = e2m1x8_rne(y[8].x, y[9].x, y[10].x, y[11].x, y[12].x, y[13].x, y[14].x, y[15].x);
+  pb.lo = e2m1x8_rne(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
+  pb.hi = e2m1x8_rne(y[8].y, y[9].y, y[10].y, y[11].y, y[12].y, y[13].y, y[14].y, y[15].y);
+  if (isinf(ra)) pa = sign_codes16<false>(v);
+  if (isinf(rb)) pb = sign_codes16<true>(v);
+}
+
+// Grid values of two blocks' codes, lane-paired.
+__device__ __forceinline__ void decode16x2(const Packed16& pa, const Packed16& pb, float2* q) {
+  float a[16], b[16];
+  e2m1x8_values(pa.lo, a);
+  e2m1x8_values(pa.hi, a + 8);
+  e2m1x8_values(pb.lo, b);
+  e2m1x8_values(pb.hi, b + 8);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) q[i] = make_float2(a[i], b[i]);
+}
+
+// sum16 of two lane-paired blocks.
+__device__ __forceinline__ float2 sum16x2(const float2* e) {
+  float2 t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = add2(e[i], e[i + 8]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t[i] = add2(t[i], t[i + 4]);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) t[i] = add2(t[i], t[i + 2]);
+  return add2(t[0], t[1]);
+}
+
+// sq_error of two lane-paired encodings.
+__device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint32_t sba, uint32_t sbb,
+                                              const Packed16& pa, const Packed16& pb) {
+  const float2 s2 = make_float2(__fmul_rn(alpha, e4m3_value(sba)), __fmul_rn(alpha, e4m3_value(sbb)));
+  float2 q[16], e[16];
+  decode16x2(pa, pb, q);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 d = sub2(v[i], mul2(q[i], s2));
+    e[i] = mul2(d, d);
+  }
+  return sum16x2(e);
 }
 
 // Unsigned division by a runtime constant d >= 1 for n < 2^32:

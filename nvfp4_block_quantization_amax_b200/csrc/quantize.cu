@@ -44,6 +44,7 @@ struct QuantArgs {
   int32_t* status;
   FastDiv nb_row;                 // C / 16
   int64_t tiles_r, tiles_c;       // tile grid (tile kernels)
+  FastDiv tiles_c_div;            // divides a tile index by tiles_c
 };
 
 constexpr uint32_t kNonFinite = 0xFFFFFFFFu;   // partial marker: a NaN / Inf was read
@@ -221,13 +222,16 @@ __global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restri
 }
 
 // Tiles of 64 x 128 bf16 staged in shared memory, two buffers so the next
-// tile streams in while this one is reduced.  The 16-byte chunks of a tile
-// row are stored with chunk c at c ^ ((c >> 3) & 1): the eight lanes that read
-// one row's eight 32-byte blocks then hit 32 distinct banks, and the lanes
-// reading a column word still see a permutation of one row's words.
+// tile streams in while this one is processed.  Chunk c (16 bytes) of tile
+// row r is stored at slot (c ^ ((c >> 3) & 1)) ^ (2 ((r >> 4) & 3)): the
+// eight lanes reading one row's eight 32-byte blocks hit 32 distinct banks,
+// and so do 32 lanes reading one 32-bit column word each from 8 columns
+// pairs x 4 row blocks, or from 32 column pairs of one row.
 constexpr int TR = 64, TC = 128, TNT = 256;
 
-__device__ __forceinline__ int tile_chunk(int c) { return c ^ ((c >> 3) & 1); }
+__device__ __forceinline__ int tile_chunk(int r, int c) { return (c ^ ((c >> 3) & 1)) ^ (((r >> 4) & 3) << 1); }
+// 32-bit word w (columns 2w, 2w + 1) of tile row r
+__device__ __forceinline__ int tile_word(int r, int w) { return (tile_chunk(r, w >> 2) << 2) | (w & 3); }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -237,10 +241,18 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
+// Tile index -> (tile row, tile column) of the row-major tile grid.
+__device__ __forceinline__ void tile_coords(uint32_t tile, const FastDiv& tiles_c, int64_t& tr, int64_t& tc) {
+  const uint32_t q = fastdiv(tile, tiles_c);
+  tr = q;
+  tc = tile - q * tiles_c.d;
+}
+
 // Issue the copies of tile `tile` (row-major tile grid) into buf.
 __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
-                                                int64_t ld, int64_t tiles_c, int64_t tile) {
-  const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+                                                int64_t ld, const FastDiv& tiles_c, uint32_t tile) {
+  int64_t tr, tc;
+  tile_coords(tile, tiles_c, tr, tc);
   const int64_t r0 = tr * TR, c0 = tc * TC;
   const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
   const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
@@ -248,7 +260,7 @@ __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint
   for (int i = 0; i < 4; ++i) {
     const int ch = threadIdx.x + TNT * i;
     const int row = ch >> 4, cc = ch & 15;
-    if (row < rows && 8 * cc < cols) cp_async16(&buf[row][tile_chunk(cc)], x + (r0 + row) * ld + c0 + 8 * cc);
+    if (row < rows && 8 * cc < cols) cp_async16(&buf[row][tile_chunk(row, cc)], x + (r0 + row) * ld + c0 + 8 * cc);
   }
   cp_async_commit();
 }
@@ -260,7 +272,7 @@ __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint
 // scaled magnitudes is the scaled maximum, applied once per CTA.
 template <bool ROW, bool COL>
 __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                        int64_t ld, int64_t tiles_c, int64_t ntiles, uint64_t seed,
+                                                        int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
                                                         uint32_t* __restrict__ part_r,
                                                         uint32_t* __restrict__ part_c) {
   __shared__ __align__(16) uint4 tiles[2][TR][TC / 8];
@@ -269,11 +281,11 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
   const int t = threadIdx.x;
   float mr = 0.0f, mc = 0.0f;
   uint32_t hin = 0;   // per-halfword max of the input magnitudes (Inf / NaN check)
-  int64_t tile = blockIdx.x;
+  uint32_t tile = blockIdx.x;
   int buf = 0;
   if (tile < ntiles) load_tile_async(tiles[0], x, R, C, ld, tiles_c, tile);
   for (; tile < ntiles; tile += gridDim.x, buf ^= 1) {
-    const int64_t next = tile + gridDim.x;
+    const uint32_t next = tile + gridDim.x;
     if (next < ntiles) {
       load_tile_async(tiles[buf ^ 1], x, R, C, ld, tiles_c, next);
       cp_async_wait<1>();
@@ -282,15 +294,17 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
     }
     __syncthreads();
     const uint4 (*s)[TC / 8] = tiles[buf];
-    const int64_t tr = tile / tiles_c, tc = tile - tr * tiles_c;
+    int64_t tr, tc;
+    tile_coords(tile, tiles_c, tr, tc);
     const int rows = static_cast<int>(R - tr * TR < TR ? R - tr * TR : TR);
     const int cols = static_cast<int>(C - tc * TC < TC ? C - tc * TC : TC);
     if constexpr (ROW) {
       // blocks (row, cb) and (row + 32, cb)
       const int row = t >> 3, cb = t & 7;
       const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
-      const uint4 a0 = s[row][tile_chunk(2 * cb)], a1 = s[row][tile_chunk(2 * cb + 1)];
-      const uint4 b0 = s[row + 32][tile_chunk(2 * cb)], b1 = s[row + 32][tile_chunk(2 * cb + 1)];
+      const uint4 a0 = s[row][tile_chunk(row, 2 * cb)], a1 = s[row][tile_chunk(row, 2 * cb + 1)];
+      const uint4 b0 = s[row + 32][tile_chunk(row + 32, 2 * cb)];
+      const uint4 b1 = s[row + 32][tile_chunk(row + 32, 2 * cb + 1)];
       if (va) {
         hin = __vmaxu2(hin, a0.x & 0x7FFF7FFFu); hin = __vmaxu2(hin, a0.y & 0x7FFF7FFFu);
         hin = __vmaxu2(hin, a0.z & 0x7FFF7FFFu); hin = __vmaxu2(hin, a0.w & 0x7FFF7FFFu);
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
       const int cp = t & 63, rb = t >> 6;
       if (16 * rb < rows && 2 * cp < cols) {
         const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
-        const int wofs = (tile_chunk(cp >> 2) << 2) | (cp & 3);
+        const int wofs = tile_word(16 * rb, cp);   // the same for all 16 rows of the block
         float2 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -440,10 +454,11 @@ __global__ void __launch_bounds__(TNT) quant_tile_kernel(const QuantArgs a) {
   const bool check = (a.flags & kAlphaProvided) != 0;
   const int t = threadIdx.x;
   const int64_t R = a.R, C = a.C;
-  const int64_t ntiles = a.tiles_r * a.tiles_c;
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
 
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
+  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    int64_t tr, tc;
+    tile_coords(tile, a.tiles_c_div, tr, tc);
     const int64_t r0 = tr * TR, c0 = tc * TC;
     const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);   // multiple of 16
     const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);   // multiple of 16
@@ -616,6 +631,291 @@ __global__ void __launch_bounds__(TNT) quant_tile_kernel(const QuantArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// quantize_block for two lane-paired blocks (x: block a, y: block b): the
+// same arithmetic, with the element-wise steps done two blocks at a time.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
+  ma = 0.0f;
+  mb = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    ma = fmaxf(ma, fabsf(v[i].x));
+    mb = fmaxf(mb, fabsf(v[i].y));
+  }
+}
+
+// Word of the scale-SR draw that block blk uses: draw blk / 4, word blk % 4.
+__device__ __forceinline__ uint32_t eden_word(const PhiloxKeys& K, uint32_t c2, uint64_t blk) {
+  const uint64_t unit = blk >> 2;
+  const uint4 w = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
+  const uint32_t sel = static_cast<uint32_t>(blk & 3);
+  return sel == 0 ? w.x : (sel == 1 ? w.y : (sel == 2 ? w.z : w.w));
+}
+
+// MS-EDEN scale of one block from its sums and its random word.
+__device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t word) {
+  if (den == 0.0f) return 0u;
+  return e4m3_sr(__fdiv_rn(num, den), word >> 8);
+}
+
+// have_words: MS-EDEN only - wa / wb already hold the blocks' scale-SR words.
+template <int MODE>
+__device__ __forceinline__ void quantize_pair(const float2* v, float alpha, const PhiloxKeys& K, uint32_t c2,
+                                              uint64_t blka, uint64_t blkb, Packed16& pa, Packed16& pb,
+                                              uint32_t& sba, uint32_t& sbb, bool have_words = false,
+                                              uint32_t wa = 0u, uint32_t wb = 0u) {
+  float ma, mb;
+  max_abs16x2(v, ma, mb);
+  if constexpr (MODE == kModeRTN) {
+    sba = e4m3_rne(scale_raw(ma, alpha, 6.0f));
+    sbb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+    encode_rne_x2(v, alpha, sba, sbb, pa, pb);
+  } else if constexpr (MODE == kModeFourSix) {
+    const uint32_t a6 = e4m3_rne(scale_raw(ma, alpha, 6.0f)), b6 = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+    const uint32_t a4 = e4m3_rne(scale_raw(ma, alpha, 4.0f)), b4 = e4m3_rne(scale_raw(mb, alpha, 4.0f));
+    Packed16 pa6, pb6, pa4, pb4;
+    encode_rne_x2(v, alpha, a6, b6, pa6, pb6);
+    encode_rne_x2(v, alpha, a4, b4, pa4, pb4);
+    const float2 e6 = sq_error_x2(v, alpha, a6, b6, pa6, pb6);
+    const float2 e4 = sq_error_x2(v, alpha, a4, b4, pa4, pb4);
+    const bool ta = e4.x < e6.x, tb = e4.y < e6.y;
+    sba = ta ? a4 : a6;
+    pa = ta ? pa4 : pa6;
+    sbb = tb ? b4 : b6;
+    pb = tb ? pb4 : pb6;
+  } else if constexpr (MODE == kModeMsEden) {
+    const uint32_t prova = e4m3_rne(scale_raw(ma, alpha, 6.0f));
+    const uint32_t provb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+    encode_rne_x2(v, alpha, prova, provb, pa, pb);
+    float2 q[16], rr[16], rq[16];
+    decode16x2(pa, pb, q);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      rr[i] = mul2(v[i], v[i]);
+      rq[i] = mul2(v[i], q[i]);
+    }
+    const float2 num = sum16x2(rr);
+    const float2 den = mul2(make_float2(alpha, alpha), sum16x2(rq));
+    if (!have_words) {
+      wa = eden_word(K, c2, blka);
+      wb = eden_word(K, c2, blkb);
+    }
+    sba = eden_scale(num.x, den.x, wa);
+    sbb = eden_scale(num.y, den.y, wb);
+  } else {  // stochastic rounding of the values: one block at a time
+    float a[16], b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      a[i] = v[i].x;
+      b[i] = v[i].y;
+    }
+    pa = quantize_block<MODE>(a, alpha, K, c2, blka, sba);
+    pb = quantize_block<MODE>(b, alpha, K, c2, blkb, sbb);
+  }
+}
+
+// ===========================================================================
+// Tiled 1D quantization (columns, or rows + columns from one read), two
+// blocks per thread per orientation, lane-paired.
+//   rows:    thread t takes row blocks (t / 8, t % 8) and (t / 8 + 32, t % 8)
+//   columns: thread t takes columns 2 (t / 4), 2 (t / 4) + 1 of row block t % 4
+// Column codes are staged transposed in shared memory and written as whole
+// 32-byte rows of the column-major output.
+// ===========================================================================
+// Tiles stream through a ring of kTileStages shared-memory buffers (dynamic
+// shared memory), so up to kTileStages - 1 tiles are in flight per CTA while
+// one is processed.
+constexpr int kTileStages = 4;
+constexpr int kTileBytes = TR * TC * 2;
+
+template <int MODE, bool ROT, bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT, 2) quant_tile_1d_kernel(const QuantArgs a) {
+  extern __shared__ __align__(16) uint8_t tile_ring[];
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(tile_ring);
+  __shared__ __align__(16) uint8_t colcodes[TC][kColPitch];
+  __shared__ uint8_t colscale[TC][TR / 16];
+  __shared__ uint32_t red[TNT / 32];
+  float alpha_r, alpha_c;
+  resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red);
+  const PhiloxKeys K = philox_keys(a.seed);
+  SignMasks sm;
+  if constexpr (ROT) {
+    sm = sign_masks(sign_bits(K));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sm.m[i] = 0u;
+  }
+  const uint32_t c2r = a.stream_id * 2u, c2c = a.stream_id * 2u + 1u;
+  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
+  const bool check = (a.flags & kAlphaProvided) != 0;
+  const int t = threadIdx.x;
+  const int64_t R = a.R, C = a.C;
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  // MS-EDEN draws one 4-word number per 4 consecutive blocks.  The lanes
+  // 4k .. 4k+3 of a warp hold the same two row-block units and the same two
+  // column-block units of a tile (when C and R are multiples of 64, so units
+  // never straddle a row or a column), each lane needing word (lane % 4) of
+  // all four draws: each lane computes one draw and a 4 x 4 shuffle
+  // transpose hands the words out.
+  const bool share = MODE == kModeMsEden && (!ROW || C % 64 == 0) && (!COL || R % 64 == 0);
+  const int lane = t & 31, j4 = t & 3;
+
+  // prologue: the first kTileStages - 1 tiles (an empty copy group when a
+  // tile does not exist keeps the group count in step)
+  uint32_t tile = blockIdx.x;
+#pragma unroll
+  for (int k = 0; k < kTileStages - 1; ++k) {
+    const uint32_t tk = tile + k * gridDim.x;
+    if (tk < ntiles) load_tile_async(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
+    else cp_async_commit();
+  }
+  int buf = 0;
+  for (; tile < ntiles; tile += gridDim.x, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
+    const uint32_t ahead = tile + (kTileStages - 1) * gridDim.x;
+    const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;   // (buf + kTileStages - 1) % kTileStages
+    if (ahead < ntiles) load_tile_async(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
+    else cp_async_commit();
+    cp_async_wait<kTileStages - 1>();   // this tile's group has landed
+    __syncthreads();
+    const uint4 (*s)[TC / 8] = tiles[buf];
+    int64_t tr, tc;
+    tile_coords(tile, a.tiles_c_div, tr, tc);
+    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
+    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
+
+    // scale-SR words of this thread's blocks: row a, row b, column 2cp, 2cp+1
+    uint32_t w_ra = 0u, w_rb = 0u, w_ca = 0u, w_cb = 0u;
+    if (share) {
+      uint64_t unit;
+      uint32_t c2;
+      if (j4 < 2) {   // row block units: row (t / 8) + 32 j4, blocks (t % 8) & ~3 ..
+        const int64_t grow = r0 + (t >> 3) + 32 * j4;
+        unit = (static_cast<uint64_t>(grow) * (C / 16) + c0 / 16 + ((t & 7) & ~3)) >> 2;
+        c2 = c2r;
+      } else {        // column units: column 2 (t / 4) + (j4 - 2), row blocks r0/16 ..
+        const int64_t gcol = c0 + 2 * (t >> 2) + (j4 - 2);
+        unit = (static_cast<uint64_t>(gcol) * (R / 16) + r0 / 16) >> 2;
+        c2 = c2c;
+      }
+      const uint4 d = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
+      uint32_t got[4];   // got[r] = word j4 of the draw of lane (j4 + r) % 4
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int wi = (j4 - r) & 3;
+        const uint32_t send = wi == 0 ? d.x : (wi == 1 ? d.y : (wi == 2 ? d.z : d.w));
+        got[r] = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((j4 + r) & 3));
+      }
+      auto pick = [&](int dj) {
+        const int r = (dj - j4) & 3;
+        return r == 0 ? got[0] : (r == 1 ? got[1] : (r == 2 ? got[2] : got[3]));
+      };
+      w_ra = pick(0);
+      w_rb = pick(1);
+      w_ca = pick(2);
+      w_cb = pick(3);
+    }
+
+    if (check) {
+      uint32_t hin = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ch = t + TNT * i;
+        const int row = ch >> 4, cc = ch & 15;
+        if (row < rows && 8 * cc < cols) {
+          const uint4 u = s[row][tile_chunk(row, cc)];
+          hin = __vmaxu2(hin, u.x & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.y & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.z & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.w & 0x7FFF7FFFu);
+        }
+      }
+      if (max(hin & 0xFFFFu, hin >> 16) >= 0x7F80u && a.status) *a.status = kStatusNonFinite;
+    }
+
+    if constexpr (ROW) {
+      const int row = t >> 3, cb = t & 7;
+      const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
+      if (va || vb) {
+        const uint4 a0 = s[row][tile_chunk(row, 2 * cb)], a1 = s[row][tile_chunk(row, 2 * cb + 1)];
+        const uint4 b0 = s[row + 32][tile_chunk(row + 32, 2 * cb)];
+        const uint4 b1 = s[row + 32][tile_chunk(row + 32, 2 * cb + 1)];
+        float2 v[16];
+        unpack16x2_signed(a0, a1, b0, b1, sm, v);
+        if constexpr (ROT) rht16x2_presigned(v);
+        const int64_t gra = r0 + row, grb = gra + 32, gcb = c0 / 16 + cb;
+        const uint64_t blka = static_cast<uint64_t>(gra) * (C / 16) + gcb;
+        const uint64_t blkb = static_cast<uint64_t>(grb) * (C / 16) + gcb;
+        Packed16 pa, pb;
+        uint32_t sa, sb;
+        quantize_pair<MODE>(v, alpha_r, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+        if (va) {
+          *reinterpret_cast<uint2*>(a.codes_row + gra * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
+          if (a.scales_row)
+            a.scales_row[gemm ? gemm_scale_offset(gra, gcb, C / 16) : static_cast<int64_t>(blka)] =
+                static_cast<uint8_t>(sa);
+        }
+        if (vb) {
+          *reinterpret_cast<uint2*>(a.codes_row + grb * (C / 2) + 8 * gcb) = make_uint2(pb.lo, pb.hi);
+          if (a.scales_row)
+            a.scales_row[gemm ? gemm_scale_offset(grb, gcb, C / 16) : static_cast<int64_t>(blkb)] =
+                static_cast<uint8_t>(sb);
+        }
+      }
+    }
+
+    if constexpr (COL) {
+      const int cp = t >> 2, rb = t & 3;
+      if (16 * rb < rows && 2 * cp < cols) {
+        const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
+        const int wofs = tile_word(16 * rb, cp);   // the same for all 16 rows of the block
+        float2 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = base[i * (TC / 2) + wofs];
+          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+        }
+        if constexpr (ROT) rht16x2_presigned(v);
+        const int64_t nbc = R / 16;
+        const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
+        Packed16 qa, qb;
+        uint32_t sa, sb;
+        quantize_pair<MODE>(v, alpha_c, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
+                            static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+        *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
+        *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
+        colscale[2 * cp][rb] = static_cast<uint8_t>(sa);
+        colscale[2 * cp + 1][rb] = static_cast<uint8_t>(sb);
+      }
+      __syncthreads();
+      {
+        const int c = t >> 1, h = t & 1;
+        const int nbytes = rows / 2;
+        if (c < cols && 16 * h < nbytes) {
+          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
+          const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
+          reinterpret_cast<uint2*>(dst)[0] = src[0];
+          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+        }
+      }
+      if (a.scales_col) {
+        const int c = t >> 1;
+        if (c < cols) {
+          for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
+            const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
+            const uint8_t sbyte = colscale[c][rb2];
+            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
+            else a.scales_col[gc * (R / 16) + grb] = sbyte;
+          }
+        }
+      }
+    }
+    __syncthreads();   // buf and the staging are reused
+  }
+  cp_async_wait<0>();
+}
+
 // ===========================================================================
 // Host-side launchers
 // ===========================================================================
@@ -651,9 +951,29 @@ static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
 
 template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
 static cudaError_t launch_tile(const QuantArgs& a, cudaStream_t st) {
-  const int64_t ntiles = a.tiles_r * a.tiles_c;
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 6));
   quant_tile_kernel<MODE, ROT, ROW, COL, TWO_D><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int MODE, bool ROT, bool ROW, bool COL>
+static cudaError_t launch_tile_1d(const QuantArgs& a, cudaStream_t st) {
+  constexpr size_t smem = static_cast<size_t>(kTileStages) * kTileBytes;
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    cudaFuncSetAttribute(quant_tile_1d_kernel<MODE, ROT, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tile_1d_kernel<MODE, ROT, ROW, COL>, TNT, smem) !=
+            cudaSuccess || n <= 0)
+      n = 1;
+    per_sm = n;
+  }
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
+  quant_tile_1d_kernel<MODE, ROT, ROW, COL><<<std::max(blocks, 1), TNT, smem, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
@@ -661,8 +981,8 @@ static cudaError_t launch_tile(const QuantArgs& a, cudaStream_t st) {
 template <int MODE, bool ROT>
 static cudaError_t dispatch_1d(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
   if (row && !col) return launch_rows<MODE, ROT>(a, st);
-  if (row && col) return launch_tile<MODE, ROT, true, true, false>(a, st);
-  return launch_tile<MODE, ROT, false, true, false>(a, st);
+  if (row && col) return launch_tile_1d<MODE, ROT, true, true>(a, st);
+  return launch_tile_1d<MODE, ROT, false, true>(a, st);
 }
 
 // Launch the amax pass: rows into partials[0, npart), columns (rotated
@@ -675,13 +995,14 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   if (!rot) {
     amax_plain_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, make_fastdiv(static_cast<uint32_t>(a.C / 8)), pr);
   } else {
-    const int64_t ntiles = a.tiles_r * a.tiles_c;
+    const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+    const FastDiv tcd = a.tiles_c_div;
     if (row && col)
-      amax_tile_kernel<true, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
+      amax_tile_kernel<true, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else if (row)
-      amax_tile_kernel<true, false><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
+      amax_tile_kernel<true, false><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else
-      amax_tile_kernel<false, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, a.tiles_c, ntiles, a.seed, pr, pc);
+      amax_tile_kernel<false, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
   }
   note_launch();
   return cudaGetLastError();
@@ -713,6 +1034,7 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   a.nb_row = make_fastdiv(static_cast<uint32_t>(C / 16));
   a.tiles_r = (R + TR - 1) / TR;
   a.tiles_c = (C + TC - 1) / TC;
+  a.tiles_c_div = make_fastdiv(static_cast<uint32_t>(a.tiles_c > 0 ? a.tiles_c : 1));
   const bool row = flags & kRowwise, col = flags & kColwise, two_d = flags & kBlock2D;
   const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || (flags & kRht)) && !two_d;
   if (rot) a.partials_col = a.partials + a.npart;
