@@ -635,14 +635,25 @@ __global__ void __launch_bounds__(TNT) quant_tile_kernel(const QuantArgs a) {
 // quantize_block for two lane-paired blocks (x: block a, y: block b): the
 // same arithmetic, with the element-wise steps done two blocks at a time.
 // ---------------------------------------------------------------------------
+// Tree-shaped (depth 4) so the two chains of dependent max operations stay
+// short; max is exact, so the order does not matter.
 __device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
-  ma = 0.0f;
-  mb = 0.0f;
+  float a[8], b[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    ma = fmaxf(ma, fabsf(v[i].x));
-    mb = fmaxf(mb, fabsf(v[i].y));
+  for (int i = 0; i < 8; ++i) {
+    a[i] = fmaxf(fabsf(v[i].x), fabsf(v[i + 8].x));
+    b[i] = fmaxf(fabsf(v[i].y), fabsf(v[i + 8].y));
   }
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      a[i] = fmaxf(a[i], a[i + w]);
+      b[i] = fmaxf(b[i], b[i + w]);
+    }
+  }
+  ma = a[0];
+  mb = b[0];
 }
 
 // Word of the scale-SR draw that block blk uses: draw blk / 4, word blk % 4.
@@ -726,11 +737,16 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
 // Tiles stream through a ring of kTileStages shared-memory buffers (dynamic
 // shared memory), so up to kTileStages - 1 tiles are in flight per CTA while
 // one is processed.
-constexpr int kTileStages = 4;
+constexpr int kTileStages = 2;
 constexpr int kTileBytes = TR * TC * 2;
 
+// Resident CTAs per SM the register budget is sized for: the kernels are
+// bound by the latency of dependent arithmetic, so more warps help.
+template <int MODE>
+constexpr int tile_1d_min_blocks() { return (MODE == kModeRTN) ? 4 : 3; }
+
 template <int MODE, bool ROT, bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT, 2) quant_tile_1d_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
   extern __shared__ __align__(16) uint8_t tile_ring[];
   auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(tile_ring);
   __shared__ __align__(16) uint8_t colcodes[TC][kColPitch];
