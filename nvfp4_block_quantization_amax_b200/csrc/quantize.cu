@@ -248,7 +248,15 @@ __device__ __forceinline__ void tile_coords(uint32_t tile, const FastDiv& tiles_
   tc = tile - q * tiles_c.d;
 }
 
-// Issue the copies of tile `tile` (row-major tile grid) into buf.
+// 2D-block layout: chunk c of row r at slot c ^ (r & 7), so that the eight
+// lanes reading one chunk column of eight consecutive rows hit 32 distinct
+// banks, as do 32 lanes reading 32 consecutive words of one row.
+__device__ __forceinline__ int tile_chunk_2d(int r, int c) { return c ^ (r & 7); }
+__device__ __forceinline__ int tile_word_2d(int r, int w) { return (tile_chunk_2d(r, w >> 2) << 2) | (w & 3); }
+
+// Issue the copies of tile `tile` (row-major tile grid) into buf, in the
+// 1D (SW2D = false) or the 2D-block (SW2D = true) layout.
+template <bool SW2D = false>
 __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
                                                 int64_t ld, const FastDiv& tiles_c, uint32_t tile) {
   int64_t tr, tc;
@@ -260,7 +268,8 @@ __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint
   for (int i = 0; i < 4; ++i) {
     const int ch = threadIdx.x + TNT * i;
     const int row = ch >> 4, cc = ch & 15;
-    if (row < rows && 8 * cc < cols) cp_async16(&buf[row][tile_chunk(row, cc)], x + (r0 + row) * ld + c0 + 8 * cc);
+    const int slot = SW2D ? tile_chunk_2d(row, cc) : tile_chunk(row, cc);
+    if (row < rows && 8 * cc < cols) cp_async16(&buf[row][slot], x + (r0 + row) * ld + c0 + 8 * cc);
   }
   cp_async_commit();
 }
@@ -363,273 +372,7 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
   }
 }
 
-// ===========================================================================
-// Rowwise quantization, streamed: one thread per 16-element block.
-// ===========================================================================
-template <int MODE, bool ROT, int NT>
-__global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
-  __shared__ uint32_t red[NT / 32];
-  float alpha, alpha_unused;
-  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red);
-  const PhiloxKeys K = philox_keys(a.seed);
-  uint32_t signs = 0;
-  if constexpr (ROT) signs = sign_bits(K);
-  const uint32_t c2 = a.stream_id * 2u;
-  const uint32_t nb = a.nb_row.d;
-  const uint32_t total = static_cast<uint32_t>(a.R) * nb;
-  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
-  const bool check = (a.flags & kAlphaProvided) != 0;
-  for (uint32_t k = blockIdx.x * NT + threadIdx.x; k < total; k += gridDim.x * NT) {
-    const uint32_t r = fastdiv(k, a.nb_row), cb = k - r * nb;
-    const uint4* p = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(r) * a.ld + 16 * cb);
-    const uint4 u0 = __ldcs(p), u1 = __ldcs(p + 1);
-    float v[16];
-    unpack8(u0, v);
-    unpack8(u1, v + 8);
-    if (check) {
-      bool bad = false;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) bad |= abs_bits(v[i]) >= 0x7F800000u;
-      if (bad && a.status) *a.status = kStatusNonFinite;
-    }
-    if constexpr (ROT) rht16(v, signs);
-    uint32_t sb;
-    const Packed16 q = quantize_block<MODE>(v, alpha, K, c2, k, sb);
-    *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(r) * (a.C / 2) + 8 * cb) =
-        make_uint2(q.lo, q.hi);
-    if (a.scales_row) {
-      const int64_t off = gemm ? gemm_scale_offset(r, cb, nb) : static_cast<int64_t>(k);
-      a.scales_row[off] = static_cast<uint8_t>(sb);
-    }
-  }
-}
-
-// ===========================================================================
-// Tiled quantization: columns, dual rows + columns, and 2D 16x16 blocks.
-// Tile: 64 rows x 128 columns of bf16 (16 KB) in shared memory.
-// ===========================================================================
 constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
-
-struct TileSmem {
-  uint4 tile[TR][TC / 8];                   // 64 x 256 B
-  uint8_t colcodes[TC][kColPitch];          // transposed codes, 32 B per column
-  uint8_t colscale[TC][TR / 16];            // column scales of the tile
-  uint8_t scale2d[TR / 16][TC / 16];        // chosen 2D scales
-};
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-}
-
-// 16 bf16 of row `row`, column block `cb` of the smem tile, read as two
-// 16-byte halves in a lane-dependent order so eight lanes hit eight distinct
-// bank groups.
-__device__ __forceinline__ void tile_row_block(const TileSmem& s, int row, int cb, float* v) {
-  const int first = (cb >> 2) & 1;
-  const uint4 h0 = s.tile[row][2 * cb + first];
-  const uint4 h1 = s.tile[row][2 * cb + (first ^ 1)];
-  if (first) {
-    unpack8(h1, v);
-    unpack8(h0, v + 8);
-  } else {
-    unpack8(h0, v);
-    unpack8(h1, v + 8);
-  }
-}
-
-template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
-__global__ void __launch_bounds__(TNT) quant_tile_kernel(const QuantArgs a) {
-  __shared__ TileSmem s;
-  __shared__ uint32_t red[TNT / 32];
-  float alpha_r, alpha_c;
-  // 2D tiles share one tensor scale (the plain amax, which both orientations
-  // read from the same partials) between orientations.
-  resolve_alpha<TNT>(a, ROW || TWO_D, COL, ROW, COL, alpha_r, alpha_c, red);
-  if constexpr (TWO_D) alpha_c = alpha_r;
-  const PhiloxKeys K = philox_keys(a.seed);
-  uint32_t signs = 0;
-  if constexpr (ROT) signs = sign_bits(K);
-  const uint32_t c2r = a.stream_id * 2u, c2c = a.stream_id * 2u + 1u;
-  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
-  const bool check = (a.flags & kAlphaProvided) != 0;
-  const int t = threadIdx.x;
-  const int64_t R = a.R, C = a.C;
-  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
-
-  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    int64_t tr, tc;
-    tile_coords(tile, a.tiles_c_div, tr, tc);
-    const int64_t r0 = tr * TR, c0 = tc * TC;
-    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);   // multiple of 16
-    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);   // multiple of 16
-
-    // ---- load the tile (16-byte async copies, 4 per thread) ----
-    __syncthreads();  // previous tile fully consumed
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int ch = t + TNT * i;
-      const int row = ch >> 4, cc = ch & 15;
-      if (row < rows && 8 * cc < cols)
-        cp_async16(&s.tile[row][cc], a.x + (r0 + row) * a.ld + c0 + 8 * cc);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-
-    if (check) {
-      bool bad = false;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int ch = t + TNT * i;
-        const int row = ch >> 4, cc = ch & 15;
-        if (row < rows && 8 * cc < cols) {
-          float v[8];
-          unpack8(s.tile[row][cc], v);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) bad |= abs_bits(v[j]) >= 0x7F800000u;
-        }
-      }
-      if (bad && a.status) *a.status = kStatusNonFinite;
-    }
-
-    if constexpr (TWO_D) {
-      // ---- 2D blocks: 16 lanes per 16x16 block, one row each ----
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int task = t + TNT * i;
-        const int bb = task >> 4, lr = task & 15;
-        const int rb = bb >> 3, cbb = bb & 7;
-        const bool valid = (16 * rb < rows) && (16 * cbb < cols);  // uniform per half-warp
-        float v[16];
-        if (valid) tile_row_block(s, 16 * rb + lr, cbb, v);
-        else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        }
-        float m = max_abs16(v);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        const uint32_t sb6 = e4m3_rne(scale_raw(m, alpha_r, 6.0f));
-        Packed16 p = encode_rne(v, alpha_r, sb6);
-        uint32_t sb = sb6;
-        if constexpr (MODE == kModeFourSix) {
-          const uint32_t sb4 = e4m3_rne(scale_raw(m, alpha_r, 4.0f));
-          const Packed16 p4 = encode_rne(v, alpha_r, sb4);
-          float e6 = sq_error(v, alpha_r, sb6, p);
-          float e4 = sq_error(v, alpha_r, sb4, p4);
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) {
-            e6 = __fadd_rn(e6, __shfl_xor_sync(0xFFFFFFFFu, e6, o));
-            e4 = __fadd_rn(e4, __shfl_xor_sync(0xFFFFFFFFu, e4, o));
-          }
-          if (e4 < e6) {
-            sb = sb4;
-            p = p4;
-          }
-        }
-        if (valid) {
-          const int64_t grow = r0 + 16 * rb + lr;
-          const int64_t gcb = c0 / 16 + cbb;
-          if (lr == 0) s.scale2d[rb][cbb] = static_cast<uint8_t>(sb);
-          if constexpr (ROW) {
-            *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(p.lo, p.hi);
-            if (a.scales_row) {
-              if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sb);
-              else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sb);
-            }
-          }
-        }
-      }
-      __syncthreads();
-    }
-
-    if constexpr (ROW && !TWO_D) {
-      // ---- row blocks: 64 rows x 8 blocks, two per thread ----
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int task = t + TNT * i;
-        const int row = task >> 3, cb = task & 7;
-        if (row < rows && 16 * cb < cols) {
-          float v[16];
-          tile_row_block(s, row, cb, v);
-          if constexpr (ROT) rht16(v, signs);
-          const int64_t grow = r0 + row, gcb = c0 / 16 + cb;
-          const uint64_t blk = static_cast<uint64_t>(grow) * (C / 16) + gcb;
-          uint32_t sb;
-          const Packed16 q = quantize_block<MODE>(v, alpha_r, K, c2r, blk, sb);
-          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(q.lo, q.hi);
-          if (a.scales_row)
-            a.scales_row[gemm ? gemm_scale_offset(grow, gcb, C / 16) : static_cast<int64_t>(blk)] =
-                static_cast<uint8_t>(sb);
-        }
-      }
-    }
-
-    if constexpr (COL) {
-      // ---- column blocks: 4 row-blocks x 128 columns; a thread owns a
-      //      column pair of one row-block ----
-      const int cp = t & 63, rb = t >> 6;
-      if (16 * rb < rows && 2 * cp < cols) {
-        float v0[16], v1[16];
-        const uint32_t* base = reinterpret_cast<const uint32_t*>(&s.tile[16 * rb][0]) + cp;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t w = base[i * (TC / 2)];
-          v0[i] = bf16lo(w);
-          v1[i] = bf16hi(w);
-        }
-        uint32_t sb0, sb1;
-        Packed16 q0, q1;
-        if constexpr (TWO_D) {
-          sb0 = sb1 = s.scale2d[rb][cp >> 3];
-          q0 = encode_rne(v0, alpha_c, sb0);
-          q1 = encode_rne(v1, alpha_c, sb1);
-        } else {
-          if constexpr (ROT) {
-            rht16(v0, signs);
-            rht16(v1, signs);
-          }
-          const int64_t nbc = R / 16;
-          const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
-          q0 = quantize_block<MODE>(v0, alpha_c, K, c2c, static_cast<uint64_t>(gc) * nbc + grb, sb0);
-          q1 = quantize_block<MODE>(v1, alpha_c, K, c2c, static_cast<uint64_t>(gc + 1) * nbc + grb, sb1);
-        }
-        *reinterpret_cast<uint2*>(&s.colcodes[2 * cp][8 * rb]) = make_uint2(q0.lo, q0.hi);
-        *reinterpret_cast<uint2*>(&s.colcodes[2 * cp + 1][8 * rb]) = make_uint2(q1.lo, q1.hi);
-        s.colscale[2 * cp][rb] = static_cast<uint8_t>(sb0);
-        s.colscale[2 * cp + 1][rb] = static_cast<uint8_t>(sb1);
-      }
-      __syncthreads();
-      // ---- write the transposed codes: column c of the tile is 32 bytes
-      //      (rows/2 valid) of output row c0 + c ----
-      {
-        const int c = t >> 1, h = t & 1;
-        const int nbytes = rows / 2;
-        if (c < cols && 16 * h < nbytes) {
-          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
-          const uint2* src = reinterpret_cast<const uint2*>(&s.colcodes[c][16 * h]);
-          const uint2 lo = src[0];
-          reinterpret_cast<uint2*>(dst)[0] = lo;
-          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
-        }
-      }
-      if (a.scales_col) {
-        const int c = t >> 1;
-        if (c < cols) {
-          for (int rb = (t & 1); rb < rows / 16; rb += 2) {
-            const int64_t gc = c0 + c, grb = r0 / 16 + rb;
-            const uint8_t sb = s.colscale[c][rb];
-            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sb;
-            else if (TWO_D) {
-              if ((c & 15) == 0) a.scales_col[(gc / 16) * (R / 16) + grb] = sb;
-            } else {
-              a.scales_col[gc * (R / 16) + grb] = sb;
-            }
-          }
-        }
-      }
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // quantize_block for two lane-paired blocks (x: block a, y: block b): the
@@ -654,14 +397,6 @@ __device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& m
   }
   ma = a[0];
   mb = b[0];
-}
-
-// Word of the scale-SR draw that block blk uses: draw blk / 4, word blk % 4.
-__device__ __forceinline__ uint32_t eden_word(const PhiloxKeys& K, uint32_t c2, uint64_t blk) {
-  const uint64_t unit = blk >> 2;
-  const uint4 w = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
-  const uint32_t sel = static_cast<uint32_t>(blk & 3);
-  return sel == 0 ? w.x : (sel == 1 ? w.y : (sel == 2 ? w.z : w.w));
 }
 
 // MS-EDEN scale of one block from its sums and its random word.
@@ -709,8 +444,13 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
     const float2 num = sum16x2(rr);
     const float2 den = mul2(make_float2(alpha, alpha), sum16x2(rq));
     if (!have_words) {
-      wa = eden_word(K, c2, blka);
-      wb = eden_word(K, c2, blkb);
+      const uint64_t ua = blka >> 2, ub = blkb >> 2;
+      const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagScaleSR);
+      const uint4 db =
+          (ua == ub) ? da : philox(K, static_cast<uint32_t>(ub), static_cast<uint32_t>(ub >> 32), c2, kTagScaleSR);
+      const uint32_t sa = static_cast<uint32_t>(blka & 3), sbw = static_cast<uint32_t>(blkb & 3);
+      wa = sa == 0 ? da.x : (sa == 1 ? da.y : (sa == 2 ? da.z : da.w));
+      wb = sbw == 0 ? db.x : (sbw == 1 ? db.y : (sbw == 2 ? db.z : db.w));
     }
     sba = eden_scale(num.x, den.x, wa);
     sbb = eden_scale(num.y, den.y, wb);
@@ -723,6 +463,66 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
     }
     pa = quantize_block<MODE>(a, alpha, K, c2, blka, sba);
     pb = quantize_block<MODE>(b, alpha, K, c2, blkb, sbb);
+  }
+}
+
+// ===========================================================================
+// Rowwise quantization, streamed: a thread takes the consecutive blocks 2k
+// and 2k + 1 of the row-major block order (64 contiguous bytes when they
+// share a row) and quantizes them lane-paired.  Both lie in MS-EDEN draw
+// unit k / 2, so one draw serves the pair.
+// ===========================================================================
+template <int MODE, bool ROT, int NT>
+__global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
+  __shared__ uint32_t red[NT / 32];
+  float alpha, alpha_unused;
+  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red);
+  const PhiloxKeys K = philox_keys(a.seed);
+  SignMasks sm;
+  if constexpr (ROT) {
+    sm = sign_masks(sign_bits(K));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sm.m[i] = 0u;
+  }
+  const uint32_t c2 = a.stream_id * 2u;
+  const uint32_t nb = a.nb_row.d;
+  const uint32_t total = static_cast<uint32_t>(a.R) * nb;
+  const uint32_t npairs = (total + 1) / 2;
+  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
+  const bool check = (a.flags & kAlphaProvided) != 0;
+  for (uint32_t pk = blockIdx.x * NT + threadIdx.x; pk < npairs; pk += gridDim.x * NT) {
+    const uint32_t ka = 2 * pk, kb = ka + 1;
+    const bool vb = kb < total;
+    const uint32_t ra = fastdiv(ka, a.nb_row), cba = ka - ra * nb;
+    const uint32_t kk = vb ? kb : ka;
+    const uint32_t rb = fastdiv(kk, a.nb_row), cbb = kk - rb * nb;
+    const uint4* pa = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(ra) * a.ld + 16 * cba);
+    const uint4* pb = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(rb) * a.ld + 16 * cbb);
+    const uint4 a0 = __ldcs(pa), a1 = __ldcs(pa + 1), b0 = __ldcs(pb), b1 = __ldcs(pb + 1);
+    if (check) {
+      uint32_t hin = 0;
+      const uint32_t w[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
+                              b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) hin = __vmaxu2(hin, w[i] & 0x7FFF7FFFu);
+      if (max(hin & 0xFFFFu, hin >> 16) >= 0x7F80u && a.status) *a.status = kStatusNonFinite;
+    }
+    float2 v[16];
+    unpack16x2_signed(a0, a1, b0, b1, sm, v);
+    if constexpr (ROT) rht16x2_presigned(v);
+    Packed16 qa, qb;
+    uint32_t sa, sb;
+    quantize_pair<MODE>(v, alpha, K, c2, ka, kb, qa, qb, sa, sb);
+    *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(ra) * (a.C / 2) + 8 * cba) = make_uint2(qa.lo, qa.hi);
+    if (a.scales_row)
+      a.scales_row[gemm ? gemm_scale_offset(ra, cba, nb) : static_cast<int64_t>(ka)] = static_cast<uint8_t>(sa);
+    if (vb) {
+      *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(rb) * (a.C / 2) + 8 * cbb) =
+          make_uint2(qb.lo, qb.hi);
+      if (a.scales_row)
+        a.scales_row[gemm ? gemm_scale_offset(rb, cbb, nb) : static_cast<int64_t>(kb)] = static_cast<uint8_t>(sb);
+    }
   }
 }
 
@@ -933,6 +733,193 @@ __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d
 }
 
 // ===========================================================================
+// Tiled 2D quantization: 16 x 16 blocks share one scale (rows of a 16-lane
+// half-warp, one tile row each), two blocks per thread lane-paired:
+// thread t takes row t % 16 of blocks (t / 128, (t / 16) % 8) and
+// (t / 128 + 2, (t / 16) % 8) of the tile's 4 x 8 block grid.  The column
+// orientation reuses the chosen block scales on the transposed blocks.
+// ===========================================================================
+template <int MODE, bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT, 3) quant_tile_2d_kernel(const QuantArgs a) {
+  extern __shared__ __align__(16) uint8_t tile_ring[];
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(tile_ring);
+  __shared__ __align__(16) uint8_t colcodes[TC][kColPitch];
+  __shared__ uint8_t scale2d[TR / 16][TC / 16];
+  __shared__ uint32_t red[TNT / 32];
+  float alpha, alpha_c;
+  // one tensor scale for both orientations: the plain amax, whose partials
+  // both orientations read (alpha_c == alpha; it is computed to publish it)
+  resolve_alpha<TNT>(a, true, COL, ROW, COL, alpha, alpha_c, red);
+  const bool gemm = (a.flags & kGemmScaleLayout) != 0;
+  const bool check = (a.flags & kAlphaProvided) != 0;
+  const int t = threadIdx.x;
+  const int64_t R = a.R, C = a.C;
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+
+  uint32_t tile = blockIdx.x;
+#pragma unroll
+  for (int k = 0; k < kTileStages - 1; ++k) {
+    const uint32_t tk = tile + k * gridDim.x;
+    if (tk < ntiles) load_tile_async<true>(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
+    else cp_async_commit();
+  }
+  int buf = 0;
+  for (; tile < ntiles; tile += gridDim.x, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
+    const uint32_t ahead = tile + (kTileStages - 1) * gridDim.x;
+    const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;
+    if (ahead < ntiles) load_tile_async<true>(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
+    else cp_async_commit();
+    cp_async_wait<kTileStages - 1>();
+    __syncthreads();
+    const uint4 (*s)[TC / 8] = tiles[buf];
+    int64_t tr, tc;
+    tile_coords(tile, a.tiles_c_div, tr, tc);
+    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);   // multiple of 16
+    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);   // multiple of 16
+
+    if (check) {
+      uint32_t hin = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ch = t + TNT * i;
+        const int row = ch >> 4, cc = ch & 15;
+        if (row < rows && 8 * cc < cols) {
+          const uint4 u = s[row][tile_chunk_2d(row, cc)];
+          hin = __vmaxu2(hin, u.x & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.y & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.z & 0x7FFF7FFFu);
+          hin = __vmaxu2(hin, u.w & 0x7FFF7FFFu);
+        }
+      }
+      if (max(hin & 0xFFFFu, hin >> 16) >= 0x7F80u && a.status) *a.status = kStatusNonFinite;
+    }
+
+    {
+      const int rb = t >> 7, cbb = (t >> 4) & 7, lr = t & 15;
+      const int rowa = 16 * rb + lr, rowb = rowa + 32;
+      // uniform per half-warp (rows and cols are multiples of 16)
+      const bool va = 16 * rb < rows && 16 * cbb < cols, vb = 16 * rb + 32 < rows && 16 * cbb < cols;
+      const uint4 a0 = s[rowa][tile_chunk_2d(rowa, 2 * cbb)], a1 = s[rowa][tile_chunk_2d(rowa, 2 * cbb + 1)];
+      const uint4 b0 = s[rowb][tile_chunk_2d(rowb, 2 * cbb)], b1 = s[rowb][tile_chunk_2d(rowb, 2 * cbb + 1)];
+      SignMasks none;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) none.m[i] = 0u;
+      float2 v[16];
+      unpack16x2_signed(a0, a1, b0, b1, none, v);
+      if (!va) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i].x = 0.0f;
+      }
+      if (!vb) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i].y = 0.0f;
+      }
+      float ma, mb;
+      max_abs16x2(v, ma, mb);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        ma = fmaxf(ma, __shfl_xor_sync(0xFFFFFFFFu, ma, o));
+        mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+      }
+      uint32_t sa = e4m3_rne(scale_raw(ma, alpha, 6.0f)), sb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+      Packed16 pa, pb;
+      encode_rne_x2(v, alpha, sa, sb, pa, pb);
+      if constexpr (MODE == kModeFourSix) {
+        const uint32_t sa4 = e4m3_rne(scale_raw(ma, alpha, 4.0f)), sb4 = e4m3_rne(scale_raw(mb, alpha, 4.0f));
+        Packed16 pa4, pb4;
+        encode_rne_x2(v, alpha, sa4, sb4, pa4, pb4);
+        float2 e6 = sq_error_x2(v, alpha, sa, sb, pa, pb);
+        float2 e4 = sq_error_x2(v, alpha, sa4, sb4, pa4, pb4);
+        // block error = the half-warp's row errors summed in butterfly order
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          e6.x = __fadd_rn(e6.x, __shfl_xor_sync(0xFFFFFFFFu, e6.x, o));
+          e6.y = __fadd_rn(e6.y, __shfl_xor_sync(0xFFFFFFFFu, e6.y, o));
+          e4.x = __fadd_rn(e4.x, __shfl_xor_sync(0xFFFFFFFFu, e4.x, o));
+          e4.y = __fadd_rn(e4.y, __shfl_xor_sync(0xFFFFFFFFu, e4.y, o));
+        }
+        if (e4.x < e6.x) {
+          sa = sa4;
+          pa = pa4;
+        }
+        if (e4.y < e6.y) {
+          sb = sb4;
+          pb = pb4;
+        }
+      }
+      const int64_t gcb = c0 / 16 + cbb;
+      if (va) {
+        const int64_t grow = r0 + rowa;
+        if (lr == 0) scale2d[rb][cbb] = static_cast<uint8_t>(sa);
+        if constexpr (ROW) {
+          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
+          if (a.scales_row) {
+            if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sa);
+            else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sa);
+          }
+        }
+      }
+      if (vb) {
+        const int64_t grow = r0 + rowb;
+        if (lr == 0) scale2d[rb + 2][cbb] = static_cast<uint8_t>(sb);
+        if constexpr (ROW) {
+          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(pb.lo, pb.hi);
+          if (a.scales_row) {
+            if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sb);
+            else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sb);
+          }
+        }
+      }
+    }
+
+    if constexpr (COL) {
+      __syncthreads();   // scale2d complete
+      // columns (2 cp, 2 cp + 1) of row block rb, both in 16-column block cp / 8
+      const int cp = t & 63, rb = t >> 6;
+      if (16 * rb < rows && 2 * cp < cols) {
+        const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
+        float2 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = base[i * (TC / 2) + tile_word_2d(i, cp)];   // row 16 rb + i: (16 rb + i) & 7 == i & 7
+          v[i] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+        }
+        const uint32_t sbyte = scale2d[rb][cp >> 3];
+        Packed16 qa, qb;
+        encode_rne_x2(v, alpha, sbyte, sbyte, qa, qb);
+        *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
+        *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
+      }
+      __syncthreads();
+      {
+        const int c = t >> 1, h = t & 1;
+        const int nbytes = rows / 2;
+        if (c < cols && 16 * h < nbytes) {
+          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
+          const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
+          reinterpret_cast<uint2*>(dst)[0] = src[0];
+          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+        }
+      }
+      if (a.scales_col) {
+        const int c = t >> 1;
+        if (c < cols) {
+          for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
+            const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
+            const uint8_t sbyte = scale2d[rb2][c >> 4];
+            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
+            else if ((c & 15) == 0) a.scales_col[(gc / 16) * (R / 16) + grb] = sbyte;
+          }
+        }
+      }
+    }
+    __syncthreads();   // buf, scale2d and the staging are reused
+  }
+  cp_async_wait<0>();
+}
+
+// ===========================================================================
 // Host-side launchers
 // ===========================================================================
 static int g_sm_count[64] = {0};
@@ -958,18 +945,29 @@ size_t quant_workspace_bytes(int64_t, int64_t, uint32_t flags) {
 
 template <int MODE, bool ROT>
 static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
-  const uint32_t total = static_cast<uint32_t>(a.R) * a.nb_row.d;
-  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
+  const uint32_t pairs = (static_cast<uint32_t>(a.R) * a.nb_row.d + 1) / 2;
+  const int blocks = static_cast<int>(std::min<int64_t>((pairs + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
   quant_rows_kernel<MODE, ROT, 256><<<std::max(blocks, 1), 256, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
 
-template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
-static cudaError_t launch_tile(const QuantArgs& a, cudaStream_t st) {
+template <int MODE, bool ROW, bool COL>
+static cudaError_t launch_tile_2d(const QuantArgs& a, cudaStream_t st) {
+  constexpr size_t smem = static_cast<size_t>(kTileStages) * kTileBytes;
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    cudaFuncSetAttribute(quant_tile_2d_kernel<MODE, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tile_2d_kernel<MODE, ROW, COL>, TNT, smem) !=
+            cudaSuccess || n <= 0)
+      n = 1;
+    per_sm = n;
+  }
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
-  const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 6));
-  quant_tile_kernel<MODE, ROT, ROW, COL, TWO_D><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
+  quant_tile_2d_kernel<MODE, ROW, COL><<<std::max(blocks, 1), TNT, smem, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1062,13 +1060,13 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   }
   if (two_d) {
     if (mode == kModeRTN) {
-      if (row && col) return launch_tile<kModeRTN, false, true, true, true>(a, st);
-      if (row) return launch_tile<kModeRTN, false, true, false, true>(a, st);
-      return launch_tile<kModeRTN, false, false, true, true>(a, st);
+      if (row && col) return launch_tile_2d<kModeRTN, true, true>(a, st);
+      if (row) return launch_tile_2d<kModeRTN, true, false>(a, st);
+      return launch_tile_2d<kModeRTN, false, true>(a, st);
     }
-    if (row && col) return launch_tile<kModeFourSix, false, true, true, true>(a, st);
-    if (row) return launch_tile<kModeFourSix, false, true, false, true>(a, st);
-    return launch_tile<kModeFourSix, false, false, true, true>(a, st);
+    if (row && col) return launch_tile_2d<kModeFourSix, true, true>(a, st);
+    if (row) return launch_tile_2d<kModeFourSix, true, false>(a, st);
+    return launch_tile_2d<kModeFourSix, false, true>(a, st);
   }
   switch (mode) {
     case kModeRTN:
