@@ -81,7 +81,14 @@ typedef enum {
 #define NVFP4_ROWWISE 0x1u          /* blocks along C (the contiguous axis)      */
 #define NVFP4_COLWISE 0x2u          /* blocks along R; output is the transpose   */
 #define NVFP4_BLOCK2D 0x4u          /* 16x16 blocks (weights, [NV] §二); RTN/4-6 */
-#define NVFP4_SINGLE_PASS 0x8u      /* amax and quantize in one cooperative pass */
+#define NVFP4_SINGLE_PASS 0x8u      /* amax and quantize in one cooperative launch:
+                                     * per-CTA maxima, a grid barrier (bounded:
+                                     * 1 s, then NVFP4_ERR_TIMEOUT in *status and
+                                     * no outputs), then the encoding; results
+                                     * identical to the two-pass call.  Needs 16
+                                     * more workspace bytes (the barrier counter,
+                                     * cleared by the call).  Pays off for small
+                                     * tensors (one launch, the re-read from L2). */
 #define NVFP4_ALPHA_PROVIDED 0x10u  /* use *alpha_in instead of Eq. 1            */
 #define NVFP4_GEMM_SCALE_LAYOUT 0x20u /* write scales in nvfp4_gemm's layout     */
 #define NVFP4_RHT 0x40u             /* rotate before RTN / FOUR_SIX encoding     */

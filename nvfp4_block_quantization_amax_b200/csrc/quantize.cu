@@ -45,6 +45,7 @@ struct QuantArgs {
   FastDiv nb_row;                 // C / 16
   int64_t tiles_r, tiles_c;       // tile grid (tile kernels)
   FastDiv tiles_c_div;            // divides a tile index by tiles_c
+  FastDiv chunks_row;             // C / 8: 16-byte chunks per row (plain amax)
 };
 
 constexpr uint32_t kNonFinite = 0xFFFFFFFFu;   // partial marker: a NaN / Inf was read
@@ -80,11 +81,11 @@ __device__ __forceinline__ uint32_t reduce_partials(const uint32_t* p, int n, ui
 template <int NT>
 __device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, bool need_c,
                                               bool pub_r, bool pub_c, float& alpha_r,
-                                              float& alpha_c, uint32_t* red) {
+                                              float& alpha_c, uint32_t* red, uint32_t cta) {
   if (a.flags & kAlphaProvided) {
     const float al = __ldg(a.alpha_in);
     alpha_r = alpha_c = al;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (cta == 0 && threadIdx.x == 0) {
       if (!(al >= 0.0f && al <= 3.402823466e38f) && a.status) *a.status = kStatusArg;
       if (pub_r && a.alpha_row) *a.alpha_row = al;
       if (pub_c && a.alpha_col) *a.alpha_col = al;
@@ -99,7 +100,7 @@ __device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, b
   const float amax_c = __uint_as_float(mc == kNonFinite ? 0u : mc);
   alpha_r = __fdiv_rn(amax_r, 2688.0f);
   alpha_c = __fdiv_rn(amax_c, 2688.0f);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (cta == 0 && threadIdx.x == 0) {
     if ((mr == kNonFinite || mc == kNonFinite) && a.status) *a.status = kStatusNonFinite;
     if (pub_r && a.alpha_row) *a.alpha_row = alpha_r;
     if (pub_c && a.alpha_col) *a.alpha_col = alpha_c;
@@ -185,17 +186,17 @@ __device__ __forceinline__ Packed16 quantize_block(const float* v, float alpha,
 // sign cleared, so two are compared at once with a per-halfword unsigned
 // max; a pattern >= 0x7F80 is an Inf or a NaN.
 template <int NT>
-__global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t ld,
-                                                        FastDiv cpr, uint32_t* __restrict__ partial) {
-  __shared__ uint32_t red[NT / 32];
+__device__ __forceinline__ void amax_plain_body(const uint16_t* __restrict__ x, int64_t R, int64_t ld, FastDiv cpr,
+                                                uint32_t* __restrict__ partial, uint32_t cta, uint32_t ncta,
+                                                uint32_t* red) {
   const uint32_t total = static_cast<uint32_t>(R) * cpr.d;   // chunks of 8 values
-  const uint32_t stride = gridDim.x * NT;
+  const uint32_t stride = ncta * NT;
   uint32_t hm = 0;
   auto chunk = [&](uint32_t k) {
     const uint32_t r = fastdiv(k, cpr), c = k - r * cpr.d;
     return __ldcs(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * ld) + c);
   };
-  uint32_t k = blockIdx.x * NT + threadIdx.x;
+  uint32_t k = cta * NT + threadIdx.x;
   for (; k + 3 * stride < total; k += 4 * stride) {
     uint4 u[4];
 #pragma unroll
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restri
   const uint32_t h = max(hm & 0xFFFFu, hm >> 16);
   uint32_t m = (h >= 0x7F80u) ? kNonFinite : (h << 16);
   m = block_max_u32<NT>(m, red);
-  if (threadIdx.x == 0) partial[blockIdx.x] = m;
+  if (threadIdx.x == 0) partial[cta] = m;
 }
 
 // Tiles of 64 x 128 bf16 staged in shared memory, two buffers so the next
@@ -280,21 +281,20 @@ __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint
 // 1/4: round-to-nearest multiplication is monotone, so the maximum of the
 // scaled magnitudes is the scaled maximum, applied once per CTA.
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                        int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
-                                                        uint32_t* __restrict__ part_r,
-                                                        uint32_t* __restrict__ part_c) {
-  __shared__ __align__(16) uint4 tiles[2][TR][TC / 8];
-  __shared__ uint32_t red[TNT / 32];
+__device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, int64_t R, int64_t C, int64_t ld,
+                                               FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
+                                               uint32_t* __restrict__ part_r, uint32_t* __restrict__ part_c,
+                                               uint32_t cta, uint32_t ncta, uint8_t* ring, uint32_t* red) {
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);   // two tile buffers
   const SignMasks sm = sign_masks(sign_bits(philox_keys(seed)));
   const int t = threadIdx.x;
   float mr = 0.0f, mc = 0.0f;
   uint32_t hin = 0;   // per-halfword max of the input magnitudes (Inf / NaN check)
-  uint32_t tile = blockIdx.x;
+  uint32_t tile = cta;
   int buf = 0;
   if (tile < ntiles) load_tile_async(tiles[0], x, R, C, ld, tiles_c, tile);
-  for (; tile < ntiles; tile += gridDim.x, buf ^= 1) {
-    const uint32_t next = tile + gridDim.x;
+  for (; tile < ntiles; tile += ncta, buf ^= 1) {
+    const uint32_t next = tile + ncta;
     if (next < ntiles) {
       load_tile_async(tiles[buf ^ 1], x, R, C, ld, tiles_c, next);
       cp_async_wait<1>();
@@ -363,12 +363,12 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
   if constexpr (ROW) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mr, 0.25f));
     m = block_max_u32<TNT>(m, red);
-    if (t == 0) part_r[blockIdx.x] = m;
+    if (t == 0) part_r[cta] = m;
   }
   if constexpr (COL) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mc, 0.25f));
     m = block_max_u32<TNT>(m, red);
-    if (t == 0) part_c[blockIdx.x] = m;
+    if (t == 0) part_c[cta] = m;
   }
 }
 
@@ -473,10 +473,9 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
 // unit k / 2, so one draw serves the pair.
 // ===========================================================================
 template <int MODE, bool ROT, int NT>
-__global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
-  __shared__ uint32_t red[NT / 32];
+__device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint32_t* red) {
   float alpha, alpha_unused;
-  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red);
+  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red, cta);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -491,7 +490,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
   const uint32_t npairs = (total + 1) / 2;
   const bool gemm = (a.flags & kGemmScaleLayout) != 0;
   const bool check = (a.flags & kAlphaProvided) != 0;
-  for (uint32_t pk = blockIdx.x * NT + threadIdx.x; pk < npairs; pk += gridDim.x * NT) {
+  for (uint32_t pk = cta * NT + threadIdx.x; pk < npairs; pk += ncta * NT) {
     const uint32_t ka = 2 * pk, kb = ka + 1;
     const bool vb = kb < total;
     const uint32_t ra = fastdiv(ka, a.nb_row), cba = ka - ra * nb;
@@ -545,15 +544,23 @@ constexpr int kTileBytes = TR * TC * 2;
 template <int MODE>
 constexpr int tile_1d_min_blocks() { return (MODE == kModeRTN) ? 4 : 3; }
 
+// Shared memory of the tile kernels besides the tile ring.
+struct TileStaging {
+  uint8_t colcodes[TC][kColPitch];   // transposed column codes of one tile
+  uint8_t colscale[TC][TR / 16];     // their scales (2D: unused)
+  uint8_t scale2d[TR / 16][TC / 16]; // chosen 16x16 scales (2D)
+  uint32_t red[TNT / 32];
+};
+
 template <int MODE, bool ROT, bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
-  extern __shared__ __align__(16) uint8_t tile_ring[];
-  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(tile_ring);
-  __shared__ __align__(16) uint8_t colcodes[TC][kColPitch];
-  __shared__ uint8_t colscale[TC][TR / 16];
-  __shared__ uint32_t red[TNT / 32];
+__device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint8_t* ring,
+                                                   TileStaging& stg) {
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);
+  auto& colcodes = stg.colcodes;
+  auto& colscale = stg.colscale;
+  uint32_t* red = stg.red;
   float alpha_r, alpha_c;
-  resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red);
+  resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -579,16 +586,16 @@ __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d
 
   // prologue: the first kTileStages - 1 tiles (an empty copy group when a
   // tile does not exist keeps the group count in step)
-  uint32_t tile = blockIdx.x;
+  uint32_t tile = cta;
 #pragma unroll
   for (int k = 0; k < kTileStages - 1; ++k) {
-    const uint32_t tk = tile + k * gridDim.x;
+    const uint32_t tk = tile + k * ncta;
     if (tk < ntiles) load_tile_async(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
     else cp_async_commit();
   }
   int buf = 0;
-  for (; tile < ntiles; tile += gridDim.x, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
-    const uint32_t ahead = tile + (kTileStages - 1) * gridDim.x;
+  for (; tile < ntiles; tile += ncta, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
+    const uint32_t ahead = tile + (kTileStages - 1) * ncta;
     const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;   // (buf + kTileStages - 1) % kTileStages
     if (ahead < ntiles) load_tile_async(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
     else cp_async_commit();
@@ -740,32 +747,32 @@ __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d
 // orientation reuses the chosen block scales on the transposed blocks.
 // ===========================================================================
 template <int MODE, bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT, 3) quant_tile_2d_kernel(const QuantArgs a) {
-  extern __shared__ __align__(16) uint8_t tile_ring[];
-  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(tile_ring);
-  __shared__ __align__(16) uint8_t colcodes[TC][kColPitch];
-  __shared__ uint8_t scale2d[TR / 16][TC / 16];
-  __shared__ uint32_t red[TNT / 32];
+__device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint8_t* ring,
+                                                   TileStaging& stg) {
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);
+  auto& colcodes = stg.colcodes;
+  auto& scale2d = stg.scale2d;
+  uint32_t* red = stg.red;
   float alpha, alpha_c;
   // one tensor scale for both orientations: the plain amax, whose partials
   // both orientations read (alpha_c == alpha; it is computed to publish it)
-  resolve_alpha<TNT>(a, true, COL, ROW, COL, alpha, alpha_c, red);
+  resolve_alpha<TNT>(a, true, COL, ROW, COL, alpha, alpha_c, red, cta);
   const bool gemm = (a.flags & kGemmScaleLayout) != 0;
   const bool check = (a.flags & kAlphaProvided) != 0;
   const int t = threadIdx.x;
   const int64_t R = a.R, C = a.C;
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
 
-  uint32_t tile = blockIdx.x;
+  uint32_t tile = cta;
 #pragma unroll
   for (int k = 0; k < kTileStages - 1; ++k) {
-    const uint32_t tk = tile + k * gridDim.x;
+    const uint32_t tk = tile + k * ncta;
     if (tk < ntiles) load_tile_async<true>(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
     else cp_async_commit();
   }
   int buf = 0;
-  for (; tile < ntiles; tile += gridDim.x, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
-    const uint32_t ahead = tile + (kTileStages - 1) * gridDim.x;
+  for (; tile < ntiles; tile += ncta, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
+    const uint32_t ahead = tile + (kTileStages - 1) * ncta;
     const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;
     if (ahead < ntiles) load_tile_async<true>(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
     else cp_async_commit();
@@ -920,6 +927,116 @@ __global__ void __launch_bounds__(TNT, 3) quant_tile_2d_kernel(const QuantArgs a
 }
 
 // ===========================================================================
+// Kernels.  Each wraps one body above with its own shared memory; the
+// single-pass kernel runs an amax body and a quantize body in one launch.
+// ===========================================================================
+template <int NT>
+__global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t ld,
+                                                        FastDiv cpr, uint32_t* __restrict__ partial) {
+  __shared__ uint32_t red[NT / 32];
+  amax_plain_body<NT>(x, R, ld, cpr, partial, blockIdx.x, gridDim.x, red);
+}
+
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                        int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
+                                                        uint32_t* __restrict__ part_r,
+                                                        uint32_t* __restrict__ part_c) {
+  __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
+  __shared__ uint32_t red[TNT / 32];
+  amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, part_r, part_c, blockIdx.x, gridDim.x, ring, red);
+}
+
+template <int MODE, bool ROT, int NT>
+__global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
+  __shared__ uint32_t red[NT / 32];
+  quant_rows_body<MODE, ROT, NT>(a, blockIdx.x, gridDim.x, red);
+}
+
+template <int MODE, bool ROT, bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
+  extern __shared__ __align__(16) uint8_t tile_ring[];
+  __shared__ __align__(16) TileStaging stg;
+  quant_tile_1d_body<MODE, ROT, ROW, COL>(a, blockIdx.x, gridDim.x, tile_ring, stg);
+}
+
+template <int MODE, bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT, 3) quant_tile_2d_kernel(const QuantArgs a) {
+  extern __shared__ __align__(16) uint8_t tile_ring[];
+  __shared__ __align__(16) TileStaging stg;
+  quant_tile_2d_body<MODE, ROW, COL>(a, blockIdx.x, gridDim.x, tile_ring, stg);
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t load_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+constexpr uint64_t kBarrierTimeoutNs = 1000000000ull;   // 1 s
+
+// Grid-wide barrier of a cooperative launch: every CTA's thread 0 releases
+// its writes, counts itself in, and waits (at most kBarrierTimeoutNs) until
+// all `n` CTAs are in.  The counter starts at 0 (the launcher clears it).
+// Returns false, with NVFP4_ERR_TIMEOUT in the status word, if the wait ran
+// out; the caller then returns without touching its outputs.
+__device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, int32_t* status, uint32_t* ok_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+    const uint64_t t0 = global_ns();
+    uint32_t ok = 1;
+    while (load_acquire_gpu(counter) < n) {
+      if (global_ns() - t0 > kBarrierTimeoutNs) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    if (!ok && status) *status = kStatusTimeout;
+    *ok_smem = ok;
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
+// Single pass: amax partials (one per CTA), a grid barrier, then the
+// quantization, all in one cooperative launch whose CTAs are co-resident.
+// For tensors that fit in L2 the quantize pass re-reads from L2, not HBM.
+template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
+__global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, uint32_t* counter) {
+  extern __shared__ __align__(16) uint8_t tile_ring[];
+  __shared__ __align__(16) TileStaging stg;
+  __shared__ uint32_t pass_ok;
+  const uint32_t cta = blockIdx.x, ncta = gridDim.x;
+  if (!(a.flags & kAlphaProvided)) {
+    uint32_t* pr = const_cast<uint32_t*>(a.partials);
+    uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
+    if constexpr (ROT) {
+      amax_tile_body<ROW, COL>(a.x, a.R, a.C, a.ld, a.tiles_c_div, static_cast<uint32_t>(a.tiles_r * a.tiles_c),
+                               a.seed, pr, pc, cta, ncta, tile_ring, stg.red);
+    } else {
+      amax_plain_body<TNT>(a.x, a.R, a.ld, a.chunks_row, pr, cta, ncta, stg.red);
+    }
+    if (!grid_barrier(counter, ncta, a.status, &pass_ok)) return;
+  }
+  if constexpr (TWO_D) {
+    quant_tile_2d_body<MODE, ROW, COL>(a, cta, ncta, tile_ring, stg);
+  } else if constexpr (ROW && !COL) {
+    quant_rows_body<MODE, ROT, TNT>(a, cta, ncta, stg.red);
+  } else {
+    quant_tile_1d_body<MODE, ROT, ROW, COL>(a, cta, ncta, tile_ring, stg);
+  }
+}
+
+// ===========================================================================
 // Host-side launchers
 // ===========================================================================
 static int g_sm_count[64] = {0};
@@ -938,9 +1055,12 @@ int sm_count() {
 
 int amax_partial_count() { return 4 * 148; }
 
+// Workspace: the amax partials of both orientations, then (single pass) the
+// grid barrier's counter in its own 16-byte slot.
 size_t quant_workspace_bytes(int64_t, int64_t, uint32_t flags) {
   if (flags & kAlphaProvided) return 0;
-  return static_cast<size_t>(2 * amax_partial_count()) * sizeof(uint32_t);
+  const size_t partials = static_cast<size_t>(2 * amax_partial_count()) * sizeof(uint32_t);
+  return (flags & kSinglePass) ? partials + 16 : partials;
 }
 
 template <int MODE, bool ROT>
@@ -999,6 +1119,38 @@ static cudaError_t dispatch_1d(const QuantArgs& a, bool row, bool col, cudaStrea
   return launch_tile_1d<MODE, ROT, false, true>(a, st);
 }
 
+template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
+static cudaError_t launch_single_pass(QuantArgs a, cudaStream_t st) {
+  auto fn = single_pass_kernel<MODE, ROT, ROW, COL, TWO_D>;
+  constexpr size_t smem = static_cast<size_t>(kTileStages) * kTileBytes;   // >= the amax pass's two tiles
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, TNT, smem) != cudaSuccess || n <= 0) n = 1;
+    per_sm = n;
+  }
+  // every CTA must be resident at once (the barrier), and each writes one
+  // partial per orientation
+  const int grid = std::min(sm_count() * per_sm, amax_partial_count());
+  uint32_t* counter = const_cast<uint32_t*>(a.partials) + 2 * amax_partial_count();
+  a.npart = grid;
+  if (a.partials_col != a.partials) a.partials_col = a.partials + amax_partial_count();
+  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  void* args[] = {&a, &counter};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(TNT), args, smem, st);
+  note_launch();
+  return e;
+}
+
+template <int MODE, bool ROT>
+static cudaError_t dispatch_single_1d(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
+  if (row && !col) return launch_single_pass<MODE, ROT, true, false, false>(a, st);
+  if (row && col) return launch_single_pass<MODE, ROT, true, true, false>(a, st);
+  return launch_single_pass<MODE, ROT, false, true, false>(a, st);
+}
+
 // Launch the amax pass: rows into partials[0, npart), columns (rotated
 // only) into partials[npart, 2 npart).  Plain amax is shared by both
 // orientations.
@@ -1007,7 +1159,7 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   uint32_t* pr = const_cast<uint32_t*>(a.partials);
   uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
   if (!rot) {
-    amax_plain_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, make_fastdiv(static_cast<uint32_t>(a.C / 8)), pr);
+    amax_plain_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.chunks_row, pr);
   } else {
     const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
     const FastDiv tcd = a.tiles_c_div;
@@ -1049,10 +1201,36 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   a.tiles_r = (R + TR - 1) / TR;
   a.tiles_c = (C + TC - 1) / TC;
   a.tiles_c_div = make_fastdiv(static_cast<uint32_t>(a.tiles_c > 0 ? a.tiles_c : 1));
+  a.chunks_row = make_fastdiv(static_cast<uint32_t>(C / 8 > 0 ? C / 8 : 1));
   const bool row = flags & kRowwise, col = flags & kColwise, two_d = flags & kBlock2D;
   const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || (flags & kRht)) && !two_d;
   if (rot) a.partials_col = a.partials + a.npart;
   if (R == 0 || C == 0) return cudaSuccess;
+
+  if ((flags & kSinglePass) && !(flags & kAlphaProvided)) {
+    if (two_d) {
+      if (mode == kModeRTN) {
+        if (row && col) return launch_single_pass<kModeRTN, false, true, true, true>(a, st);
+        if (row) return launch_single_pass<kModeRTN, false, true, false, true>(a, st);
+        return launch_single_pass<kModeRTN, false, false, true, true>(a, st);
+      }
+      if (row && col) return launch_single_pass<kModeFourSix, false, true, true, true>(a, st);
+      if (row) return launch_single_pass<kModeFourSix, false, true, false, true>(a, st);
+      return launch_single_pass<kModeFourSix, false, false, true, true>(a, st);
+    }
+    switch (mode) {
+      case kModeRTN:
+        return rot ? dispatch_single_1d<kModeRTN, true>(a, row, col, st)
+                   : dispatch_single_1d<kModeRTN, false>(a, row, col, st);
+      case kModeFourSix:
+        return rot ? dispatch_single_1d<kModeFourSix, true>(a, row, col, st)
+                   : dispatch_single_1d<kModeFourSix, false>(a, row, col, st);
+      case kModeRhtSR:
+        return dispatch_single_1d<kModeRhtSR, true>(a, row, col, st);
+      default:
+        return dispatch_single_1d<kModeMsEden, true>(a, row, col, st);
+    }
+  }
 
   if (!(flags & kAlphaProvided)) {
     cudaError_t e = launch_amax(a, row || two_d, col && !two_d, rot, st);

@@ -70,6 +70,13 @@ def test_host_argument_checks_need_no_gpu(lib):
     assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_ERR_WORKSPACE
     assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE) > 0
     assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE | L.NVFP4_ALPHA_PROVIDED) == 0
+    # single pass: the partials plus a 16-byte slot for the grid barrier's counter
+    two = L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE)
+    assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE | L.NVFP4_SINGLE_PASS) == two + 16
+    assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE | L.NVFP4_SINGLE_PASS | L.NVFP4_ALPHA_PROVIDED) == 0
+    # single pass is checked like the two-pass call (here: its workspace is missing)
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE | L.NVFP4_SINGLE_PASS, 0, 0, None, out, None, 0,
+                            None) == L.NVFP4_ERR_WORKSPACE
     # empty tensors are a no-op
     assert L.nvfp4_quantize(None, 0, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_OK
     # dequantize / gemm checks

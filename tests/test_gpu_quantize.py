@@ -308,3 +308,85 @@ def test_full_size_rotated_rtn_requantization(api, layer8b):
     # features, X along tokens (columns), RTN with the gradient's sign vector
     _sampled_rows_check(api, layer8b["w"], 0, COL | RHT, seed=1002, stream_id=2, nsample=8)
     _sampled_rows_check(api, layer8b["x"], 0, COL | RHT, seed=1002, stream_id=3, nsample=8)
+
+
+# ---------------------------------------------------------------------------
+# Single pass (NVFP4_SINGLE_PASS): amax, a grid barrier and the quantization
+# in one cooperative launch.  Same results as the two-pass path, bit for bit,
+# so the same oracle comparisons apply.
+# ---------------------------------------------------------------------------
+SP = 0x8
+
+
+def assert_amax(g, o, flags):
+    if flags & ROW:
+        assert float(g["amax"][0]) == o["amax_row"]
+    if flags & COL:
+        assert float(g["amax"][1]) == o["amax_col"]
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("orient", ["row", "col", "dual"])
+def test_single_pass_all_modes(api, pr1, mode, orient):
+    flags = {"row": ROW, "col": COL, "dual": ROW | COL}[orient] | SP
+    g, o, _ = run_both(api, pr1["x"], MODES[mode], flags, seed=1234, stream_id=3)
+    assert_same(g, o, flags)
+    assert_amax(g, o, flags)
+
+
+@pytest.mark.parametrize("mode", ["rtn", "four_six"])
+@pytest.mark.parametrize("extra", [RHT, B2D, B2D | GEMM])
+def test_single_pass_rotated_and_2d(api, pr1, mode, extra):
+    flags = ROW | COL | SP | extra
+    x = pr1["w"] if extra & B2D else pr1["x"]
+    g, o, _ = run_both(api, x, MODES[mode], flags, seed=77)
+    assert_same(g, o, flags)
+
+
+@pytest.mark.parametrize("shape", [(48, 144), (37, 48), (1, 16), (80, 272), (1040, 1552)])
+@pytest.mark.parametrize("mode", list(MODES))
+def test_single_pass_ragged_and_many_tiles(api, shape, mode):
+    R, C = shape
+    x = synthetic.normal_with_entry_outliers(R, C, seed=R * 1000 + C + 1)
+    flags = (ROW | COL if R % 16 == 0 else ROW) | SP
+    g, o, _ = run_both(api, x, MODES[mode], flags, seed=6, stream_id=2)
+    assert_same(g, o, flags)
+    assert_amax(g, o, flags)
+
+
+def test_single_pass_equals_two_pass_full_size(api, layer8b):
+    # the dY dual MS-EDEN call of the step, GEMM scale layout, both ways
+    dy = layer8b["dy"].cuda()
+    flags = ROW | COL | GEMM
+    a = api.nvfp4_quantize(dy, 3, flags, seed=11, stream_id=1)
+    b = api.nvfp4_quantize(dy, 3, flags | SP, seed=11, stream_id=1)
+    torch.cuda.synchronize()
+    for name in ("codes_row", "scales_row", "alpha_row", "codes_col", "scales_col", "alpha_col", "amax"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    # and sampled rows of it against the oracle
+    _sampled_rows_check(api, layer8b["dy"], 3, ROW | COL | SP, seed=12, stream_id=1, nsample=4)
+
+
+def test_single_pass_nonfinite_sets_status(api):
+    x = torch.randn(64, 128, dtype=torch.bfloat16, device="cuda")
+    x[5, 3] = float("nan")
+    for mode, flags in ((0, ROW), (3, ROW | COL), (1, ROW | B2D)):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        api.nvfp4_quantize(x, mode, flags | SP, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == -4, (mode, flags)
+
+
+def test_single_pass_workspace_is_scratch(api, pr1):
+    # the barrier counter is cleared by the call itself: a workspace full of
+    # garbage, reused call after call, gives the same result
+    x = pr1["x"].cuda()
+    R, C = x.shape
+    ws = torch.full((api.workspace_for(R, C, ROW | COL | SP, x.device).numel(),), 0x7B,
+                    dtype=torch.uint8, device="cuda")
+    ref = api.nvfp4_quantize(x, 3, ROW | COL, seed=3)
+    for _ in range(3):
+        q = api.nvfp4_quantize(x, 3, ROW | COL | SP, seed=3, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(q.codes_row, ref.codes_row) and torch.equal(q.codes_col, ref.codes_col)
+        assert torch.equal(q.scales_row, ref.scales_row) and torch.equal(q.scales_col, ref.scales_col)
