@@ -207,11 +207,18 @@ __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
 // Lane-paired arithmetic: two independent blocks share each float2 (x = the
 // first block's element, y = the second's), so one packed sm_100 instruction
 // does the work of two.  Each component is rounded exactly as the scalar
-// __f*_rn operation.  a - b is formed as fma(b, -1, a): the product b * -1 is
-// exact, so the single rounding gives RN(a - b), signed zeros included.
+// __f*_rn operation.
+// sub2 forms a - b as fma(b, -1, a): the product b * -1 is exact, so the one
+// rounding gives RN(a - b), signed zeros included.  It is for operands that
+// are sums (the butterflies): when b is itself a product, the compiler may
+// fold the two into one fma and drop the product's rounding, so a - RN(p)
+// uses sub2_exact (two scalar subtractions, which are never merged).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+__device__ __forceinline__ float2 sub2_exact(float2 a, float2 b) {
+  return make_float2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y));
+}
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // Sign masks of the rotation's diagonal: bit 31 set where element i flips.
@@ -454,11 +461,15 @@ __device__ __forceinline__ void decode16x2(const Packed16& pa, const Packed16& p
   for (int i = 0; i < 16; ++i) q[i] = make_float2(a[i], b[i]);
 }
 
-// sum16 of two lane-paired blocks.
+// sum16 of two lane-paired blocks of products.  The packed multiply that
+// made e[] may be contracted with a packed add into one fma (measured: the
+// rounding of d * d vanished from 4/6 errors), so the first level, which
+// consumes the products, adds with the scalar __fadd_rn, which is never
+// merged; the later levels add sums only.
 __device__ __forceinline__ float2 sum16x2(const float2* e) {
   float2 t[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = add2(e[i], e[i + 8]);
+  for (int i = 0; i < 8; ++i) t[i] = make_float2(__fadd_rn(e[i].x, e[i + 8].x), __fadd_rn(e[i].y, e[i + 8].y));
 #pragma unroll
   for (int i = 0; i < 4; ++i) t[i] = add2(t[i], t[i + 4]);
 #pragma unroll
@@ -474,7 +485,7 @@ __device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint
   decode16x2(pa, pb, q);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float2 d = sub2(v[i], mul2(q[i], s2));
+    const float2 d = sub2_exact(v[i], mul2(q[i], s2));
     e[i] = mul2(d, d);
   }
   return sum16x2(e);

@@ -390,3 +390,21 @@ def test_single_pass_workspace_is_scratch(api, pr1):
         torch.cuda.synchronize()
         assert torch.equal(q.codes_row, ref.codes_row) and torch.equal(q.codes_col, ref.codes_col)
         assert torch.equal(q.scales_row, ref.scales_row) and torch.equal(q.scales_col, ref.scales_col)
+
+
+def test_four_six_near_tie_blocks(api):
+    # Two blocks of the 4096 x 1024 sweep tensor whose M = 4 and M = 6 squared
+    # errors lie two ulps apart (0.119696319 vs 0.119696334 for the first):
+    # the selector must see exactly the oracle's rounded products q * s.
+    blocks = [[0.337890625, -1.2109375, 0.5078125, -1.8515625, -0.056640625, -1.5390625, -0.328125, 0.462890625,
+               -1.828125, 0.294921875, -0.9453125, 0.6796875, -0.45703125, 0.400390625, 1.1015625, 0.447265625],
+              [-1.578125, 0.05615234375, -1.03125, 1.046875, -2.203125, 0.26171875, 0.90625, -0.10595703125,
+               -1.265625, 0.65234375, -0.5234375, -0.1689453125, 0.69921875, -0.478515625, 0.93359375, -0.99609375]]
+    alpha = float(np.float32(0.0714285746216774))
+    a = np.zeros((64, 128), np.float32)
+    a[0, :16], a[33, 32:48] = blocks[0], blocks[1]   # rows 0 / 33: both lanes of a row pair
+    a[17, 16:32] = blocks[1]
+    x = synthetic.to_bf16(a)
+    for flags in (ROW, ROW | COL, COL):
+        g, o, _ = run_both(api, x if flags != COL else synthetic.to_bf16(a.T.copy()), 1, flags, alpha=alpha)
+        assert_same(g, o, flags)
