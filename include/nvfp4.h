@@ -214,6 +214,30 @@ NVFP4_API nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const f
                           int64_t ldd, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* nvfp4_gemm whose epilogue also quantizes the output for the next layer
+ * ([NV] §九 counts the separate amax and quantize passes over an activation
+ * as overhead; here the output is encoded while it is still in registers):
+ *   D_bf16 = the bf16 result nvfp4_gemm would write (same arithmetic);
+ *   codes [M, N/2], scales: exactly what
+ *     nvfp4_quantize(D_bf16, mode, NVFP4_ROWWISE | NVFP4_ALPHA_PROVIDED | flags,
+ *                    alpha_in = alpha_out)
+ *     writes (16-element blocks along N; mode NVFP4_RTN or NVFP4_FOUR_SIX;
+ *     flags: 0 or NVFP4_GEMM_SCALE_LAYOUT, the scales then [M, N/16] row-major
+ *     or in the GEMM layout);
+ *   amax_out (optional device float): max |D_bf16| over the whole output,
+ *     from which a caller forms the next call's tensor scale amax / 2688
+ *     (delayed scaling: the pages' Eq. 1 applied one step late);
+ *   D (optional, bf16, row stride ldd): written only when not NULL.
+ * alpha_out is a device float (the tensor scale of Eq. 1 for this output).
+ * M % 256 == 0, N % 256 == 0, K % 128 == 0; pointers 16-byte aligned.  The
+ * workspace is optional as for nvfp4_gemm (status word). */
+NVFP4_API nvfp4_status_t nvfp4_gemm_quantize(const uint8_t* A, const uint8_t* sA, const float* alphaA,
+                                   const uint8_t* B, const uint8_t* sB, const float* alphaB,
+                                   int64_t M, int64_t N, int64_t K, void* D, int64_t ldd,
+                                   nvfp4_mode_t mode, uint32_t flags, const float* alpha_out,
+                                   uint8_t* codes, uint8_t* scales, float* amax_out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Number of kernels this library has launched in the calling process since
  * it was loaded (all devices, all streams).  Instrumentation for callers that
  * account for their launches; not a page-defined operation. */

@@ -30,7 +30,7 @@ NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
 EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
-            "nvfp4_gemm", "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
+            "nvfp4_gemm", "nvfp4_gemm_quantize", "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
 
 
 class nvfp4_qtensor_t(ctypes.Structure):
@@ -65,6 +65,9 @@ def load(path=LIB_PATH):
     L.nvfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
     L.nvfp4_gemm.restype = ctypes.c_int
+    L.nvfp4_gemm_quantize.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, ctypes.c_int, u32, vp,
+                                      vp, vp, vp, vp, sz, vp]
+    L.nvfp4_gemm_quantize.restype = ctypes.c_int
     L.nvfp4_status_string.argtypes = [ctypes.c_int]
     L.nvfp4_status_string.restype = ctypes.c_char_p
     L.nvfp4_version.argtypes = []
@@ -102,6 +105,12 @@ def nvfp4_gemm(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, workspa
                workspace_bytes, stream):
     return int(load().nvfp4_gemm(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd,
                                  workspace, workspace_bytes, stream))
+
+
+def nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, flags, alpha_out, codes, scales,
+                        amax_out, workspace, workspace_bytes, stream):
+    return int(load().nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, flags, alpha_out,
+                                          codes, scales, amax_out, workspace, workspace_bytes, stream))
 
 
 def nvfp4_status_string(status):

@@ -123,3 +123,27 @@ def nvfp4_gemm(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch
                       D.stride(0), None, 0, _stream())
     _check(st, "nvfp4_gemm")
     return D
+
+
+def nvfp4_gemm_quantize(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch.Tensor,
+                        sB: torch.Tensor, alphaB: torch.Tensor, mode: int, alpha_out: torch.Tensor,
+                        flags: int = NVFP4_GEMM_SCALE_LAYOUT, write_d: bool = True,
+                        out: Optional[torch.Tensor] = None):
+    """nvfp4_gemm with the bf16 output also quantized rowwise in the epilogue
+    (RTN or FOUR_SIX, tensor scale alpha_out).  Returns (D or None, codes
+    [M, N/2], scales, amax [1])."""
+    M, K2 = A.shape
+    N = B.shape[0]
+    K = 2 * K2
+    dev = A.device
+    D = None
+    if write_d:
+        D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((M, N // 16), dtype=torch.uint8, device=dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    st = L.nvfp4_gemm_quantize(_p(A), _p(sA), _p(alphaA), _p(B), _p(sB), _p(alphaB), M, N, K,
+                               _p(D) if D is not None else None, D.stride(0) if D is not None else N,
+                               mode, flags, _p(alpha_out), _p(codes), _p(scales), _p(amax), None, 0, _stream())
+    _check(st, "nvfp4_gemm_quantize")
+    return D, codes, scales, amax

@@ -132,4 +132,30 @@ nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const float* alph
                                           static_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status_t nvfp4_gemm_quantize(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                                   const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
+                                   int64_t ldd, nvfp4_mode_t mode, uint32_t flags, const float* alpha_out,
+                                   uint8_t* codes, uint8_t* scales, float* amax_out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (mode != NVFP4_RTN && mode != NVFP4_FOUR_SIX) return NVFP4_ERR_ARG;
+  if (flags & ~NVFP4_GEMM_SCALE_LAYOUT) return NVFP4_ERR_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return NVFP4_ERR_SHAPE;
+  if (M % 256 || N % 256 || K % 128) return NVFP4_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (M * (N / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (D && ldd < N) return NVFP4_ERR_SHAPE;
+  if (!A || !sA || !alphaA || !B || !sB || !alphaB || !alpha_out || !codes || !scales) return NVFP4_ERR_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) || !aligned(sB, 16) || !aligned(codes, 16))
+    return NVFP4_ERR_ALIGN;
+  if (D && (!aligned(D, 16) || (ldd * 2) % 16)) return NVFP4_ERR_ALIGN;
+  if (amax_out && !aligned(amax_out, 4)) return NVFP4_ERR_ALIGN;
+  int32_t* status = (workspace && workspace_bytes >= sizeof(int32_t) && aligned(workspace, 4))
+                        ? static_cast<int32_t*>(workspace)
+                        : nullptr;
+  return launch_status(nvfp4::gemm_quantize_launch(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd,
+                                                   static_cast<int>(mode), (flags & NVFP4_GEMM_SCALE_LAYOUT) != 0,
+                                                   alpha_out, codes, scales, amax_out, status,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

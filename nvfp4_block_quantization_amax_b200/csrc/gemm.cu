@@ -30,8 +30,10 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
+#include "nvfp4_device.cuh"
 #include "nvfp4_internal.h"
 
 namespace nvfp4 {
@@ -546,11 +548,32 @@ constexpr uint32_t P_TMEM_COLS = 512;            // 256 accumulator + 2 x 4 K bl
 // M = 256 (>> 4 = 16 at bit 24), N = 256 (>> 3 = 32 at bit 17), E2M1 x E2M1, E4M3 scales
 constexpr uint32_t P_IDESC = (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
 
+// Optional NVFP4 quantization of the bf16 output rows in the epilogue (the
+// next layer's rowwise input), with a provided tensor scale.
+struct EpiQuant {
+  uint8_t* codes;        // [M, N/2]
+  uint8_t* scales;       // [M, N/16] row-major, or the GEMM scale layout
+  const float* alpha;    // tensor scale of the output (device)
+  uint32_t* amax;        // max |D| over the output (float bits), or null
+  int gemm_layout;
+  int write_d;           // also store D (bf16)
+};
+
+constexpr int kNoEpiQuant = -1;
+
+// Byte offset of the scale of (row m, K-block j) in the GEMM scale layout
+// (512-byte atoms of 128 rows x 4 K-blocks, K-atoms fastest).
+__device__ __forceinline__ int64_t gemm_scale_byte(int64_t m, int64_t j, int64_t kblocks) {
+  return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
+}
+
+template <int QMODE>
 __global__ void __launch_bounds__(P_THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
                            const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
-                           const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status) {
+                           const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status,
+                           const EpiQuant eq) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -685,6 +708,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     uint8_t* buf = sOut + (warp - 2) * 2048;
     const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
+    float eq_alpha = 0.0f, epi_amax = 0.0f;
+    if constexpr (QMODE != kNoEpiQuant) eq_alpha = __ldg(eq.alpha);
     int ti = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++ti) {
       const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
@@ -711,6 +736,36 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        if constexpr (QMODE != kNoEpiQuant) {
+          // this lane's output row, 8 blocks of 16 columns, two at a time,
+          // from the bf16 values just formed (exact in fp32)
+          const int64_t grow = row0 + lane;
+#pragma unroll
+          for (int jb = 0; jb < 8; jb += 2) {
+            float2 v[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t wa = packed[8 * jb + e], wb = packed[8 * jb + 8 + e];
+              v[2 * e] = make_float2(__uint_as_float(wa << 16), __uint_as_float(wb << 16));
+              v[2 * e + 1] = make_float2(__uint_as_float(wa & 0xFFFF0000u), __uint_as_float(wb & 0xFFFF0000u));
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) epi_amax = fmaxf(epi_amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+            Packed16 pa, pb;
+            uint32_t sa, sb;
+            quantize_pair_rne<QMODE == kModeFourSix>(v, eq_alpha, pa, pb, sa, sb);
+            const int64_t gcb = (col0 + 16 * jb) / 16;
+            *reinterpret_cast<uint4*>(eq.codes + grow * (N / 2) + 8 * gcb) = make_uint4(pa.lo, pa.hi, pb.lo, pb.hi);
+            if (eq.gemm_layout) {
+              eq.scales[gemm_scale_byte(grow, gcb, N / 16)] = static_cast<uint8_t>(sa);
+              eq.scales[gemm_scale_byte(grow, gcb + 1, N / 16)] = static_cast<uint8_t>(sb);
+            } else {
+              eq.scales[grow * (N / 16) + gcb] = static_cast<uint8_t>(sa);
+              eq.scales[grow * (N / 16) + gcb + 1] = static_cast<uint8_t>(sb);
+            }
+          }
+          if (!eq.write_d) continue;
+        }
 #pragma unroll
         for (int p = 0; p < 2; ++p) {        // 64-column pieces
 #pragma unroll
@@ -769,6 +824,13 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       }
     }
     if (lane == 0) bulk_wait_all();
+    if constexpr (QMODE != kNoEpiQuant) {
+      if (eq.amax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) epi_amax = fmaxf(epi_amax, __shfl_xor_sync(0xFFFFFFFFu, epi_amax, o));
+        if (lane == 0) atomicMax(eq.amax, __float_as_uint(epi_amax));
+      }
+    }
   }
   fence_before();
   __syncwarp();
@@ -866,21 +928,29 @@ bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int QMODE>
 cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                         const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
-                        int32_t* status, cudaStream_t st) {
+                        int32_t* status, const EpiQuant& eq, cudaStream_t st) {
   const bool fp32 = out_dtype == NVFP4_OUT_DTYPE_FP32;
   CUtensorMap ma, mb, md, msa, msb;
-  if (!make_map(&ma, A, M, K / 2, 128) || !make_map(&mb, B, N, K / 2, 128) ||
-      !make_out_map(&md, D, M, N, ldd, fp32) || !make_sf_map(&msa, sA, M, K) || !make_sf_map(&msb, sB, N, K))
+  std::memset(&md, 0, sizeof(md));   // unused when the epilogue writes no D
+  if (!make_map(&ma, A, M, K / 2, 128) || !make_map(&mb, B, N, K / 2, 128) || !make_sf_map(&msa, sA, M, K) ||
+      !make_sf_map(&msb, sB, N, K))
     return cudaErrorInvalidValue;
+  if (D && !make_out_map(&md, D, M, N, ldd, fp32)) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(nvfp4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
+  }
+  if (QMODE != kNoEpiQuant && eq.amax) {
+    cudaError_t e = cudaMemsetAsync(eq.amax, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
   }
   const int64_t tiles = (M / 256) * (N / 256);
   const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;  // persistent: one pair per TPC
@@ -896,9 +966,9 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel, ma, mb, md, msa, msb, alphaA, alphaB,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE>, ma, mb, md, msa, msb, alphaA, alphaB,
                                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                                     static_cast<int>(fp32), status);
+                                     static_cast<int>(fp32), status, eq);
   note_launch();
   return e;
 }
@@ -908,10 +978,24 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
 cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                         const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
                         int32_t* status, cudaStream_t st) {
-  if (M % 256 == 0 && N % 256 == 0)
-    return launch_pair(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
+  if (M % 256 == 0 && N % 256 == 0) {
+    const EpiQuant none{nullptr, nullptr, nullptr, nullptr, 0, 1};
+    return launch_pair<kNoEpiQuant>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, none, st);
+  }
   if (N % 256 == 0) return launch<256>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
   return launch<128>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
+}
+
+cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                                 const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
+                                 int64_t ldd, int mode, bool gemm_layout, const float* alpha_out, uint8_t* codes,
+                                 uint8_t* scales, float* amax_out, int32_t* status, cudaStream_t st) {
+  const EpiQuant eq{codes, scales, alpha_out, reinterpret_cast<uint32_t*>(amax_out), gemm_layout ? 1 : 0,
+                    D ? 1 : 0};
+  if (mode == kModeFourSix)
+    return launch_pair<kModeFourSix>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, NVFP4_OUT_DTYPE_BF16, ldd, status,
+                                     eq, st);
+  return launch_pair<kModeRTN>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, NVFP4_OUT_DTYPE_BF16, ldd, status, eq, st);
 }
 
 }  // namespace nvfp4

@@ -491,6 +491,56 @@ __device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint
   return sum16x2(e);
 }
 
+// Tree-shaped (depth 4) so the two chains of dependent max operations stay
+// short; max is exact, so the order does not matter.
+__device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
+  float a[8], b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    a[i] = fmaxf(fabsf(v[i].x), fabsf(v[i + 8].x));
+    b[i] = fmaxf(fabsf(v[i].y), fabsf(v[i + 8].y));
+  }
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      a[i] = fmaxf(a[i], a[i + w]);
+      b[i] = fmaxf(b[i], b[i + w]);
+    }
+  }
+  ma = a[0];
+  mb = b[0];
+}
+
+// Round-to-nearest block quantization of two lane-paired blocks (Four Over
+// Six §2.1 Eq. 2-3): scale for M = 6 (or, with four_six, the better of the
+// M = 6 and M = 4 candidates by squared error in the original domain, ties
+// to M = 6; §1 Table 1), then the E2M1 codes.
+template <bool FOUR_SIX>
+__device__ __forceinline__ void quantize_pair_rne(const float2* v, float alpha, Packed16& pa, Packed16& pb,
+                                                  uint32_t& sba, uint32_t& sbb) {
+  float ma, mb;
+  max_abs16x2(v, ma, mb);
+  if constexpr (!FOUR_SIX) {
+    sba = e4m3_rne(scale_raw(ma, alpha, 6.0f));
+    sbb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+    encode_rne_x2(v, alpha, sba, sbb, pa, pb);
+  } else {
+    const uint32_t a6 = e4m3_rne(scale_raw(ma, alpha, 6.0f)), b6 = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+    const uint32_t a4 = e4m3_rne(scale_raw(ma, alpha, 4.0f)), b4 = e4m3_rne(scale_raw(mb, alpha, 4.0f));
+    Packed16 pa6, pb6, pa4, pb4;
+    encode_rne_x2(v, alpha, a6, b6, pa6, pb6);
+    encode_rne_x2(v, alpha, a4, b4, pa4, pb4);
+    const float2 e6 = sq_error_x2(v, alpha, a6, b6, pa6, pb6);
+    const float2 e4 = sq_error_x2(v, alpha, a4, b4, pa4, pb4);
+    const bool ta = e4.x < e6.x, tb = e4.y < e6.y;
+    sba = ta ? a4 : a6;
+    pa = ta ? pa4 : pa6;
+    sbb = tb ? b4 : b6;
+    pb = tb ? pb4 : pb6;
+  }
+}
+
 // Unsigned division by a runtime constant d >= 1 for n < 2^32:
 // q = (n * mul) >> (32 + shift), mul = ceil(2^(32+shift) / d) (33 bits),
 // shift = ceil(log2 d).  The rounding error of mul is below d <= 2^shift, so

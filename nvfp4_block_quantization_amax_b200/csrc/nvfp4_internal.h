@@ -54,4 +54,13 @@ cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA
                         const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K,
                         void* D, int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st);
 
+// NVFP4 GEMM whose epilogue also quantizes the bf16 output rowwise (RTN or
+// FOUR_SIX, tensor scale *alpha_out): codes [M, N/2], scales (row-major or
+// GEMM layout), optional max |D| (amax_out, float).  D may be null.
+// Requires M % 256 == 0 and N % 256 == 0 (the CTA-pair kernel).
+cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                                 const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
+                                 int64_t ldd, int mode, bool gemm_layout, const float* alpha_out, uint8_t* codes,
+                                 uint8_t* scales, float* amax_out, int32_t* status, cudaStream_t st);
+
 }  // namespace nvfp4

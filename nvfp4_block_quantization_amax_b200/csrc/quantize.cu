@@ -378,27 +378,6 @@ constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
 // quantize_block for two lane-paired blocks (x: block a, y: block b): the
 // same arithmetic, with the element-wise steps done two blocks at a time.
 // ---------------------------------------------------------------------------
-// Tree-shaped (depth 4) so the two chains of dependent max operations stay
-// short; max is exact, so the order does not matter.
-__device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
-  float a[8], b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    a[i] = fmaxf(fabsf(v[i].x), fabsf(v[i + 8].x));
-    b[i] = fmaxf(fabsf(v[i].y), fabsf(v[i + 8].y));
-  }
-#pragma unroll
-  for (int w = 4; w > 0; w >>= 1) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      a[i] = fmaxf(a[i], a[i + w]);
-      b[i] = fmaxf(b[i], b[i + w]);
-    }
-  }
-  ma = a[0];
-  mb = b[0];
-}
-
 // MS-EDEN scale of one block from its sums and its random word.
 __device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t word) {
   if (den == 0.0f) return 0u;
@@ -411,26 +390,11 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
                                               uint64_t blka, uint64_t blkb, Packed16& pa, Packed16& pb,
                                               uint32_t& sba, uint32_t& sbb, bool have_words = false,
                                               uint32_t wa = 0u, uint32_t wb = 0u) {
-  float ma, mb;
-  max_abs16x2(v, ma, mb);
-  if constexpr (MODE == kModeRTN) {
-    sba = e4m3_rne(scale_raw(ma, alpha, 6.0f));
-    sbb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
-    encode_rne_x2(v, alpha, sba, sbb, pa, pb);
-  } else if constexpr (MODE == kModeFourSix) {
-    const uint32_t a6 = e4m3_rne(scale_raw(ma, alpha, 6.0f)), b6 = e4m3_rne(scale_raw(mb, alpha, 6.0f));
-    const uint32_t a4 = e4m3_rne(scale_raw(ma, alpha, 4.0f)), b4 = e4m3_rne(scale_raw(mb, alpha, 4.0f));
-    Packed16 pa6, pb6, pa4, pb4;
-    encode_rne_x2(v, alpha, a6, b6, pa6, pb6);
-    encode_rne_x2(v, alpha, a4, b4, pa4, pb4);
-    const float2 e6 = sq_error_x2(v, alpha, a6, b6, pa6, pb6);
-    const float2 e4 = sq_error_x2(v, alpha, a4, b4, pa4, pb4);
-    const bool ta = e4.x < e6.x, tb = e4.y < e6.y;
-    sba = ta ? a4 : a6;
-    pa = ta ? pa4 : pa6;
-    sbb = tb ? b4 : b6;
-    pb = tb ? pb4 : pb6;
+  if constexpr (MODE == kModeRTN || MODE == kModeFourSix) {
+    quantize_pair_rne<MODE == kModeFourSix>(v, alpha, pa, pb, sba, sbb);
   } else if constexpr (MODE == kModeMsEden) {
+    float ma, mb;
+    max_abs16x2(v, ma, mb);
     const uint32_t prova = e4m3_rne(scale_raw(ma, alpha, 6.0f));
     const uint32_t provb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
     encode_rne_x2(v, alpha, prova, provb, pa, pb);

@@ -85,3 +85,12 @@ def test_host_argument_checks_need_no_gpu(lib):
     assert L.nvfp4_gemm(fake, fake, fake, fake, fake, fake, 100, 128, 128, fake, 0, 128, None, 0, None) == L.NVFP4_ERR_SHAPE
     assert L.nvfp4_gemm(fake, fake, fake, fake, fake, fake, 128, 128, 128, fake, 5, 128, None, 0, None) == L.NVFP4_ERR_ARG
     assert L.nvfp4_gemm(None, fake, fake, fake, fake, fake, 128, 128, 128, fake, 0, 128, None, 0, None) == L.NVFP4_ERR_ARG
+    # gemm with epilogue quantization: RTN / FOUR_SIX only, CTA-pair shapes only
+    assert L.nvfp4_gemm_quantize(fake, fake, fake, fake, fake, fake, 256, 256, 128, None, 256, 3, 0, fake, fake,
+                                 fake, None, None, 0, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_gemm_quantize(fake, fake, fake, fake, fake, fake, 256, 384, 128, None, 384, 1, 0, fake, fake,
+                                 fake, None, None, 0, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_gemm_quantize(fake, fake, fake, fake, fake, fake, 256, 256, 128, None, 256, 1, 0x1, fake, fake,
+                                 fake, None, None, 0, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_gemm_quantize(fake, fake, fake, fake, fake, fake, 256, 256, 128, None, 256, 1, 0, None, fake,
+                                 fake, None, None, 0, None) == L.NVFP4_ERR_ARG

@@ -243,3 +243,65 @@ def test_dgrad_wgrad_8b_sampled(api, layer8b, mode):
     e = frob(got, ref)
     print(f"wgrad mode {mode} frob {e:.2e}")
     assert e <= FROB_TOL
+
+
+# ----------------------------------------- epilogue quantization (fused)
+def _fused_operands(api, M, N, K, seed):
+    a = synthetic.normal_with_channel_outliers(M, K, seed=seed)
+    w = synthetic.weight(N, K, seed=seed + 1)
+    qa = api.nvfp4_quantize(a.cuda(), 1, ROW | GEMM)
+    qw = api.nvfp4_quantize(w.cuda(), 1, ROW | B2D | GEMM)
+    return qa, qw
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 512, 384), (768, 1024, 2048)])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("layout", [0, GEMM])
+def test_gemm_quantize_epilogue_matches_quantize_of_output(api, M, N, K, mode, layout):
+    qa, qw = _fused_operands(api, M, N, K, seed=M + N + K)
+    ops = (qa.codes_row, qa.scales_row, qa.alpha_row, qw.codes_row, qw.scales_row, qw.alpha_row)
+    D_ref = api.nvfp4_gemm(*ops)
+    torch.cuda.synchronize()
+    # the output's tensor scale, as a caller would take it from the previous step
+    alpha_out = torch.tensor([float(D_ref.float().abs().max()) / 2688.0], dtype=torch.float32, device="cuda")
+    D, codes, scales, amax = api.nvfp4_gemm_quantize(*ops, mode, alpha_out, flags=layout)
+    torch.cuda.synchronize()
+    assert torch.equal(D, D_ref)
+    assert float(amax.item()) == float(D_ref.float().abs().max())
+    bits = synthetic.bf16_bits(D.cpu())
+    o = oracle.quantize(bits, mode, ROW, alpha=float(alpha_out.item()))
+    assert np.array_equal(codes.cpu().numpy(), o["codes_row"])
+    s = scales.cpu().numpy().reshape(-1)
+    if layout:
+        m = np.arange(M)[:, None]
+        j = np.arange(N // 16)[None, :]
+        kb = N // 16
+        off = ((m >> 7) * (kb >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3)
+        s = s[off]
+    else:
+        s = s.reshape(M, N // 16)
+    assert np.array_equal(s, o["scales_row"])
+    # without writing D: the same codes, scales and amax
+    D2, codes2, scales2, amax2 = api.nvfp4_gemm_quantize(*ops, mode, alpha_out, flags=layout, write_d=False)
+    torch.cuda.synchronize()
+    assert D2 is None
+    assert torch.equal(codes2, codes) and torch.equal(scales2, scales) and torch.equal(amax2, amax)
+
+
+def test_gemm_quantize_epilogue_8b_sampled(api, layer8b):
+    x, w = layer8b["x"], layer8b["w"]
+    qa = api.nvfp4_quantize(x.cuda(), 1, ROW | GEMM)
+    qw = api.nvfp4_quantize(w.cuda(), 1, ROW | B2D | GEMM)
+    ops = (qa.codes_row, qa.scales_row, qa.alpha_row, qw.codes_row, qw.scales_row, qw.alpha_row)
+    alpha_out = torch.tensor([0.37 / 2688.0], dtype=torch.float32, device="cuda")
+    D, codes, scales, amax = api.nvfp4_gemm_quantize(*ops, 1, alpha_out, flags=0)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(4)
+    rows = np.unique(np.concatenate([[0, D.shape[0] - 1], rng.integers(0, D.shape[0], 12)]))
+    bits = synthetic.bf16_bits(D[torch.as_tensor(rows, device="cuda")].cpu())
+    a = float(alpha_out.item())
+    for i, r in enumerate(rows):
+        c, s = oracle.quantize_1d_range(bits[i:i + 1], 0, 1, 0, 0, 0, a, 0, 1)
+        assert np.array_equal(codes[r].cpu().numpy(), c[0]), r
+        assert np.array_equal(scales[r].cpu().numpy(), s[0]), r
+    assert float(amax.item()) == float(D.float().abs().max())
