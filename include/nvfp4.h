@@ -92,6 +92,9 @@ typedef enum {
 #define NVFP4_ALPHA_PROVIDED 0x10u  /* use *alpha_in instead of Eq. 1            */
 #define NVFP4_GEMM_SCALE_LAYOUT 0x20u /* write scales in nvfp4_gemm's layout     */
 #define NVFP4_RHT 0x40u             /* rotate before RTN / FOUR_SIX encoding     */
+#define NVFP4_HEADROOM 0x200u       /* alpha = amax / (4 * 448) instead of Eq. 1's
+                                     * amax / (6 * 448): the M = 4 candidate of
+                                     * Four Over Six then never saturates        */
 /* nvfp4_dequantize flags (NVFP4_BLOCK2D and NVFP4_GEMM_SCALE_LAYOUT also apply) */
 #define NVFP4_INVERSE_RHT 0x80u     /* undo the rotation after decoding          */
 #define NVFP4_OUT_BF16 0x100u       /* write bf16 instead of fp32                */

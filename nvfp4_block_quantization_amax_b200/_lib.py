@@ -20,6 +20,7 @@ NVFP4_ROWWISE = 0x1
 NVFP4_COLWISE = 0x2
 NVFP4_BLOCK2D = 0x4
 NVFP4_SINGLE_PASS = 0x8
+NVFP4_HEADROOM = 0x200
 NVFP4_ALPHA_PROVIDED = 0x10
 NVFP4_GEMM_SCALE_LAYOUT = 0x20
 NVFP4_RHT = 0x40

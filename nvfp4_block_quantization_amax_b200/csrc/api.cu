@@ -9,7 +9,7 @@
 
 namespace {
 
-constexpr uint32_t kQuantFlags = NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_BLOCK2D | NVFP4_SINGLE_PASS |
+constexpr uint32_t kQuantFlags = NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_BLOCK2D | NVFP4_SINGLE_PASS | NVFP4_HEADROOM |
                                  NVFP4_ALPHA_PROVIDED | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_RHT;
 constexpr uint32_t kDequantFlags = NVFP4_BLOCK2D | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_INVERSE_RHT | NVFP4_OUT_BF16;
 

@@ -16,6 +16,7 @@ constexpr uint32_t kRowwise = NVFP4_ROWWISE;
 constexpr uint32_t kColwise = NVFP4_COLWISE;
 constexpr uint32_t kBlock2D = NVFP4_BLOCK2D;
 constexpr uint32_t kSinglePass = NVFP4_SINGLE_PASS;
+constexpr uint32_t kHeadroom = NVFP4_HEADROOM;
 constexpr uint32_t kAlphaProvided = NVFP4_ALPHA_PROVIDED;
 constexpr uint32_t kGemmScaleLayout = NVFP4_GEMM_SCALE_LAYOUT;
 constexpr uint32_t kRht = NVFP4_RHT;

@@ -95,11 +95,12 @@ __device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, b
   uint32_t mr = 0, mc = 0;
   if (need_r) mr = reduce_partials<NT>(a.partials, a.npart, red);
   if (need_c) mc = reduce_partials<NT>(a.partials_col, a.npart, red);
-  // Eq. 1: alpha = amax / (6 * 448)
+  // Eq. 1: alpha = amax / (6 * 448); with NVFP4_HEADROOM amax / (4 * 448)
   const float amax_r = __uint_as_float(mr == kNonFinite ? 0u : mr);
   const float amax_c = __uint_as_float(mc == kNonFinite ? 0u : mc);
-  alpha_r = __fdiv_rn(amax_r, 2688.0f);
-  alpha_c = __fdiv_rn(amax_c, 2688.0f);
+  const float den = (a.flags & kHeadroom) ? 1792.0f : 2688.0f;
+  alpha_r = __fdiv_rn(amax_r, den);
+  alpha_c = __fdiv_rn(amax_c, den);
   if (cta == 0 && threadIdx.x == 0) {
     if ((mr == kNonFinite || mc == kNonFinite) && a.status) *a.status = kStatusNonFinite;
     if (pub_r && a.alpha_row) *a.alpha_row = alpha_r;

@@ -18,6 +18,7 @@ import numpy as np
 from . import build as _build
 
 ROWWISE, COLWISE, BLOCK2D, ALPHA_PROVIDED, RHT, INVERSE_RHT = 0x1, 0x2, 0x4, 0x10, 0x40, 0x80
+HEADROOM = 0x200
 RTN, FOUR_SIX, RHT_SR, MS_EDEN = 0, 1, 2, 3
 OK, ERR_ARG, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -4
 
@@ -55,6 +56,8 @@ def lib():
         L.oracle_irht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
         L.oracle_alpha_from_amax.argtypes = [ctypes.c_float]
         L.oracle_alpha_from_amax.restype = ctypes.c_float
+        L.oracle_alpha_headroom.argtypes = [ctypes.c_float]
+        L.oracle_alpha_headroom.restype = ctypes.c_float
         L.oracle_amax.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_uint64, _f32p]
         L.oracle_amax.restype = ctypes.c_int
@@ -160,6 +163,10 @@ def irht16(r, signs):
 
 def alpha_from_amax(amax):
     return float(lib().oracle_alpha_from_amax(float(amax)))
+
+
+def alpha_headroom(amax):
+    return float(lib().oracle_alpha_headroom(float(amax)))
 
 
 # ---- tensor level ----------------------------------------------------------

@@ -49,6 +49,7 @@
 #define OR_COLWISE 0x2u
 #define OR_BLOCK2D 0x4u
 #define OR_ALPHA_PROVIDED 0x10u
+#define OR_HEADROOM 0x200u
 #define OR_RHT 0x40u
 #define OR_INVERSE_RHT 0x80u
 
@@ -261,6 +262,12 @@ static float sum16(const float e[16]) {
 /* Eq. 1: tensor scale alpha = amax / (6 * 448)  ([46] §2.1; [NV] §六).      */
 /* ------------------------------------------------------------------------ */
 float oracle_alpha_from_amax(float amax) { return amax / 2688.0f; }
+
+/* Headroom variant of Eq. 1: alpha = amax / (4 * 448).  Under Four Over Six
+ * the M = 4 candidate's raw scale amax_b / (alpha * 4) then stays within the
+ * E4M3 range instead of saturating at 448 (Eq. 2 with M = 4 and the plain
+ * Eq. 1 reaches 672). */
+float oracle_alpha_headroom(float amax) { return amax / 1792.0f; }
 
 /* Block encoding of 16 values (one 1D block) under candidate max M.         */
 typedef struct {
@@ -560,7 +567,8 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld,
     float amax = 0.0f;
     int st = oracle_amax(x, R, C, ld, o, rot, seed, &amax);
     if (st) return st;
-    float alpha = alpha_in ? *alpha_in : oracle_alpha_from_amax(amax);
+    float alpha = alpha_in ? *alpha_in
+                           : ((flags & OR_HEADROOM) ? oracle_alpha_headroom(amax) : oracle_alpha_from_amax(amax));
     if (o == 0) {
       if (amax_row) *amax_row = amax;
       if (alpha_row) *alpha_row = alpha;
@@ -578,7 +586,8 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld,
     float amax = 0.0f;
     int st = oracle_amax(x, R, C, ld, 0, 0, seed, &amax);
     if (st) return st;
-    float alpha = alpha_in ? *alpha_in : oracle_alpha_from_amax(amax);
+    float alpha = alpha_in ? *alpha_in
+                           : ((flags & OR_HEADROOM) ? oracle_alpha_headroom(amax) : oracle_alpha_from_amax(amax));
     oracle_quantize_2d(x, R, C, ld, mode, alpha, 0, R / 16,
                        want_row ? codes_row : NULL, want_row ? scales_row : NULL,
                        want_col ? codes_col : NULL, want_col ? scales_col : NULL);

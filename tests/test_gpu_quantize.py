@@ -13,6 +13,7 @@ from nvfp4_block_quantization_amax_b200 import synthetic
 pytestmark = pytest.mark.gpu
 
 ROW, COL, B2D, RHT, GEMM = 0x1, 0x2, 0x4, 0x40, 0x20
+HEADROOM = 0x200
 MODES = {"rtn": 0, "four_six": 1, "rht_sr": 2, "ms_eden": 3}
 
 
@@ -39,7 +40,7 @@ def run_both(api, x_t, mode, flags, seed=0, stream_id=0, alpha=None):
     q = api.nvfp4_quantize(x_dev, mode, flags, seed=seed, stream_id=stream_id, alpha=a_dev)
     torch.cuda.synchronize()
     bits = synthetic.bf16_bits(x_t)
-    o = oracle.quantize(bits, mode, flags & (ROW | COL | B2D | RHT), seed=seed, stream_id=stream_id,
+    o = oracle.quantize(bits, mode, flags & (ROW | COL | B2D | RHT | HEADROOM), seed=seed, stream_id=stream_id,
                         alpha=alpha)
     g = {}
     R, C = x_t.shape
@@ -408,3 +409,22 @@ def test_four_six_near_tie_blocks(api):
     for flags in (ROW, ROW | COL, COL):
         g, o, _ = run_both(api, x if flags != COL else synthetic.to_bf16(a.T.copy()), 1, flags, alpha=alpha)
         assert_same(g, o, flags)
+
+
+# ---------------------------------------------------------------------------
+# Headroom tensor scale (NVFP4_HEADROOM): alpha = amax / (4 * 448).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("orient", ["row", "col", "dual"])
+def test_headroom_all_modes(api, pr1, mode, orient):
+    flags = {"row": ROW, "col": COL, "dual": ROW | COL}[orient] | HEADROOM
+    g, o, _ = run_both(api, pr1["x"], MODES[mode], flags, seed=99, stream_id=2)
+    assert_same(g, o, flags)
+
+
+@pytest.mark.parametrize("extra", [B2D, B2D | SP, SP, SP | RHT])
+def test_headroom_four_six_2d_and_single_pass(api, pr1, extra):
+    flags = ROW | COL | HEADROOM | extra
+    x = pr1["w"] if extra & B2D else pr1["x"]
+    g, o, _ = run_both(api, x, MODES["four_six"], flags, seed=8)
+    assert_same(g, o, flags)

@@ -651,3 +651,31 @@ def test_stream_ids_and_seeds_change_the_noise(pr1):
     c = oracle.quantize(x, oracle.RHT_SR, oracle.ROWWISE, seed=3, stream_id=0)
     assert not np.array_equal(a["codes_row"], b["codes_row"])
     assert np.array_equal(a["codes_row"], c["codes_row"])
+
+
+def test_headroom_alpha_keeps_the_four_candidate_in_range():
+    """Four Over Six (§2.1 Eq. 1-2, §1 Table 1) with the plain tensor scale
+    amax / (6 * 448): a block whose maximum exceeds 2/3 of the tensor amax gets
+    an M = 4 raw scale above 448, which E4M3 clips.  With the headroom scale
+    amax / (4 * 448) no M = 4 raw scale passes 448 (beyond the rounding of
+    alpha).  Either way every stored scale is one of the block's two
+    candidates, computed here in float32 from the block maxima."""
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    x = synthetic.normal_with_channel_outliers(64, 256, seed=11)
+    bits = synthetic.bf16_bits(x)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    amax_b = np.abs(vals.reshape(-1, 16)).max(axis=1).astype(np.float32)
+    for flags, expect_clip in ((oracle.ROWWISE, True), (oracle.ROWWISE | oracle.HEADROOM, False)):
+        out = oracle.quantize(bits, 1, flags)
+        a = np.float32(out["alpha_row"])
+        amax = np.float32(out["amax_row"])
+        assert a == (amax / np.float32(1792 if flags & oracle.HEADROOM else 2688))
+        raw4 = amax_b / np.float32(a * np.float32(4))
+        raw6 = amax_b / np.float32(a * np.float32(6))
+        s4 = np.array([oracle.e4m3_rne(float(r)) for r in raw4])
+        s6 = np.array([oracle.e4m3_rne(float(r)) for r in raw6])
+        chosen = out["scales_row"].reshape(-1)
+        assert np.all((chosen == s4) | (chosen == s6))
+        assert bool(np.any(raw4 > 448 * (1 + 2 ** -20))) == expect_clip
+        if not expect_clip:
+            assert np.any(chosen == s4)  # the M = 4 candidate still wins somewhere
