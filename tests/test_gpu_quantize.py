@@ -428,3 +428,27 @@ def test_headroom_four_six_2d_and_single_pass(api, pr1, extra):
     x = pr1["w"] if extra & B2D else pr1["x"]
     g, o, _ = run_both(api, x, MODES["four_six"], flags, seed=8)
     assert_same(g, o, flags)
+
+
+@pytest.mark.parametrize("mode", ["rtn", "four_six", "ms_eden"])
+@pytest.mark.parametrize("eps", [2.0 ** -22, -(2.0 ** -23), 0.0])
+def test_scale_rounding_near_e4m3_midpoints(api, mode, eps):
+    # alpha = 0.5 (1 + eps) makes the M = 6 divisor 3 (1 + eps): block maxima
+    # 3 m, m an E4M3 rounding midpoint, give quotients within a few ulps of m
+    # (eps = 0: exactly m, a tie).  The scale must still round as the oracle's
+    # correctly rounded quotient does.
+    alpha = float(np.float32(0.5) * np.float32(1.0 + eps))
+    mids = [1.0625, 1.1875, 1.3125, 1.4375, 1.5625, 1.6875, 1.8125, 1.9375, 0.53125, 2.125, 4.25, 9.5,
+            19.0, 38.0, 0.28125, 0.140625]
+    rng = np.random.default_rng(17)
+    a = (rng.standard_normal((64, 256)) * 0.1).astype(np.float32)
+    blocks = a.reshape(64, 16, 16)
+    for r in range(64):
+        for b in range(16):
+            m = mids[(r + b) % len(mids)]
+            blocks[r, b, (r * 7 + b) % 16] = np.float32(3.0 * m) * (1 if (r + b) % 3 else -1)
+            blocks[r, b] = np.clip(blocks[r, b], -abs(3.0 * m), abs(3.0 * m))
+    x = synthetic.to_bf16(blocks.reshape(64, 256))
+    for flags in (ROW, ROW | COL):
+        g, o, _ = run_both(api, x, MODES[mode], flags, seed=13, alpha=alpha)
+        assert_same(g, o, flags)
