@@ -162,6 +162,21 @@ __device__ __forceinline__ float e2m1_sr_value(float y, uint32_t u16) {
   return copysignf(q, y);
 }
 
+// e2m1_sr_value without branches: the same operations, with the division by
+// m (a power of two, so exact) done as a multiplication by 1 / m.
+__device__ __forceinline__ float e2m1_sr_value_nb(float y, uint32_t u16) {
+  const float a = fabsf(y);
+  const bool lt2 = a < 2.0f, lt4 = a < 4.0f;
+  const float m = lt2 ? 2.0f : (lt4 ? 1.0f : 0.5f);
+  const float inv_m = lt2 ? 0.5f : (lt4 ? 1.0f : 2.0f);
+  const float t = __fmul_rn(a, m);
+  const float fl = floorf(t);
+  const float f = __fsub_rn(t, fl);
+  const float up = (static_cast<float>(u16) < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
+  const float q = (a >= 6.0f) ? 6.0f : __fmul_rn(__fadd_rn(fl, up), inv_m);
+  return copysignf(q, y);
+}
+
 // ---------------------------------------------------------------------------
 // 16-wide Hadamard butterfly, natural (Sylvester) order, strides 1, 2, 4, 8.
 // r = (1/4) H16 D v where D flips the signs selected by `signs`.

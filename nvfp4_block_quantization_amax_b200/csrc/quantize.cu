@@ -419,15 +419,39 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
     }
     sba = eden_scale(num.x, den.x, wa);
     sbb = eden_scale(num.y, den.y, wb);
-  } else {  // stochastic rounding of the values: one block at a time
-    float a[16], b[16];
+  } else {  // RHT + stochastic rounding of the values
+    float ma, mb;
+    max_abs16x2(v, ma, mb);
+    sba = e4m3_ceil(scale_raw(ma, alpha, 6.0f));
+    sbb = e4m3_ceil(scale_raw(mb, alpha, 6.0f));
+    const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
+    const float rb = __frcp_rn(__fmul_rn(alpha, e4m3_value(sbb)));
+    // element i uses half (i & 1) of word (i >> 1) & 3 of draw i >> 3 (unit 2 blk + draw)
+    uint32_t wa[8], wb[8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint64_t ua = 2 * blka + j, ub = 2 * blkb + j;
+      const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagValueSR);
+      const uint4 db = philox(K, static_cast<uint32_t>(ub), static_cast<uint32_t>(ub >> 32), c2, kTagValueSR);
+      wa[4 * j] = da.x; wa[4 * j + 1] = da.y; wa[4 * j + 2] = da.z; wa[4 * j + 3] = da.w;
+      wb[4 * j] = db.x; wb[4 * j + 1] = db.y; wb[4 * j + 2] = db.z; wb[4 * j + 3] = db.w;
+    }
+    const float2 r2 = make_float2(ra, rb);
+    float qa[16], qb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      a[i] = v[i].x;
-      b[i] = v[i].y;
+      const float2 y = mul2(v[i], r2);
+      const int w = ((i >> 3) << 2) | ((i >> 1) & 3), sh = 16 * (i & 1);
+      qa[i] = e2m1_sr_value_nb(y.x, (wa[w] >> sh) & 0xFFFFu);
+      qb[i] = e2m1_sr_value_nb(y.y, (wb[w] >> sh) & 0xFFFFu);
     }
-    pa = quantize_block<MODE>(a, alpha, K, c2, blka, sba);
-    pb = quantize_block<MODE>(b, alpha, K, c2, blkb, sbb);
+    // the rounded values lie on the grid, so their encoding is exact
+    pa.lo = e2m1x8_rne(qa[0], qa[1], qa[2], qa[3], qa[4], qa[5], qa[6], qa[7]);
+    pa.hi = e2m1x8_rne(qa[8], qa[9], qa[10], qa[11], qa[12], qa[13], qa[14], qa[15]);
+    pb.lo = e2m1x8_rne(qb[0], qb[1], qb[2], qb[3], qb[4], qb[5], qb[6], qb[7]);
+    pb.hi = e2m1x8_rne(qb[8], qb[9], qb[10], qb[11], qb[12], qb[13], qb[14], qb[15]);
+    if (isinf(ra)) pa = sign_codes16<false>(v);
+    if (isinf(rb)) pb = sign_codes16<true>(v);
   }
 }
 
