@@ -22,6 +22,7 @@ own batch; no data-path collective).  Rank 0 prints one JSON line.
   python bench.py --impl reference ...   # the CPU oracle, bounded sample
 """
 import argparse
+import functools
 import hashlib
 import json
 import os
@@ -383,6 +384,14 @@ def run_device(args, rank, world, local_rank):
 # --------------------------------------------------------------------------
 # the CPU oracle on a bounded sample of the same step
 # --------------------------------------------------------------------------
+@functools.lru_cache(maxsize=4)
+def _sample_tensors(budget_rows):
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    return (synthetic.bf16_bits(synthetic.normal_with_channel_outliers(budget_rows * 16, HIDDEN, seed=0)),
+            synthetic.bf16_bits(synthetic.weight(budget_rows * 16, HIDDEN, seed=1)),
+            synthetic.bf16_bits(synthetic.laplace_with_spikes(budget_rows * 16, OUT, seed=2)))
+
+
 def oracle_sample(budget_rows=64, gemm_rows=16, gemm_cols=16, bwd_mode="eden"):
     """Time the oracle on a sample of every part of the step and extrapolate
     to one full step.  Returns (step_seconds_extrapolated, sample description,
@@ -391,9 +400,7 @@ def oracle_sample(budget_rows=64, gemm_rows=16, gemm_cols=16, bwd_mode="eden"):
     import oracle
     from nvfp4_block_quantization_amax_b200 import synthetic
     rng = np.random.default_rng(0)
-    xb = synthetic.bf16_bits(synthetic.normal_with_channel_outliers(budget_rows * 16, HIDDEN, seed=0))
-    wb = synthetic.bf16_bits(synthetic.weight(budget_rows * 16, HIDDEN, seed=1))
-    dyb = synthetic.bf16_bits(synthetic.laplace_with_spikes(budget_rows * 16, OUT, seed=2))
+    xb, wb, dyb = _sample_tensors(budget_rows)
     bwd = MS_EDEN if bwd_mode == "eden" else RHT_SR
     t_total = 0.0
     parts = []
@@ -432,8 +439,12 @@ def run_reference(args):
         return None
     t_step = []
     desc = threads = None
+    # each step is a bounded sample: 1024-row slices for a short run, fewer
+    # rows (down to 16) when many steps are asked for, so that the whole run
+    # stays within a few minutes
+    budget_rows = max(1, min(64, (64 * 32) // (args.warmup + args.steps)))
     for i in range(args.warmup + args.steps):
-        dt, desc, threads = oracle_sample(bwd_mode=args.bwd_mode)
+        dt, desc, threads = oracle_sample(budget_rows=budget_rows, bwd_mode=args.bwd_mode)
         if i >= args.warmup:
             t_step.append(dt)
     s = statistics.mean(t_step)
