@@ -8,10 +8,14 @@
 //   2. a quantize kernel reduces those partials to amax and alpha in its
 //      prologue, then encodes every block.
 // Rowwise-only work streams straight from HBM into registers (128-bit loads,
-// one 16-element block per thread).  Column, dual (row + column from one
-// read) and 2D 16x16 work stage a 64 x 128 tile in shared memory with
-// cp.async, so that both orientations are read conflict-free and the
-// transposed outputs are written in full 32-byte sectors.
+// two consecutive 16-element blocks per thread).  Column, dual (row + column
+// from one read) and 2D 16x16 work stream 64 x 128 tiles through a two-buffer
+// cp.async ring in shared memory, swizzled so both orientations are read
+// without bank conflicts; transposed outputs are written in full 32-byte
+// sectors.  Every kernel holds two independent blocks per thread in float2
+// registers and runs the element-wise steps with packed f32x2 instructions.
+// Single pass (NVFP4_SINGLE_PASS): the amax and quantize bodies run in one
+// cooperative launch separated by a bounded grid barrier.
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstdint>
