@@ -74,7 +74,15 @@ typedef enum {
   /* MS-EDEN ([Q2] §一): rotate, round the values to nearest, and put the
    * randomness only on the E4M3 scale, stochastically rounded from the
    * unbiasing value ||r||^2 / (alpha <r, q>). */
-  NVFP4_MS_EDEN = 3
+  NVFP4_MS_EDEN = 3,
+  /* As NVFP4_RHT_SR, with the values stochastically rounded by the sm_100a
+   * convert instruction that takes caller random bits ([NV] §四 names
+   * hardware stochastic rounding).  One Philox draw per block (tag 4,
+   * unit = block index) gives one 32-bit word per group of four elements;
+   * the instruction derives each element's 16-bit field from it.  Codes
+   * differ from NVFP4_RHT_SR's draw for draw; both are unbiased.  Not
+   * accepted with NVFP4_BLOCK2D. */
+  NVFP4_RHT_SR_HW = 4
 } nvfp4_mode_t;
 
 /* nvfp4_quantize flags */

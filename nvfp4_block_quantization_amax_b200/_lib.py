@@ -14,7 +14,7 @@ NVFP4_OK, NVFP4_ERR_ARG, NVFP4_ERR_SHAPE, NVFP4_ERR_ALIGN = 0, -1, -2, -3
 NVFP4_ERR_NONFINITE, NVFP4_ERR_LAUNCH, NVFP4_ERR_TIMEOUT, NVFP4_ERR_CUDA = -4, -5, -6, -7
 NVFP4_ERR_WORKSPACE = -8
 
-NVFP4_RTN, NVFP4_FOUR_SIX, NVFP4_RHT_SR, NVFP4_MS_EDEN = 0, 1, 2, 3
+NVFP4_RTN, NVFP4_FOUR_SIX, NVFP4_RHT_SR, NVFP4_MS_EDEN, NVFP4_RHT_SR_HW = 0, 1, 2, 3, 4
 
 NVFP4_ROWWISE = 0x1
 NVFP4_COLWISE = 0x2

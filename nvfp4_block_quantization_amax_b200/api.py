@@ -10,7 +10,7 @@ import torch
 from . import _lib as L
 from ._lib import (NVFP4_ALPHA_PROVIDED, NVFP4_BLOCK2D, NVFP4_COLWISE, NVFP4_FOUR_SIX,  # noqa: F401
                    NVFP4_GEMM_SCALE_LAYOUT, NVFP4_INVERSE_RHT, NVFP4_MS_EDEN, NVFP4_OUT_BF16,
-                   NVFP4_OUT_DTYPE_BF16, NVFP4_OUT_DTYPE_FP32, NVFP4_RHT, NVFP4_RHT_SR,
+                   NVFP4_OUT_DTYPE_BF16, NVFP4_OUT_DTYPE_FP32, NVFP4_RHT, NVFP4_RHT_SR, NVFP4_RHT_SR_HW,
                    NVFP4_ROWWISE, NVFP4_RTN, NVFP4_SINGLE_PASS)
 
 

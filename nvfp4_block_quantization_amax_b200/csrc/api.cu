@@ -62,12 +62,13 @@ nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, n
                               const float* alpha_in, const nvfp4_qtensor_t* out, void* workspace,
                               size_t workspace_bytes, void* stream) {
   if (!out) return NVFP4_ERR_ARG;
-  if (static_cast<int>(mode) < NVFP4_RTN || static_cast<int>(mode) > NVFP4_MS_EDEN) return NVFP4_ERR_ARG;
+  if (static_cast<int>(mode) < NVFP4_RTN || static_cast<int>(mode) > NVFP4_RHT_SR_HW) return NVFP4_ERR_ARG;
   if (flags & ~kQuantFlags) return NVFP4_ERR_ARG;
   const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE, two_d = flags & NVFP4_BLOCK2D;
   const bool gemm = flags & NVFP4_GEMM_SCALE_LAYOUT;
   if (!row && !col) return NVFP4_ERR_ARG;
-  if (two_d && (mode == NVFP4_RHT_SR || mode == NVFP4_MS_EDEN || (flags & NVFP4_RHT))) return NVFP4_ERR_ARG;
+  if (two_d && (mode == NVFP4_RHT_SR || mode == NVFP4_MS_EDEN || mode == NVFP4_RHT_SR_HW || (flags & NVFP4_RHT)))
+    return NVFP4_ERR_ARG;
   if (stream_id >= 0x80000000u) return NVFP4_ERR_ARG;
   if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (C % 16) return NVFP4_ERR_SHAPE;

@@ -61,6 +61,7 @@ __device__ __forceinline__ uint4 philox(const PhiloxKeys& K, uint32_t c0, uint32
 constexpr uint32_t kTagValueSR = 1u;   // 16-bit fields for element rounding
 constexpr uint32_t kTagScaleSR = 2u;   // 24-bit field for the E4M3 scale
 constexpr uint32_t kTagSigns = 3u;     // the sign diagonal of the rotation
+constexpr uint32_t kTagValueSRHw = 4u; // one word per 4 elements for the hardware SR convert
 
 // ---------------------------------------------------------------------------
 // bf16 <-> f32
@@ -175,6 +176,17 @@ __device__ __forceinline__ float e2m1_sr_value_nb(float y, uint32_t u16) {
   const float up = (static_cast<float>(u16) < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
   const float q = (a >= 6.0f) ? 6.0f : __fmul_rn(__fadd_rn(fl, up), inv_m);
   return copysignf(q, y);
+}
+
+// Four values stochastically rounded to E2M1 by the sm_100a convert with
+// caller random bits: a lands in bits 15:12, d in bits 3:0.  Each input draws
+// its own 16-bit field from `rbits`; it rounds up when that field plus its
+// fraction between grid points, scaled by 2^16, reaches 2^16.  Magnitudes of
+// 6 and above saturate to 6.
+__device__ __forceinline__ uint32_t e2m1x4_sr_hw(float a, float b, float c, float d, uint32_t rbits) {
+  uint16_t r;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;" : "=h"(r) : "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbits));
+  return r;
 }
 
 // ---------------------------------------------------------------------------

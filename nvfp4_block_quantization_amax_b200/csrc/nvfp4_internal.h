@@ -11,6 +11,7 @@ constexpr int kModeRTN = NVFP4_RTN;
 constexpr int kModeFourSix = NVFP4_FOUR_SIX;
 constexpr int kModeRhtSR = NVFP4_RHT_SR;
 constexpr int kModeMsEden = NVFP4_MS_EDEN;
+constexpr int kModeRhtSRHw = NVFP4_RHT_SR_HW;
 
 constexpr uint32_t kRowwise = NVFP4_ROWWISE;
 constexpr uint32_t kColwise = NVFP4_COLWISE;

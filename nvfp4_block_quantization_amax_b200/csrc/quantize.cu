@@ -423,6 +423,37 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
     }
     sba = eden_scale(num.x, den.x, wa);
     sbb = eden_scale(num.y, den.y, wb);
+  } else if constexpr (MODE == kModeRhtSRHw) {
+    // RHT + stochastic rounding by the convert instruction: ceil scales as
+    // below; one draw per block (unit blk), word g rounds elements 4g..4g+3,
+    // handed over last element first so that nibble j holds element 4g + j.
+    float ma, mb;
+    max_abs16x2(v, ma, mb);
+    sba = e4m3_ceil(scale_raw(ma, alpha, 6.0f));
+    sbb = e4m3_ceil(scale_raw(mb, alpha, 6.0f));
+    const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
+    const float rb = __frcp_rn(__fmul_rn(alpha, e4m3_value(sbb)));
+    const uint4 da = philox(K, static_cast<uint32_t>(blka), static_cast<uint32_t>(blka >> 32), c2, kTagValueSRHw);
+    const uint4 db = philox(K, static_cast<uint32_t>(blkb), static_cast<uint32_t>(blkb >> 32), c2, kTagValueSRHw);
+    const uint32_t wa[4] = {da.x, da.y, da.z, da.w}, wb[4] = {db.x, db.y, db.z, db.w};
+    const float2 r2 = make_float2(ra, rb);
+    float2 y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = mul2(v[i], r2);
+    uint32_t ca[4], cb[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      ca[g] = e2m1x4_sr_hw(y[4 * g + 3].x, y[4 * g + 2].x, y[4 * g + 1].x, y[4 * g].x, wa[g]);
+      cb[g] = e2m1x4_sr_hw(y[4 * g + 3].y, y[4 * g + 2].y, y[4 * g + 1].y, y[4 * g].y, wb[g]);
+    }
+    // the sign nibble follows the input's sign bit, zeros included
+    const Packed16 sa = sign_codes16<false>(v), sb = sign_codes16<true>(v);
+    pa.lo = (ca[0] | (ca[1] << 16)) | sa.lo;
+    pa.hi = (ca[2] | (ca[3] << 16)) | sa.hi;
+    pb.lo = (cb[0] | (cb[1] << 16)) | sb.lo;
+    pb.hi = (cb[2] | (cb[3] << 16)) | sb.hi;
+    if (isinf(ra)) pa = sa;
+    if (isinf(rb)) pb = sb;
   } else {  // RHT + stochastic rounding of the values
     float ma, mb;
     max_abs16x2(v, ma, mb);
@@ -1196,7 +1227,7 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   a.tiles_c_div = make_fastdiv(static_cast<uint32_t>(a.tiles_c > 0 ? a.tiles_c : 1));
   a.chunks_row = make_fastdiv(static_cast<uint32_t>(C / 8 > 0 ? C / 8 : 1));
   const bool row = flags & kRowwise, col = flags & kColwise, two_d = flags & kBlock2D;
-  const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || (flags & kRht)) && !two_d;
+  const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || mode == kModeRhtSRHw || (flags & kRht)) && !two_d;
   if (rot) a.partials_col = a.partials + a.npart;
   if (R == 0 || C == 0) return cudaSuccess;
 
@@ -1220,6 +1251,8 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
                    : dispatch_single_1d<kModeFourSix, false>(a, row, col, st);
       case kModeRhtSR:
         return dispatch_single_1d<kModeRhtSR, true>(a, row, col, st);
+      case kModeRhtSRHw:
+        return dispatch_single_1d<kModeRhtSRHw, true>(a, row, col, st);
       default:
         return dispatch_single_1d<kModeMsEden, true>(a, row, col, st);
     }
@@ -1247,6 +1280,8 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
                  : dispatch_1d<kModeFourSix, false>(a, row, col, st);
     case kModeRhtSR:
       return dispatch_1d<kModeRhtSR, true>(a, row, col, st);
+    case kModeRhtSRHw:
+      return dispatch_1d<kModeRhtSRHw, true>(a, row, col, st);
     default:
       return dispatch_1d<kModeMsEden, true>(a, row, col, st);
   }

@@ -19,7 +19,7 @@ from . import build as _build
 
 ROWWISE, COLWISE, BLOCK2D, ALPHA_PROVIDED, RHT, INVERSE_RHT = 0x1, 0x2, 0x4, 0x10, 0x40, 0x80
 HEADROOM = 0x200
-RTN, FOUR_SIX, RHT_SR, MS_EDEN = 0, 1, 2, 3
+RTN, FOUR_SIX, RHT_SR, MS_EDEN, RHT_SR_HW = 0, 1, 2, 3, 4
 OK, ERR_ARG, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -4
 
 _lib = None
@@ -47,7 +47,9 @@ def lib():
         for n in ("oracle_e4m3_rne", "oracle_e4m3_ceil", "oracle_e2m1_rne"):
             getattr(L, n).argtypes = [ctypes.c_float]
             getattr(L, n).restype = ctypes.c_uint8
-        for n in ("oracle_e4m3_sr", "oracle_e2m1_sr"):
+        L.oracle_sr_hw_field.argtypes = [ctypes.c_uint32, ctypes.c_int]
+        L.oracle_sr_hw_field.restype = ctypes.c_uint32
+        for n in ("oracle_e4m3_sr", "oracle_e2m1_sr", "oracle_e2m1_sr_hw"):
             getattr(L, n).argtypes = [ctypes.c_float, ctypes.c_uint32]
             getattr(L, n).restype = ctypes.c_uint8
         L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
@@ -145,6 +147,17 @@ def e2m1_rne(y):
 
 def e2m1_sr(y, u16):
     return int(lib().oracle_e2m1_sr(float(y), int(u16)))
+
+
+def e2m1_sr_hw(y, r16):
+    """E2M1 code of y stochastically rounded the way the sm_100a convert with
+    caller random bits does it, for its 16-bit field r16."""
+    return int(lib().oracle_e2m1_sr_hw(float(y), int(r16)))
+
+
+def sr_hw_field(w, j):
+    """16-bit field of the 32-bit word w used for element j of a group of four."""
+    return int(lib().oracle_sr_hw_field(int(w) & 0xFFFFFFFF, int(j)))
 
 
 def rht16(x, signs):

@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 ROW, COL, B2D, SP, RHT, GEMM = 0x1, 0x2, 0x4, 0x8, 0x40, 0x20
 FP32 = 1
 FROB_TOL = 1e-5
-MODES = {"rtn": 0, "four_six": 1, "rht_sr": 2, "ms_eden": 3}
+MODES = {"rtn": 0, "four_six": 1, "rht_sr": 2, "ms_eden": 3, "rht_sr_hw": 4}
 
 
 @pytest.fixture(scope="module")

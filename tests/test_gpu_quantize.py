@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 ROW, COL, B2D, RHT, GEMM = 0x1, 0x2, 0x4, 0x40, 0x20
 HEADROOM = 0x200
-MODES = {"rtn": 0, "four_six": 1, "rht_sr": 2, "ms_eden": 3}
+MODES = {"rtn": 0, "four_six": 1, "rht_sr": 2, "ms_eden": 3, "rht_sr_hw": 4}
 
 
 @pytest.fixture(scope="module")
