@@ -157,8 +157,8 @@ NVFP4_API size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
  *   3. per element: q = E2M1(x / (alpha * Delta)), computed as x times the
  *      correctly rounded reciprocal of alpha * Delta                 (Eq. 3)
  * with the mode choosing M, the rounding of Delta and q, and the 4/6 choice
- * (see nvfp4_mode_t).  Rotating modes (RHT_SR, MS_EDEN, or the NVFP4_RHT
- * flag) first replace each 16-block v by (1/4) H16 D v, D = diag of 16 random
+ * (see nvfp4_mode_t).  Rotating modes (RHT_SR, MS_EDEN, RHT_SR_HW, or the
+ * NVFP4_RHT flag) first replace each 16-block v by (1/4) H16 D v, D = diag of 16 random
  * signs drawn from `seed`; the same D serves every block and both
  * orientations, so two operands quantized with the same seed along their
  * shared K axis multiply to the unrotated product.

@@ -119,17 +119,6 @@ __device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t u24) {
 // ---------------------------------------------------------------------------
 // E2M1 values: codes sign | index into {0, .5, 1, 1.5, 2, 3, 4, 6}.
 // ---------------------------------------------------------------------------
-// Two values -> one byte (lo in bits 0-3, hi in bits 4-7), round to nearest
-// even with saturation at +-6 (PTX cvt.rn.satfinite.e2m1x2.f32).
-__device__ __forceinline__ uint32_t e2m1x2_rne(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 // Byte of two codes -> their two signed grid values (PTX cvt.rn.f16x2.e2m1x2,
 // exact), widened to float.
 __device__ __forceinline__ void e2m1x2_values(uint32_t byte, float& lo, float& hi) {
@@ -147,24 +136,7 @@ __device__ __forceinline__ void e2m1x2_values(uint32_t byte, float& lo, float& h
 // is exact, f = t - floor(t) is the position between the neighbours, and the
 // magnitude rounds up iff u16 < f * 65536.  |y| >= 6 -> 6.  Returns the
 // signed grid value (exactly representable, so its encoding is exact).
-__device__ __forceinline__ float e2m1_sr_value(float y, uint32_t u16) {
-  const float a = fabsf(y);
-  float q;
-  if (a >= 6.0f) {
-    q = 6.0f;
-  } else {
-    const float m = (a < 2.0f) ? 2.0f : ((a < 4.0f) ? 1.0f : 0.5f);
-    const float t = __fmul_rn(a, m);
-    const float fl = floorf(t);
-    const float f = __fsub_rn(t, fl);
-    const float up = (static_cast<float>(u16) < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
-    q = __fdiv_rn(__fadd_rn(fl, up), m);  // m is a power of two: exact
-  }
-  return copysignf(q, y);
-}
-
-// e2m1_sr_value without branches: the same operations, with the division by
-// m (a power of two, so exact) done as a multiplication by 1 / m.
+// Branch-free: the segment's m and 1 / m (powers of two) are selected.
 __device__ __forceinline__ float e2m1_sr_value_nb(float y, uint32_t u16) {
   const float a = fabsf(y);
   const bool lt2 = a < 2.0f, lt4 = a < 4.0f;
@@ -191,28 +163,9 @@ __device__ __forceinline__ uint32_t e2m1x4_sr_hw(float a, float b, float c, floa
 
 // ---------------------------------------------------------------------------
 // 16-wide Hadamard butterfly, natural (Sylvester) order, strides 1, 2, 4, 8.
-// r = (1/4) H16 D v where D flips the signs selected by `signs`.
+// The forward transform is r = (1/4) H16 D v, D flipping the signs selected
+// by `signs` (lane-paired below); the inverse is x = D (1/4) H16 r.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void rht16(float* v, uint32_t signs) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((signs >> i) & 1u) << 31));
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = __fadd_rn(a, b);
-        v[i + h] = __fsub_rn(a, b);
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
-}
-
-// Inverse: x = D (1/4) H16 r.
 __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
 #pragma unroll
   for (int h = 1; h < 16; h <<= 1) {
@@ -273,8 +226,8 @@ __device__ __forceinline__ void unpack16x2_signed(const uint4 a0, const uint4 a1
   }
 }
 
-// H16 v for two lane-paired blocks (signs already applied): the butterfly of
-// rht16 without its final 1/4.
+// H16 v for two lane-paired blocks (signs already applied): the butterfly
+// without the final 1/4.
 __device__ __forceinline__ void hadamard16x2(float2* v) {
 #pragma unroll
   for (int h = 1; h < 16; h <<= 1) {
@@ -289,31 +242,12 @@ __device__ __forceinline__ void hadamard16x2(float2* v) {
   }
 }
 
-// rht16 of two lane-paired blocks whose signs are already applied.
+// (1/4) H16 v of two lane-paired blocks whose signs are already applied.
 __device__ __forceinline__ void rht16x2_presigned(float2* v) {
   hadamard16x2(v);
   const float2 q = make_float2(0.25f, 0.25f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = mul2(v[i], q);
-}
-
-// Pairwise sum with strides 8, 4, 2, 1 (the stated summation order).
-__device__ __forceinline__ float sum16(const float* e) {
-  float t[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = __fadd_rn(e[i], e[i + 8]);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) t[i] = __fadd_rn(t[i], t[i + 4]);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) t[i] = __fadd_rn(t[i], t[i + 2]);
-  return __fadd_rn(t[0], t[1]);
-}
-
-__device__ __forceinline__ float max_abs16(const float* v) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-  return m;
 }
 
 // ---------------------------------------------------------------------------
@@ -331,87 +265,10 @@ __device__ __forceinline__ float scale_raw(float amax_b, float alpha, float M) {
   return (den == 0.0f) ? 0.0f : __fdiv_rn(amax_b, den);
 }
 
-// Eq. 3 with round to nearest: codes of v under stored scale byte sb.  When
-// s = alpha * Delta is 0, or 1/s overflows, the magnitudes are 0 and the
-// codes keep the signs of v.
-__device__ __forceinline__ Packed16 encode_rne(const float* v, float alpha, uint32_t sb) {
-  const float s = __fmul_rn(alpha, e4m3_value(sb));
-  const float rinv = __frcp_rn(s);
-  Packed16 p{0u, 0u};
-  if (isinf(rinv)) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t sign = (__float_as_uint(v[i]) >> 31) << 3;
-      if (i < 8) p.lo |= sign << (4 * i);
-      else p.hi |= sign << (4 * (i - 8));
-    }
-    return p;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t b = e2m1x2_rne(__fmul_rn(v[2 * j], rinv), __fmul_rn(v[2 * j + 1], rinv));
-    if (j < 4) p.lo |= b << (8 * j);
-    else p.hi |= b << (8 * (j - 4));
-  }
-  return p;
-}
-
-// Eq. 3 with stochastic rounding of the values; u16[i] are the element's
-// 16-bit uniforms.
-__device__ __forceinline__ Packed16 encode_sr(const float* v, float alpha, uint32_t sb,
-                                              const uint32_t* words /* 8 words */) {
-  const float s = __fmul_rn(alpha, e4m3_value(sb));
-  const float rinv = __frcp_rn(s);
-  Packed16 p{0u, 0u};
-  if (isinf(rinv)) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t sign = (__float_as_uint(v[i]) >> 31) << 3;
-      if (i < 8) p.lo |= sign << (4 * i);
-      else p.hi |= sign << (4 * (i - 8));
-    }
-    return p;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    // elements 2j, 2j+1 share word (j & 3) of draw (j >> 2): low / high half
-    const uint32_t w = words[((j >> 2) << 2) | (j & 3)];
-    const float q0 = e2m1_sr_value(__fmul_rn(v[2 * j], rinv), w & 0xFFFFu);
-    const float q1 = e2m1_sr_value(__fmul_rn(v[2 * j + 1], rinv), w >> 16);
-    const uint32_t b = e2m1x2_rne(q0, q1);
-    if (j < 4) p.lo |= b << (8 * j);
-    else p.hi |= b << (8 * (j - 4));
-  }
-  return p;
-}
-
-// Signed grid values of the 16 codes.
-__device__ __forceinline__ void decode16(const Packed16& p, float* q) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t b = ((j < 4) ? (p.lo >> (8 * j)) : (p.hi >> (8 * (j - 4)))) & 0xFFu;
-    e2m1x2_values(b, q[2 * j], q[2 * j + 1]);
-  }
-}
-
-// Squared error of an encoding in the original domain, summed with sum16:
-// e_i = (v_i - q_i s)^2.
-__device__ __forceinline__ float sq_error(const float* v, float alpha, uint32_t sb,
-                                          const Packed16& p) {
-  const float s = __fmul_rn(alpha, e4m3_value(sb));
-  float q[16], e[16];
-  decode16(p, q);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float d = __fsub_rn(v[i], __fmul_rn(q[i], s));
-    e[i] = __fmul_rn(d, d);
-  }
-  return sum16(e);
-}
-
 // ---------------------------------------------------------------------------
 // Eight values <-> one word of eight E2M1 codes (element k in bits 4k..4k+3).
-// Same conversions as e2m1x2_rne / e2m1x2_values, four at a time.
+// Encoding rounds to nearest even with saturation at +-6 (PTX
+// cvt.rn.satfinite.e2m1x2.f32, two values per byte); decoding is exact.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t e2m1x8_rne(float y0, float y1, float y2, float y3, float y4, float y5,
                                                float y6, float y7) {
@@ -460,7 +317,10 @@ __device__ __forceinline__ Packed16 sign_codes16(const float2* v) {
   return p;
 }
 
-// encode_rne for two lane-paired blocks with scale bytes sba (x) and sbb (y).
+// Eq. 3 with round to nearest for two lane-paired blocks with scale bytes sba
+// (x) and sbb (y): codes of v times the correctly rounded 1 / (alpha Delta).
+// When alpha Delta is 0, or its reciprocal overflows, the magnitudes are 0
+// and the codes keep the signs of v.
 __device__ __forceinline__ void encode_rne_x2(const float2* v, float alpha, uint32_t sba, uint32_t sbb,
                                               Packed16& pa, Packed16& pb) {
   const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
@@ -488,7 +348,8 @@ __device__ __forceinline__ void decode16x2(const Packed16& pa, const Packed16& p
   for (int i = 0; i < 16; ++i) q[i] = make_float2(a[i], b[i]);
 }
 
-// sum16 of two lane-paired blocks of products.  The packed multiply that
+// Pairwise sum of 16 terms with strides 8, 4, 2, 1 (the stated summation
+// order), two lane-paired blocks at a time.  The packed multiply that
 // made e[] may be contracted with a packed add into one fma (measured: the
 // rounding of d * d vanished from 4/6 errors), so the first level, which
 // consumes the products, adds with the scalar __fadd_rn, which is never
@@ -504,7 +365,8 @@ __device__ __forceinline__ float2 sum16x2(const float2* e) {
   return add2(t[0], t[1]);
 }
 
-// sq_error of two lane-paired encodings.
+// Squared error of two lane-paired encodings in the original domain,
+// e_i = (v_i - q_i s)^2 summed with sum16x2.
 __device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint32_t sba, uint32_t sbb,
                                               const Packed16& pa, const Packed16& pb) {
   const float2 s2 = make_float2(__fmul_rn(alpha, e4m3_value(sba)), __fmul_rn(alpha, e4m3_value(sbb)));
@@ -518,7 +380,8 @@ __device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint
   return sum16x2(e);
 }
 
-// Tree-shaped (depth 4) so the two chains of dependent max operations stay
+// Block maxima of |v| for two lane-paired blocks.  Tree-shaped (depth 4) so
+// the two chains of dependent max operations stay
 // short; max is exact, so the order does not matter.
 __device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
   float a[8], b[8];

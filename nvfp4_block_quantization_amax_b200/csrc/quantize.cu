@@ -127,61 +127,6 @@ __device__ __forceinline__ int64_t gemm_scale_offset(int64_t m, int64_t j, int64
   return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
 }
 
-// ---------------------------------------------------------------------------
-// One 16-element block in a mode.  v holds the (rotated) values; the block's
-// random streams are keyed by (seed, c2 = 2 stream_id + orientation, blk).
-// ---------------------------------------------------------------------------
-template <int MODE>
-__device__ __forceinline__ Packed16 quantize_block(const float* v, float alpha,
-                                                   const PhiloxKeys& K, uint32_t c2,
-                                                   uint64_t blk, uint32_t& sb) {
-  const float amax_b = max_abs16(v);
-  if constexpr (MODE == kModeRTN) {
-    sb = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
-    return encode_rne(v, alpha, sb);
-  } else if constexpr (MODE == kModeFourSix) {
-    const uint32_t sb6 = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
-    const uint32_t sb4 = e4m3_rne(scale_raw(amax_b, alpha, 4.0f));
-    const Packed16 p6 = encode_rne(v, alpha, sb6);
-    const Packed16 p4 = encode_rne(v, alpha, sb4);
-    const float e6 = sq_error(v, alpha, sb6, p6);
-    const float e4 = sq_error(v, alpha, sb4, p4);
-    const bool take4 = e4 < e6;
-    sb = take4 ? sb4 : sb6;
-    return take4 ? p4 : p6;
-  } else if constexpr (MODE == kModeRhtSR) {
-    sb = e4m3_ceil(scale_raw(amax_b, alpha, 6.0f));
-    const uint64_t u0 = 2 * blk, u1 = 2 * blk + 1;
-    const uint4 w0 = philox(K, static_cast<uint32_t>(u0), static_cast<uint32_t>(u0 >> 32), c2, kTagValueSR);
-    const uint4 w1 = philox(K, static_cast<uint32_t>(u1), static_cast<uint32_t>(u1 >> 32), c2, kTagValueSR);
-    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    return encode_sr(v, alpha, sb, words);
-  } else {  // MS-EDEN
-    const uint32_t prov = e4m3_rne(scale_raw(amax_b, alpha, 6.0f));
-    const Packed16 p = encode_rne(v, alpha, prov);
-    float q[16], rr[16], rq[16];
-    decode16(p, q);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      rr[i] = __fmul_rn(v[i], v[i]);
-      rq[i] = __fmul_rn(v[i], q[i]);
-    }
-    const float num = sum16(rr);
-    const float den = __fmul_rn(alpha, sum16(rq));
-    if (den == 0.0f) {
-      sb = 0u;
-    } else {
-      const float dstar = __fdiv_rn(num, den);
-      const uint64_t unit = blk >> 2;
-      const uint4 w = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
-      const uint32_t sel = static_cast<uint32_t>(blk & 3);
-      const uint32_t word = sel == 0 ? w.x : (sel == 1 ? w.y : (sel == 2 ? w.z : w.w));
-      sb = e4m3_sr(dstar, word >> 8);
-    }
-    return p;
-  }
-}
-
 // ===========================================================================
 // amax kernels.  Each CTA leaves one partial maximum (float bits, or
 // kNonFinite) per orientation; the quantize kernels reduce them.
@@ -380,8 +325,10 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
 constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
 
 // ---------------------------------------------------------------------------
-// quantize_block for two lane-paired blocks (x: block a, y: block b): the
-// same arithmetic, with the element-wise steps done two blocks at a time.
+// One mode's quantization of two lane-paired 16-element blocks (x: block a,
+// y: block b), the element-wise steps done two blocks at a time.  v holds the
+// (rotated) values; a block's random streams are keyed by (seed,
+// c2 = 2 stream_id + orientation, block index).
 // ---------------------------------------------------------------------------
 // MS-EDEN scale of one block from its sums and its random word.
 __device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t word) {
