@@ -38,13 +38,18 @@ if ROOT not in sys.path:
 
 METRIC = "NVFP4 quantize Gelem/s & % HBM roofline; NVFP4 GEMM TFLOPS & % FP4 peak"
 TOKENS, HIDDEN, OUT = 8192, 4096, 14336
-WORKLOAD = ("linear fwd+bwd, 8B-shaped: X 8192x4096 (4/6 1D), W 14336x4096 (4/6 2D), "
-            "dY 8192x14336 (MS-EDEN rows+cols), fprop/dgrad/wgrad NVFP4 GEMMs, bf16 out")
+BWD_NAMES = {"eden": "MS-EDEN", "sr": "RHT+SR", "sr_hw": "RHT+hardware SR"}
+
+
+def workload(bwd_mode="eden"):
+    return ("linear fwd+bwd, 8B-shaped: X 8192x4096 (4/6 1D), W 14336x4096 (4/6 2D), "
+            f"dY 8192x14336 ({BWD_NAMES[bwd_mode]} rows+cols), fprop/dgrad/wgrad NVFP4 GEMMs, bf16 out")
 FP4_PER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 ROW, COL, B2D, RHT, GEMM = 0x1, 0x2, 0x4, 0x40, 0x20
-RTN, FOUR_SIX, RHT_SR, MS_EDEN = 0, 1, 2, 3
+RTN, FOUR_SIX, RHT_SR, MS_EDEN, RHT_SR_HW = 0, 1, 2, 3, 4
+BWD_MODES = {"eden": MS_EDEN, "sr": RHT_SR, "sr_hw": RHT_SR_HW}
 
 
 def gemm_flops():
@@ -281,7 +286,7 @@ def run_device(args, rank, world, local_rank):
     _lib.load()
     layer = synthetic.fwd_bwd_8b(seed=17 * rank)
     x, w, dy = (layer[k].to(device) for k in ("x", "w", "dy"))
-    bwd = MS_EDEN if args.bwd_mode == "eden" else RHT_SR
+    bwd = BWD_MODES[args.bwd_mode]
     step = LayerStep(x, w, dy, bwd, device)
 
     # --- device-resident timing ---
@@ -362,7 +367,7 @@ def run_device(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e2m1 x e2m1 -> f32 (GEMM), f32 (quantizer)",
         "data": "synthetic (seeded; shapes and distributions of the pages' 8B workload)",
-        "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN, "out_features": OUT,
+        "config": {"workload": workload(args.bwd_mode), "tokens": TOKENS, "hidden": HIDDEN, "out_features": OUT,
                    "bwd_mode": args.bwd_mode, "parallelism": f"replicas x{world} (weak)",
                    "l2": "inputs larger than L2: 419 MB of bf16 per step"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
@@ -401,7 +406,7 @@ def oracle_sample(budget_rows=64, gemm_rows=16, gemm_cols=16, bwd_mode="eden"):
     from nvfp4_block_quantization_amax_b200 import synthetic
     rng = np.random.default_rng(0)
     xb, wb, dyb = _sample_tensors(budget_rows)
-    bwd = MS_EDEN if bwd_mode == "eden" else RHT_SR
+    bwd = BWD_MODES[bwd_mode]
     t_total = 0.0
     parts = []
 
@@ -452,7 +457,7 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer, f64 GEMM (CPU oracle)",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "bwd_mode": args.bwd_mode},
+            "data": "synthetic", "config": {"workload": workload(args.bwd_mode), "bwd_mode": args.bwd_mode},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -463,8 +468,8 @@ def cpu_baseline_line(bwd_mode):
             "sample": desc, "step_seconds_extrapolated": dt}
 
 
-KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_w_rot",
-                "quant_x_rot")
+KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_dy_sr",
+                "quant_dy_sr_hw", "quant_w_rot", "quant_x_rot")
 
 
 def run_kernel_case(name, iters=3):
@@ -491,6 +496,8 @@ def run_kernel_case(name, iters=3):
         "quant_x": lambda: step.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0),
         "quant_w2d": lambda: step.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1),
         "quant_dy": lambda: step.quantize("dy", MS_EDEN, ROW | COL | GEMM, 7, 0),
+        "quant_dy_sr": lambda: step.quantize("dy", RHT_SR, ROW | COL | GEMM, 7, 0),
+        "quant_dy_sr_hw": lambda: step.quantize("dy", RHT_SR_HW, ROW | COL | GEMM, 7, 0),
         "quant_w_rot": lambda: step.quantize("w_rot", RTN, COL | RHT | GEMM, 7, 1),
         "quant_x_rot": lambda: step.quantize("x_rot", RTN, COL | RHT | GEMM, 7, 2),
     }
@@ -505,7 +512,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--bwd-mode", choices=["eden", "sr"], default="eden")
+    ap.add_argument("--bwd-mode", choices=sorted(BWD_MODES), default="eden")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=KERNEL_CASES,
                     help="run one call of the step a few times and exit (for profiler captures)")
