@@ -85,6 +85,15 @@ def lib():
         L.oracle_quantize_block16.restype = ctypes.c_int
         L.oracle_block_sq_error.argtypes = [_f32p, ctypes.c_float, _u8p, ctypes.c_uint8]
         L.oracle_block_sq_error.restype = ctypes.c_float
+        L.oracle_mx_exponent.argtypes = [ctypes.c_float]
+        L.oracle_mx_exponent.restype = ctypes.c_int
+        L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0_value.restype = ctypes.c_float
+        L.oracle_mx_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64,
+                                         _u8p, _u8p, _u8p, _u8p]
+        L.oracle_mx_quantize.restype = ctypes.c_int
+        L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64, _f32p]
+        L.oracle_mx_dequantize.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -310,3 +319,44 @@ def unpack_codes(codes):
     out[..., 0::2] = codes & 0xF
     out[..., 1::2] = codes >> 4
     return out
+
+
+# --------------------------------------------------------------------- MXFP4
+def mx_exponent(amax):
+    """Shared exponent of a 32-block with maximum magnitude amax."""
+    return int(lib().oracle_mx_exponent(float(amax)))
+
+
+def e8m0_value(b):
+    return float(lib().oracle_e8m0_value(int(b)))
+
+
+def mx_quantize(x, flags, seed=0, C=None):
+    """MXFP4 quantization of a [R, ld] uint16 (bf16) array in the requested
+    orientations (ROWWISE / COLWISE, optional RHT)."""
+    x = _bf16_bits(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    cr = sr = cc = sc = None
+    if flags & ROWWISE:
+        cr = np.zeros((R, C // 2), np.uint8)
+        sr = np.zeros((R, C // 32), np.uint8)
+    if flags & COLWISE:
+        cc = np.zeros((C, R // 2), np.uint8)
+        sc = np.zeros((C, R // 32), np.uint8)
+    _check(lib().oracle_mx_quantize(_p(x, _u16p), R, C, ld, flags, seed, _p(cr, _u8p), _p(sr, _u8p),
+                                    _p(cc, _u8p), _p(sc, _u8p)))
+    out = {}
+    if flags & ROWWISE:
+        out.update(codes_row=cr, scales_row=sr)
+    if flags & COLWISE:
+        out.update(codes_col=cc, scales_col=sc)
+    return out
+
+
+def mx_dequantize(codes, scales, R, C, flags=0, seed=0):
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    y = np.zeros((R, C), np.float32)
+    _check(lib().oracle_mx_dequantize(_p(codes, _u8p), _p(scales, _u8p), R, C, flags, seed, _p(y, _f32p)))
+    return y

@@ -747,3 +747,105 @@ float oracle_block_sq_error(const float v[16], float alpha, const uint8_t codes[
   b.scale = scale;
   return block_sq_error(v, alpha, &b);
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4: 32-element blocks, one power-of-two (UE8M0) scale per block, E2M1  */
+/* values, no tensor scale ([NV] §一 and §五; the AMD MI355X write-up, 01-02, */
+/* with a fixed rotation).                                                   */
+/* ------------------------------------------------------------------------ */
+/* READING: the pages give the block size (32), the scale format (UE8M0,
+ * power-of-two) and nothing of how the scale is chosen.  The oracle takes the
+ * OCP microscaling rule: shared exponent e = floor(log2(amax_b)) - 2 (2 being
+ * the largest E2M1 exponent), clamped to the UE8M0 range [-127, 127]; an
+ * all-zero block takes -127.  Stored byte = e + 127.  Values are
+ * q_i = E2M1-RNE(v_i / 2^e), saturating at 6 (so block maxima in [6, 8) * 2^e
+ * clip to 6). */
+int oracle_mx_exponent(float amax) {
+  if (!(amax > 0.0f)) return -127;
+  int k;
+  frexpf(amax, &k);          /* amax = m 2^k, m in [0.5, 1): floor(log2) = k - 1 */
+  int e = (k - 1) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+float oracle_e8m0_value(uint8_t b) {
+  if (b == 0xFF) return NAN;
+  return ldexpf(1.0f, (int)b - 127);
+}
+
+/* One 32-vector: scale byte and codes. */
+static void mx_block(const float v[32], uint8_t code[32], uint8_t* scale) {
+  float m = 0.0f;
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  int e = oracle_mx_exponent(m);
+  *scale = (uint8_t)(e + 127);
+  for (int i = 0; i < 32; ++i) code[i] = oracle_e2m1_rne(ldexpf(v[i], -e));
+}
+
+/* Quantize bf16 x [R, C] to MXFP4 in the requested orientations: rows (32
+ * consecutive elements of a row; codes [R, C/2], scales [R, C/32]) and / or
+ * columns (32 consecutive rows of a column, stored transposed: codes
+ * [C, R/2], scales [C, R/32]).  With OR_RHT each 16-element half of a block
+ * is first rotated by (1/4) H16 D, D drawn from seed as for NVFP4 (a fixed
+ * seed gives the deterministic rotation).  Non-finite input returns
+ * OR_ERR_NONFINITE. */
+int oracle_mx_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld,
+                       uint32_t flags, uint64_t seed, uint8_t* codes_row,
+                       uint8_t* scales_row, uint8_t* codes_col,
+                       uint8_t* scales_col) {
+  int want_row = (flags & OR_ROWWISE) != 0, want_col = (flags & OR_COLWISE) != 0;
+  if (!want_row && !want_col) return OR_ERR_ARG;
+  if (R < 0 || C < 0 || ld < C) return OR_ERR_SHAPE;
+  if ((want_row && C % 32) || (want_col && R % 32)) return OR_ERR_SHAPE;
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t c = 0; c < C; ++c)
+      if (!isfinite(bf16_to_f32(x[r * ld + c]))) return OR_ERR_NONFINITE;
+  int rot = (flags & OR_RHT) != 0;
+  uint32_t signs = oracle_sign_bits(seed);
+  for (int orient = 0; orient < 2; ++orient) {
+    if (orient == 0 && !want_row) continue;
+    if (orient == 1 && !want_col) continue;
+    int64_t nvec = orient ? C : R, len = orient ? R : C;
+    uint8_t* codes = orient ? codes_col : codes_row;
+    uint8_t* scales = orient ? scales_col : scales_row;
+    for (int64_t i = 0; i < nvec; ++i)
+      for (int64_t b = 0; b < len / 32; ++b) {
+        float v[32];
+        gather_block(x, ld, orient, i, 2 * b, rot, signs, v);
+        gather_block(x, ld, orient, i, 2 * b + 1, rot, signs, v + 16);
+        uint8_t q[32];
+        mx_block(v, q, &scales[i * (len / 32) + b]);
+        for (int k = 0; k < 16; ++k)
+          codes[i * (len / 2) + 16 * b + k] = (uint8_t)(q[2 * k] | (q[2 * k + 1] << 4));
+      }
+  }
+  return OR_OK;
+}
+
+/* Decode MXFP4 codes [R, C/2] and scales [R, C/32] to fp32: y = q 2^e, then
+ * with OR_INVERSE_RHT each 16-element half goes through D (1/4) H16. */
+int oracle_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R,
+                         int64_t C, uint32_t flags, uint64_t seed, float* y) {
+  if (R < 0 || C < 0 || C % 32) return OR_ERR_SHAPE;
+  uint32_t signs = oracle_sign_bits(seed);
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t b = 0; b < C / 16; ++b) {
+      float s = oracle_e8m0_value(scales[r * (C / 32) + b / 2]);
+      float v[16];
+      for (int k = 0; k < 16; ++k) {
+        int64_t c = 16 * b + k;
+        uint8_t byte = codes[r * (C / 2) + c / 2];
+        uint8_t q = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+        v[k] = oracle_e2m1_value(q) * s;
+      }
+      if (flags & OR_INVERSE_RHT) {
+        float t[16];
+        oracle_irht16(v, signs, t);
+        memcpy(v, t, sizeof t);
+      }
+      for (int k = 0; k < 16; ++k) y[r * C + 16 * b + k] = v[k];
+    }
+  return OR_OK;
+}
