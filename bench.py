@@ -469,7 +469,7 @@ def cpu_baseline_line(bwd_mode):
 
 
 KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_dy_sr",
-                "quant_dy_sr_hw", "quant_w_rot", "quant_x_rot")
+                "quant_dy_sr_hw", "quant_w_rot", "quant_x_rot", "mx_dy")
 
 
 def run_kernel_case(name, iters=3):
@@ -500,6 +500,7 @@ def run_kernel_case(name, iters=3):
         "quant_dy_sr_hw": lambda: step.quantize("dy", RHT_SR_HW, ROW | COL | GEMM, 7, 0),
         "quant_w_rot": lambda: step.quantize("w_rot", RTN, COL | RHT | GEMM, 7, 1),
         "quant_x_rot": lambda: step.quantize("x_rot", RTN, COL | RHT | GEMM, 7, 2),
+        "mx_dy": lambda: api.mxfp4_quantize(dy, ROW | COL | RHT, seed=7),
     }
     for _ in range(iters):
         calls[name]()

@@ -249,6 +249,46 @@ NVFP4_API nvfp4_status_t nvfp4_gemm_quantize(const uint8_t* A, const uint8_t* sA
                                    uint8_t* codes, uint8_t* scales, float* amax_out,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * MXFP4 ([NV] §一 and §五 contrast it with NVFP4; the AMD MI355X write-up,
+ * 01-02, trains in it with a fixed Hadamard rotation).  Blocks of 32
+ * consecutive elements, one power-of-two scale per block stored as a UE8M0
+ * byte (2^(byte - 127)), E2M1 values, no tensor scale.
+ *
+ * READING (the pages give the format, not how the scale is chosen): the
+ * OCP microscaling rule.  Per block e = floor(log2(max |v|)) - 2 (2 being
+ * the largest E2M1 exponent), clamped to [-127, 127]; an all-zero block has
+ * e = -127.  The stored byte is e + 127 and q_i = E2M1(v_i / 2^e) rounded to
+ * nearest even, saturating at +-6 (a block maximum in [6, 8) 2^e clips).
+ * ------------------------------------------------------------------------ */
+
+/* Quantize the bf16 tensor x [R, C] (row stride ld) to MXFP4 in one read.
+ *   flags: NVFP4_ROWWISE and / or NVFP4_COLWISE, optionally NVFP4_RHT (each
+ *     16-element half of a block is first rotated by (1/4) H16 D, D the sign
+ *     diagonal drawn from `seed` exactly as for nvfp4_quantize; a fixed seed
+ *     gives the fixed rotation).
+ *   rowwise: codes_row [R, C/2] (element 2j in the low nibble), scales_row
+ *     [R, C/32] row-major.  columnwise (blocks of 32 rows of a column, stored
+ *     transposed): codes_col [C, R/2], scales_col [C, R/32].
+ *   status (optional device int32, sticky): NVFP4_ERR_NONFINITE when the
+ *     input holds an Inf or a NaN (the outputs are then unspecified).
+ * All pointers are device memory owned by the caller.  Shapes: C % 32 == 0
+ * (rowwise), R % 32 == 0 (columnwise), C % 16 == 0, ld >= C, ld % 8 == 0;
+ * x and the code buffers 16-byte aligned.  No workspace.  Asynchronous on
+ * `stream` (a cudaStream_t, NULL = legacy default stream). */
+NVFP4_API nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags,
+                                        uint64_t seed, uint8_t* codes_row, uint8_t* scales_row,
+                                        uint8_t* codes_col, uint8_t* scales_col, int32_t* status,
+                                        void* stream);
+
+/* Decode MXFP4 codes [R, C/2] with scales [R, C/32]:  y = q * 2^(byte - 127),
+ * optionally followed by the inverse rotation D (1/4) H16 of each 16-element
+ * half (NVFP4_INVERSE_RHT, key `seed`).  y is fp32 [R, C], or bf16 with
+ * NVFP4_OUT_BF16 (rounded to nearest even), row-major, contiguous.
+ * C % 32 == 0; codes 8-byte and y 16-byte aligned. */
+NVFP4_API nvfp4_status_t mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t C,
+                                          uint32_t flags, uint64_t seed, void* y, void* stream);
+
 /* Number of kernels this library has launched in the calling process since
  * it was loaded (all devices, all streams).  Instrumentation for callers that
  * account for their launches; not a page-defined operation. */

@@ -31,7 +31,8 @@ NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
 EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
-            "nvfp4_gemm", "nvfp4_gemm_quantize", "nvfp4_launch_count", "nvfp4_status_string", "nvfp4_version")
+            "nvfp4_gemm", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "nvfp4_launch_count",
+            "nvfp4_status_string", "nvfp4_version")
 
 
 class nvfp4_qtensor_t(ctypes.Structure):
@@ -69,6 +70,10 @@ def load(path=LIB_PATH):
     L.nvfp4_gemm_quantize.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, ctypes.c_int, u32, vp,
                                       vp, vp, vp, vp, sz, vp]
     L.nvfp4_gemm_quantize.restype = ctypes.c_int
+    L.mxfp4_quantize.argtypes = [vp, i64, i64, i64, u32, u64, vp, vp, vp, vp, vp, vp]
+    L.mxfp4_quantize.restype = ctypes.c_int
+    L.mxfp4_dequantize.argtypes = [vp, vp, i64, i64, u32, u64, vp, vp]
+    L.mxfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_status_string.argtypes = [ctypes.c_int]
     L.nvfp4_status_string.restype = ctypes.c_char_p
     L.nvfp4_version.argtypes = []
@@ -112,6 +117,15 @@ def nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, fla
                         amax_out, workspace, workspace_bytes, stream):
     return int(load().nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, flags, alpha_out,
                                           codes, scales, amax_out, workspace, workspace_bytes, stream))
+
+
+def mxfp4_quantize(x, R, C, ld, flags, seed, codes_row, scales_row, codes_col, scales_col, status, stream):
+    return int(load().mxfp4_quantize(x, R, C, ld, flags, seed, codes_row, scales_row, codes_col, scales_col,
+                                     status, stream))
+
+
+def mxfp4_dequantize(codes, scales, R, C, flags, seed, y, stream):
+    return int(load().mxfp4_dequantize(codes, scales, R, C, flags, seed, y, stream))
 
 
 def nvfp4_status_string(status):

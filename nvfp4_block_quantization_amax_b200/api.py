@@ -147,3 +147,50 @@ def nvfp4_gemm_quantize(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor,
                                mode, flags, _p(alpha_out), _p(codes), _p(scales), _p(amax), None, 0, _stream())
     _check(st, "nvfp4_gemm_quantize")
     return D, codes, scales, amax
+
+
+@dataclass
+class MXTensor:
+    """MXFP4 outputs of one quantize call (device tensors): codes [rows, len/2],
+    UE8M0 scale bytes [rows, len/32] per requested orientation."""
+    codes_row: Optional[torch.Tensor] = None
+    scales_row: Optional[torch.Tensor] = None
+    codes_col: Optional[torch.Tensor] = None
+    scales_col: Optional[torch.Tensor] = None
+
+
+def mxfp4_quantize(x: torch.Tensor, flags: int, seed: int = 0, status: Optional[torch.Tensor] = None,
+                   out: Optional[MXTensor] = None) -> MXTensor:
+    """Quantize a 2D bf16 CUDA tensor (unit column stride) to MXFP4 with the C
+    ABI's mxfp4_quantize (flags: NVFP4_ROWWISE / NVFP4_COLWISE, NVFP4_RHT)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2D bfloat16 CUDA tensor")
+    if x.numel() and x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    R, C = x.shape
+    ld = x.stride(0) if x.numel() else C
+    q = out
+    if q is None:
+        q = MXTensor()
+        u8 = dict(dtype=torch.uint8, device=x.device)
+        if flags & NVFP4_ROWWISE:
+            q.codes_row = torch.empty((R, C // 2), **u8)
+            q.scales_row = torch.empty((R, C // 32), **u8)
+        if flags & NVFP4_COLWISE:
+            q.codes_col = torch.empty((C, R // 2), **u8)
+            q.scales_col = torch.empty((C, R // 32), **u8)
+    st = L.mxfp4_quantize(_p(x), R, C, ld, flags, seed, _p(q.codes_row), _p(q.scales_row), _p(q.codes_col),
+                          _p(q.scales_col), _p(status), _stream())
+    _check(st, "mxfp4_quantize")
+    return q
+
+
+def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, R: int, C: int, flags: int = 0, seed: int = 0,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Decode MXFP4 codes [R, C/2] and scales [R, C/32] to fp32 (or bf16 with
+    NVFP4_OUT_BF16)."""
+    dtype = torch.bfloat16 if flags & NVFP4_OUT_BF16 else torch.float32
+    y = out if out is not None else torch.empty((R, C), dtype=dtype, device=codes.device)
+    st = L.mxfp4_dequantize(_p(codes), _p(scales), R, C, flags, seed, _p(y), _stream())
+    _check(st, "mxfp4_dequantize")
+    return y

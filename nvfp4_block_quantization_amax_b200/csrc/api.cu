@@ -36,6 +36,37 @@ extern "C" {
 
 uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
+                              uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col, uint8_t* scales_col,
+                              int32_t* status, void* stream) {
+  if (flags & ~(NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_RHT)) return NVFP4_ERR_ARG;
+  const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE;
+  if (!row && !col) return NVFP4_ERR_ARG;
+  if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
+  if (C % 16 || (row && C % 32) || (col && R % 32)) return NVFP4_ERR_SHAPE;
+  if (R * (C / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (R == 0 || C == 0) return NVFP4_OK;
+  if (!x || (row && (!codes_row || !scales_row)) || (col && (!codes_col || !scales_col))) return NVFP4_ERR_ARG;
+  if (!aligned(x, 16) || ld % 8) return NVFP4_ERR_ALIGN;
+  if ((row && !aligned(codes_row, 16)) || (col && !aligned(codes_col, 16))) return NVFP4_ERR_ALIGN;
+  return launch_status(nvfp4::mx_quantize_launch(x, R, C, ld, flags, seed, row ? codes_row : nullptr,
+                                                 row ? scales_row : nullptr, col ? codes_col : nullptr,
+                                                 col ? scales_col : nullptr, status,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status_t mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t C, uint32_t flags,
+                                uint64_t seed, void* y, void* stream) {
+  if (flags & ~(NVFP4_INVERSE_RHT | NVFP4_OUT_BF16)) return NVFP4_ERR_ARG;
+  if (R < 0 || C < 0 || C % 32) return NVFP4_ERR_SHAPE;
+  if (R * (C / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (R == 0 || C == 0) return NVFP4_OK;
+  if (!codes || !scales || !y) return NVFP4_ERR_ARG;
+  if (!aligned(codes, 8) || !aligned(y, 16)) return NVFP4_ERR_ALIGN;
+  return launch_status(nvfp4::mx_dequantize_launch(codes, scales, R, C, flags, seed, y,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_version(void) { return 10000; }
 
 const char* nvfp4_status_string(nvfp4_status_t s) {

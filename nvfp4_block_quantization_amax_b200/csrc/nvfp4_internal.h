@@ -65,4 +65,11 @@ cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const floa
                                  int64_t ldd, int mode, bool gemm_layout, const float* alpha_out, uint8_t* codes,
                                  uint8_t* scales, float* amax_out, int32_t* status, cudaStream_t st);
 
+// MXFP4 (mx.cu): one tile kernel for rows and / or columns; dequantization.
+cudaError_t mx_quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
+                               uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col, uint8_t* scales_col,
+                               int32_t* status, cudaStream_t st);
+cudaError_t mx_dequantize_launch(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t C, uint32_t flags,
+                                 uint64_t seed, void* y, cudaStream_t st);
+
 }  // namespace nvfp4

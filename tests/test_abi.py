@@ -12,7 +12,7 @@ HEADER = os.path.join(ROOT, "include", "nvfp4.h")
 
 def declared_functions():
     text = open(HEADER).read()
-    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b((?:nv|mx)fp4_\w+)\s*\(", text)
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +25,7 @@ def lib():
 def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert {"nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_workspace_size",
-            "nvfp4_status_string", "nvfp4_version"} <= names
+            "nvfp4_status_string", "nvfp4_version", "mxfp4_quantize", "mxfp4_dequantize"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -94,3 +94,28 @@ def test_host_argument_checks_need_no_gpu(lib):
                                  fake, None, None, 0, None) == L.NVFP4_ERR_ARG
     assert L.nvfp4_gemm_quantize(fake, fake, fake, fake, fake, fake, 256, 256, 128, None, 256, 1, 0, None, fake,
                                  fake, None, None, 0, None) == L.NVFP4_ERR_ARG
+
+
+def test_mxfp4_host_checks_need_no_gpu(lib):
+    from nvfp4_block_quantization_amax_b200 import _lib as L
+    fake = 0x10000  # never dereferenced: every call below fails its checks first
+    ROW, COL = L.NVFP4_ROWWISE, L.NVFP4_COLWISE
+    q = lambda x, R, C, ld, flags, cr=fake, sr=fake, cc=fake, sc=fake: L.mxfp4_quantize(
+        x, R, C, ld, flags, 0, cr, sr, cc, sc, None, None)
+    assert q(fake, 32, 32, 32, 0) == L.NVFP4_ERR_ARG                      # no orientation
+    assert q(fake, 32, 32, 32, ROW | L.NVFP4_BLOCK2D) == L.NVFP4_ERR_ARG  # NVFP4-only flag
+    assert q(fake, 32, 48, 48, ROW) == L.NVFP4_ERR_SHAPE                  # rows need C % 32
+    assert q(fake, 48, 32, 32, COL) == L.NVFP4_ERR_SHAPE                  # columns need R % 32
+    assert q(fake, 32, 32, 16, ROW) == L.NVFP4_ERR_SHAPE                  # ld < C
+    assert q(fake, 32, 32, 32, ROW, cr=None) == L.NVFP4_ERR_ARG
+    assert q(fake, 32, 32, 32, COL, sc=None) == L.NVFP4_ERR_ARG
+    assert q(fake + 2, 32, 32, 32, ROW) == L.NVFP4_ERR_ALIGN
+    assert q(fake, 32, 32, 36, ROW) == L.NVFP4_ERR_ALIGN                  # ld % 8
+    assert q(fake, 32, 32, 32, ROW, cr=fake + 8) == L.NVFP4_ERR_ALIGN
+    assert q(None, 0, 32, 32, ROW) == L.NVFP4_OK                          # empty: no-op
+    d = L.mxfp4_dequantize
+    assert d(fake, fake, 16, 48, 0, 0, fake, None) == L.NVFP4_ERR_SHAPE
+    assert d(fake, fake, 16, 32, L.NVFP4_BLOCK2D, 0, fake, None) == L.NVFP4_ERR_ARG
+    assert d(None, fake, 16, 32, 0, 0, fake, None) == L.NVFP4_ERR_ARG
+    assert d(fake + 4, fake, 16, 32, 0, 0, fake, None) == L.NVFP4_ERR_ALIGN
+    assert d(None, None, 0, 32, 0, 0, None, None) == L.NVFP4_OK

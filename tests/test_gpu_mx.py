@@ -1,0 +1,117 @@
+"""GPU parity of the MXFP4 path (mxfp4_quantize / mxfp4_dequantize through
+the C ABI) against the CPU oracle: codes and UE8M0 scale bytes bit-exact,
+dequantized values exact (fp32) or equal after the same bf16 rounding."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_block_quantization_amax_b200 import synthetic
+
+pytestmark = pytest.mark.gpu
+
+ROW, COL, RHT, INV, BF16 = 0x1, 0x2, 0x40, 0x80, 0x100
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from nvfp4_block_quantization_amax_b200 import api as _api
+    return _api
+
+
+def run_both(api, x, flags, seed=0):
+    q = api.mxfp4_quantize(x.cuda(), flags, seed=seed)
+    torch.cuda.synchronize()
+    o = oracle.mx_quantize(synthetic.bf16_bits(x), flags, seed=seed)
+    for side, bit in (("row", ROW), ("col", COL)):
+        if flags & bit:
+            assert np.array_equal(getattr(q, f"scales_{side}").cpu().numpy(), o[f"scales_{side}"]), side
+            assert np.array_equal(getattr(q, f"codes_{side}").cpu().numpy(), o[f"codes_{side}"]), side
+    return q, o
+
+
+@pytest.mark.parametrize("orient", [ROW, COL, ROW | COL])
+@pytest.mark.parametrize("rot", [0, RHT])
+def test_pr1_shapes(api, orient, rot):
+    x = synthetic.pr1()["x"]
+    run_both(api, x, orient | rot, seed=17)
+
+
+@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (64, 128), (1056, 1568), (224, 4128)])
+@pytest.mark.parametrize("rot", [0, RHT])
+def test_ragged_and_many_tiles(api, shape, rot):
+    x = synthetic.normal_with_entry_outliers(*shape, seed=shape[0] + shape[1])
+    run_both(api, x, ROW | COL | rot, seed=3)
+
+
+@pytest.mark.parametrize("shape", [(37, 64), (1, 32), (5, 96)])
+def test_rows_only_any_row_count(api, shape):
+    run_both(api, synthetic.weight(*shape, seed=1), ROW)
+
+
+def test_every_bf16_value_through_the_encoder(api):
+    # blocks [6, v1..v31]: the block maximum is 6, so e = 0 and y = v for every
+    # bf16 v in [-6, 6], ties included
+    bits = np.arange(65536, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32)
+    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 6)]
+    n = -(-len(vals) // 31)
+    pad = np.zeros(n * 31, np.float32)
+    pad[:len(vals)] = vals
+    blocks = np.concatenate([np.full((n, 1), 6.0, np.float32), pad.reshape(n, 31)], axis=1)
+    R = -(-n // 4)
+    arr = np.zeros((R * 4, 32), np.float32)
+    arr[:n] = blocks
+    run_both(api, synthetic.to_bf16(arr.reshape(R, 128)), ROW)
+
+
+def test_extreme_exponents_and_zeros(api):
+    rng = np.random.default_rng(8)
+    a = rng.standard_normal((64, 256)).astype(np.float64)
+    a *= np.exp2(rng.integers(-133, 126, (64, 1)).astype(np.float64))   # subnormal to near-max bf16 rows
+    a[5] = 0.0
+    a[6, :32] = -0.0
+    a[7, 3] = 3.0e38
+    x = synthetic.to_bf16(np.clip(a, -3.0e38, 3.0e38).astype(np.float32))
+    run_both(api, x, ROW | COL)
+    run_both(api, x, ROW | COL | RHT, seed=2)
+
+
+def test_nonfinite_sets_status(api):
+    for v in (float("inf"), float("nan")):
+        x = torch.zeros((64, 128), dtype=torch.bfloat16)
+        x[40, 77] = v
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        api.mxfp4_quantize(x.cuda(), ROW | COL, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == -4
+
+
+@pytest.mark.parametrize("flags", [0, BF16, INV, INV | BF16])
+def test_dequantize_matches_oracle(api, flags):
+    x = synthetic.normal_with_channel_outliers(256, 1024, seed=4)
+    rot = RHT if flags & INV else 0
+    q = api.mxfp4_quantize(x.cuda(), ROW | rot, seed=11)
+    y = api.mxfp4_dequantize(q.codes_row, q.scales_row, 256, 1024, flags, seed=11)
+    torch.cuda.synchronize()
+    want = oracle.mx_dequantize(q.codes_row.cpu().numpy(), q.scales_row.cpu().numpy(), 256, 1024,
+                                flags & INV, seed=11)
+    if flags & BF16:
+        assert torch.equal(y.cpu(), torch.from_numpy(want).to(torch.bfloat16))
+    else:
+        assert np.array_equal(y.cpu().numpy(), want)
+
+
+def test_full_size_activation_dual_rotated(api):
+    """X [8192, 4096] rows + columns with the fixed rotation: the first 1024
+    rows (32-row column blocks never cross them) compared in full."""
+    x = synthetic.fwd_bwd_8b(seed=0)["x"]
+    q = api.mxfp4_quantize(x.cuda(), ROW | COL | RHT, seed=0)
+    torch.cuda.synchronize()
+    o = oracle.mx_quantize(synthetic.bf16_bits(x[:1024]), ROW | COL | RHT, seed=0)
+    assert np.array_equal(q.codes_row[:1024].cpu().numpy(), o["codes_row"])
+    assert np.array_equal(q.scales_row[:1024].cpu().numpy(), o["scales_row"])
+    assert np.array_equal(q.codes_col[:, :512].cpu().numpy(), o["codes_col"])
+    assert np.array_equal(q.scales_col[:, :32].cpu().numpy(), o["scales_col"])
