@@ -65,3 +65,13 @@ def test_step_accounting():
     assert flops == 3 * 2 * 8192 * 14336 * 4096
     calls = bench.quant_calls()
     assert [n for _, n, _ in calls] == [8192 * 4096, 14336 * 4096, 8192 * 14336, 14336 * 4096, 8192 * 4096]
+
+
+@pytest.mark.parametrize("mode", sorted(bench.BWD_MODES))
+def test_reference_arm_sample_runs_in_every_backward_mode(mode):
+    """The CPU reference arm times the oracle on a bounded sample in each
+    backward mode the bench offers, and names that mode in its workload."""
+    dt, desc, threads = bench.oracle_sample(budget_rows=1, gemm_rows=2, gemm_cols=2, bwd_mode=mode)
+    assert dt > 0 and threads >= 1
+    assert "dY rows+cols: 16x14336" in desc
+    assert bench.BWD_NAMES[mode] in bench.workload(mode)
