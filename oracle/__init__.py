@@ -94,6 +94,8 @@ def lib():
         L.oracle_mx_quantize.restype = ctypes.c_int
         L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64, _f32p]
         L.oracle_mx_dequantize.restype = ctypes.c_int
+        L.oracle_mx_gemm_f64.argtypes = [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
+        L.oracle_mx_gemm_f64.restype = None
         _lib = L
     return _lib
 
@@ -360,3 +362,20 @@ def mx_dequantize(codes, scales, R, C, flags=0, seed=0):
     y = np.zeros((R, C), np.float32)
     _check(lib().oracle_mx_dequantize(_p(codes, _u8p), _p(scales, _u8p), R, C, flags, seed, _p(y, _f32p)))
     return y
+
+
+def mx_gemm_f64(A, sA, B, sB, M, N, K, rows=None, cols=None):
+    """FP64 reference D = (qA 2^eA)(qB 2^eB)^T for MXFP4 operands (row-major
+    UE8M0 scales) on the given rows / columns (None = all)."""
+    A = _c(A, np.uint8)
+    B = _c(B, np.uint8)
+    sA = _c(sA, np.uint8)
+    sB = _c(sB, np.uint8)
+    r = None if rows is None else _c(rows, np.int64)
+    c = None if cols is None else _c(cols, np.int64)
+    nr = M if r is None else len(r)
+    nc = N if c is None else len(c)
+    D = np.zeros((nr, nc), np.float64)
+    lib().oracle_mx_gemm_f64(_p(A, _u8p), _p(sA, _u8p), _p(B, _u8p), _p(sB, _u8p), M, N, K,
+                             _p(r, _i64p), nr, _p(c, _i64p), nc, _p(D, _f64p))
+    return D

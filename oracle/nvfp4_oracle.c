@@ -849,3 +849,36 @@ int oracle_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R,
     }
   return OR_OK;
 }
+
+/* MXFP4 GEMM reference in FP64: D[m, n] = sum_k (qA 2^eA)(qB 2^eB) for TN
+ * operands A [M, K] and B [N, K] (codes [rows, K/2], UE8M0 scales
+ * [rows, K/32] row-major); no tensor scales.  Rows / columns as for
+ * oracle_gemm_f64. */
+void oracle_mx_gemm_f64(const uint8_t* A, const uint8_t* sA, const uint8_t* B,
+                        const uint8_t* sB, int64_t M, int64_t N, int64_t K,
+                        const int64_t* rows, int64_t nrows, const int64_t* cols,
+                        int64_t ncols, double* D) {
+  if (!rows) nrows = M;
+  if (!cols) ncols = N;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t m = rows ? rows[i] : i;
+    double* arow = (double*)malloc(sizeof(double) * (size_t)K);
+    for (int64_t k = 0; k < K; ++k) {
+      uint8_t byte = A[m * (K / 2) + k / 2];
+      uint8_t q = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+      arow[k] = (double)oracle_e2m1_value(q) * (double)oracle_e8m0_value(sA[m * (K / 32) + k / 32]);
+    }
+    for (int64_t j = 0; j < ncols; ++j) {
+      int64_t n = cols ? cols[j] : j;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        uint8_t byte = B[n * (K / 2) + k / 2];
+        uint8_t q = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+        acc += arow[k] * (double)oracle_e2m1_value(q) * (double)oracle_e8m0_value(sB[n * (K / 32) + k / 32]);
+      }
+      D[i * ncols + j] = acc;
+    }
+    free(arow);
+  }
+}

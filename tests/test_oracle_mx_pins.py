@@ -173,3 +173,22 @@ def test_errors():
         oracle.mx_quantize(x, ROW)
     z = oracle.mx_quantize(np.zeros((32, 32), np.uint16), ROW | COL)
     assert (z["scales_row"] == 0).all() and (z["codes_row"] == 0).all()
+
+
+def test_mx_gemm_matches_numpy_on_library_decoded_operands():
+    """The FP64 MXFP4 GEMM equals numpy's float64 matmul of the operands
+    decoded with ml_dtypes (E2M1 x UE8M0), on all and on selected outputs."""
+    rng = np.random.default_rng(12)
+    M, N, K = 48, 40, 256
+    A = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    B = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sA = rng.integers(100, 150, (M, K // 32), dtype=np.uint8)
+    sB = rng.integers(100, 150, (N, K // 32), dtype=np.uint8)
+    da = e2m1_lib_value(nibbles(A)).astype(np.float64) * np.repeat(e8m0_lib_value(sA), 32, 1)
+    db = e2m1_lib_value(nibbles(B)).astype(np.float64) * np.repeat(e8m0_lib_value(sB), 32, 1)
+    want = da @ db.T
+    got = oracle.mx_gemm_f64(A, sA, B, sB, M, N, K)
+    assert np.allclose(got, want, rtol=1e-12, atol=0)
+    rows, cols = np.array([3, 47, 0]), np.array([39, 5])
+    sub = oracle.mx_gemm_f64(A, sA, B, sB, M, N, K, rows=rows, cols=cols)
+    assert np.array_equal(sub, got[np.ix_(rows, cols)])
