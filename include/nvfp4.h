@@ -266,7 +266,10 @@ NVFP4_API nvfp4_status_t nvfp4_gemm_quantize(const uint8_t* A, const uint8_t* sA
  *   flags: NVFP4_ROWWISE and / or NVFP4_COLWISE, optionally NVFP4_RHT (each
  *     16-element half of a block is first rotated by (1/4) H16 D, D the sign
  *     diagonal drawn from `seed` exactly as for nvfp4_quantize; a fixed seed
- *     gives the fixed rotation).
+ *     gives the fixed rotation) and NVFP4_GEMM_SCALE_LAYOUT (scales written
+ *     in the GEMM layout described at NVFP4_GEMM_SCALE_LAYOUT, with K-blocks
+ *     of 32 elements: one 512-byte atom per 128 rows x 128 K; R % 128 == 0
+ *     and C % 128 == 0).
  *   rowwise: codes_row [R, C/2] (element 2j in the low nibble), scales_row
  *     [R, C/32] row-major.  columnwise (blocks of 32 rows of a column, stored
  *     transposed): codes_col [C, R/2], scales_col [C, R/32].
@@ -280,6 +283,18 @@ NVFP4_API nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int
                                         uint64_t seed, uint8_t* codes_row, uint8_t* scales_row,
                                         uint8_t* codes_col, uint8_t* scales_col, int32_t* status,
                                         void* stream);
+
+/* Block-scaled MXFP4 GEMM on the tcgen05 tensor cores:
+ *     D[m, n] = sum_k (qA[m,k] 2^eA[m,k/32]) (qB[n,k] 2^eB[n,k/32])
+ * A: codes [M, K/2], B: codes [N, K/2] (K-major, "TN"); sA, sB: UE8M0 scales
+ * in the GEMM layout (mxfp4_quantize with NVFP4_GEMM_SCALE_LAYOUT).  No
+ * tensor scales.  FP32 accumulation; D bf16 (NVFP4_OUT_DTYPE_BF16) or fp32,
+ * row-major with row stride ldd elements.  M % 256 == 0, N % 256 == 0,
+ * K % 128 == 0 (the CTA-pair kernel); A, B, sA, sB, D 16-byte aligned.  The
+ * workspace is optional as for nvfp4_gemm (status word). */
+NVFP4_API nvfp4_status_t mxfp4_gemm(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB,
+                                    int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Decode MXFP4 codes [R, C/2] with scales [R, C/32]:  y = q * 2^(byte - 127),
  * optionally followed by the inverse rotation D (1/4) H16 of each 16-element

@@ -31,7 +31,7 @@ NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
 EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
-            "nvfp4_gemm", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "nvfp4_launch_count",
+            "nvfp4_gemm", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "nvfp4_launch_count",
             "nvfp4_status_string", "nvfp4_version")
 
 
@@ -73,6 +73,8 @@ def load(path=LIB_PATH):
     L.mxfp4_quantize.argtypes = [vp, i64, i64, i64, u32, u64, vp, vp, vp, vp, vp, vp]
     L.mxfp4_quantize.restype = ctypes.c_int
     L.mxfp4_dequantize.argtypes = [vp, vp, i64, i64, u32, u64, vp, vp]
+    L.mxfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
+    L.mxfp4_gemm.restype = ctypes.c_int
     L.mxfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_status_string.argtypes = [ctypes.c_int]
     L.nvfp4_status_string.restype = ctypes.c_char_p
@@ -122,6 +124,10 @@ def nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, fla
 def mxfp4_quantize(x, R, C, ld, flags, seed, codes_row, scales_row, codes_col, scales_col, status, stream):
     return int(load().mxfp4_quantize(x, R, C, ld, flags, seed, codes_row, scales_row, codes_col, scales_col,
                                      status, stream))
+
+
+def mxfp4_gemm(A, sA, B, sB, M, N, K, D, out_dtype, ldd, workspace, workspace_bytes, stream):
+    return int(load().mxfp4_gemm(A, sA, B, sB, M, N, K, D, out_dtype, ldd, workspace, workspace_bytes, stream))
 
 
 def mxfp4_dequantize(codes, scales, R, C, flags, seed, y, stream):

@@ -173,12 +173,13 @@ def mxfp4_quantize(x: torch.Tensor, flags: int, seed: int = 0, status: Optional[
     if q is None:
         q = MXTensor()
         u8 = dict(dtype=torch.uint8, device=x.device)
+        gemm = bool(flags & NVFP4_GEMM_SCALE_LAYOUT)
         if flags & NVFP4_ROWWISE:
             q.codes_row = torch.empty((R, C // 2), **u8)
-            q.scales_row = torch.empty((R, C // 32), **u8)
+            q.scales_row = torch.empty((R * (C // 32),) if gemm else (R, C // 32), **u8)
         if flags & NVFP4_COLWISE:
             q.codes_col = torch.empty((C, R // 2), **u8)
-            q.scales_col = torch.empty((C, R // 32), **u8)
+            q.scales_col = torch.empty((C * (R // 32),) if gemm else (C, R // 32), **u8)
     st = L.mxfp4_quantize(_p(x), R, C, ld, flags, seed, _p(q.codes_row), _p(q.scales_row), _p(q.codes_col),
                           _p(q.scales_col), _p(status), _stream())
     _check(st, "mxfp4_quantize")
@@ -194,3 +195,17 @@ def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, R: int, C: int, 
     st = L.mxfp4_dequantize(_p(codes), _p(scales), R, C, flags, seed, _p(y), _stream())
     _check(st, "mxfp4_dequantize")
     return y
+
+
+def mxfp4_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Tensor,
+               out_dtype: int = NVFP4_OUT_DTYPE_BF16, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """D[M, N] = (A dequantized) (B dequantized)^T for MXFP4 operands: codes
+    [M, K/2] and [N, K/2], UE8M0 scales in the GEMM layout."""
+    M, K2 = A.shape
+    N = B.shape[0]
+    K = 2 * K2
+    dt = torch.bfloat16 if out_dtype == NVFP4_OUT_DTYPE_BF16 else torch.float32
+    D = out if out is not None else torch.empty((M, N), dtype=dt, device=A.device)
+    st = L.mxfp4_gemm(_p(A), _p(sA), _p(B), _p(sB), M, N, K, _p(D), out_dtype, D.stride(0), None, 0, _stream())
+    _check(st, "mxfp4_gemm")
+    return D

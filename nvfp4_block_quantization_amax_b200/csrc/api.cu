@@ -39,11 +39,12 @@ uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_rel
 nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
                               uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col, uint8_t* scales_col,
                               int32_t* status, void* stream) {
-  if (flags & ~(NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_RHT)) return NVFP4_ERR_ARG;
+  if (flags & ~(NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_RHT | NVFP4_GEMM_SCALE_LAYOUT)) return NVFP4_ERR_ARG;
   const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE;
   if (!row && !col) return NVFP4_ERR_ARG;
   if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (C % 16 || (row && C % 32) || (col && R % 32)) return NVFP4_ERR_SHAPE;
+  if ((flags & NVFP4_GEMM_SCALE_LAYOUT) && (R % 128 || C % 128)) return NVFP4_ERR_SHAPE;
   if (R * (C / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
   if (R == 0 || C == 0) return NVFP4_OK;
   if (!x || (row && (!codes_row || !scales_row)) || (col && (!codes_col || !scales_col))) return NVFP4_ERR_ARG;
@@ -53,6 +54,24 @@ nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, u
                                                  row ? scales_row : nullptr, col ? codes_col : nullptr,
                                                  col ? scales_col : nullptr, status,
                                                  static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status_t mxfp4_gemm(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB, int64_t M,
+                          int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (out_dtype != NVFP4_OUT_DTYPE_BF16 && out_dtype != NVFP4_OUT_DTYPE_FP32) return NVFP4_ERR_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return NVFP4_ERR_SHAPE;
+  if (M % 256 || N % 256 || K % 128 || ldd < N) return NVFP4_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (!A || !sA || !B || !sB || !D) return NVFP4_ERR_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) || !aligned(sB, 16) || !aligned(D, 16))
+    return NVFP4_ERR_ALIGN;
+  if ((ldd * (out_dtype == NVFP4_OUT_DTYPE_BF16 ? 2 : 4)) % 16) return NVFP4_ERR_ALIGN;
+  int32_t* status = (workspace && workspace_bytes >= sizeof(int32_t) && aligned(workspace, 4))
+                        ? static_cast<int32_t*>(workspace)
+                        : nullptr;
+  return launch_status(nvfp4::mx_gemm_launch(A, sA, B, sB, M, N, K, D, out_dtype, ldd, status,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status_t mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t C, uint32_t flags,

@@ -259,6 +259,19 @@ __device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t tmem_d, uint64_t ades
       : "memory");
 }
 
+// MXFP4 operands: E2M1 values with UE8M0 scales per 32 K (two scale bytes per
+// row per K = 64 MMA, chosen inside each 32-bit TMEM scale column by the
+// descriptor's scale-factor ids).
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate, uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -534,19 +547,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ===========================================================================
 constexpr int P_STAGE_A = 128 * BK_BYTES;        // own A rows
 constexpr int P_STAGE_B = 128 * BK_BYTES;        // own B rows
-constexpr int P_STAGE_SFA = KB_PER_STAGE * 512;  // own A rows' scales
-constexpr int P_STAGE_SFB = 2 * KB_PER_STAGE * 512;  // all 256 B rows' scales
-constexpr int P_STAGE = P_STAGE_A + P_STAGE_B + P_STAGE_SFA + P_STAGE_SFB;
 constexpr int P_EPI_WARPS = 8;                   // two per TMEM lane quarter, 128 columns each
 constexpr int P_THREADS = 64 + 32 * P_EPI_WARPS;
 constexpr int P_OUT_STAGING = P_EPI_WARPS * 2048;
-constexpr int P_STAGES = (232448 - P_OUT_STAGING - 1024 - 512) / P_STAGE;
-constexpr int P_SMEM = P_STAGES * P_STAGE + P_OUT_STAGING + 1024 + 512;
+// Per-stage scale data: 512-byte atoms of 128 rows x 4 scale bytes.  NVFP4
+// (16-element blocks) needs 4 atoms per 128 rows for a K = 256 stage, MXFP4
+// (32-element blocks) 2.
+template <bool MX>
+struct PairCfg {
+  static constexpr int ATOMS = MX ? 2 : KB_PER_STAGE;
+  static constexpr int SFA = ATOMS * 512;       // own A rows' scales
+  static constexpr int SFB = 2 * ATOMS * 512;   // all 256 B rows' scales
+  static constexpr int STAGE = P_STAGE_A + P_STAGE_B + SFA + SFB;
+  static constexpr int STAGES = (232448 - P_OUT_STAGING - 1024 - 512) / STAGE;
+  static constexpr int SMEM = STAGES * STAGE + P_OUT_STAGING + 1024 + 512;
+};
 constexpr uint32_t P_SF_W = 4 + 8;               // SFA 4 + SFB (256 rows) 8 columns per K block
 constexpr uint32_t P_SF_COL = 256;
 constexpr uint32_t P_TMEM_COLS = 512;            // 256 accumulator + 2 x 4 K blocks x 12 scale columns
 // M = 256 (>> 4 = 16 at bit 24), N = 256 (>> 3 = 32 at bit 17), E2M1 x E2M1, E4M3 scales
 constexpr uint32_t P_IDESC = (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((256u >> 4) << 24);
+// MXFP4: the same with UE8M0 scales (bit 23); the scale-factor ids (bits
+// 29-30 for A, 4-5 for B) are added per MMA.
+constexpr uint32_t P_IDESC_MX = P_IDESC | (1u << 23);
 
 // Optional NVFP4 quantization of the bf16 output rows in the epilogue (the
 // next layer's rowwise input), with a provided tensor scale.
@@ -567,26 +590,27 @@ __device__ __forceinline__ int64_t gemm_scale_byte(int64_t m, int64_t j, int64_t
   return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
 }
 
-template <int QMODE>
+template <int QMODE, bool MX = false>
 __global__ void __launch_bounds__(P_THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
                            const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
                            const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status,
                            const EpiQuant eq) {
+  using PC = PairCfg<MX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + P_STAGES * P_STAGE_A;
-  uint8_t* sSFA = sB + P_STAGES * P_STAGE_B;
-  uint8_t* sSFB = sSFA + P_STAGES * P_STAGE_SFA;
-  uint8_t* sOut = sSFB + P_STAGES * P_STAGE_SFB;
+  uint8_t* sB = sA + PC::STAGES * P_STAGE_A;
+  uint8_t* sSFA = sB + PC::STAGES * P_STAGE_B;
+  uint8_t* sSFB = sSFA + PC::STAGES * PC::SFA;
+  uint8_t* sOut = sSFB + PC::STAGES * PC::SFB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + P_OUT_STAGING);
   uint64_t* full = bars;
-  uint64_t* empty = bars + P_STAGES;
-  uint64_t* acc_full = bars + 2 * P_STAGES;
-  uint64_t* acc_empty = bars + 2 * P_STAGES + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * P_STAGES + 2);
+  uint64_t* empty = bars + PC::STAGES;
+  uint64_t* acc_full = bars + 2 * PC::STAGES;
+  uint64_t* acc_empty = bars + 2 * PC::STAGES + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PC::STAGES + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -596,10 +620,11 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   const int m_tiles = M / 256;
   const int num_tiles = m_tiles * (N / 256);
   const int kblocks64 = K / 64;
+  const int katoms = MX ? K / 128 : K / 64;   // scale atoms along K per 128 rows
   const int kstages = (K + 255) / 256;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < P_STAGES; ++s) {
+    for (int s = 0; s < PC::STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
@@ -627,8 +652,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
       const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
       for (int kt = 0; kt < kstages; ++kt, ++it) {
-        const int s = it % P_STAGES;
-        const uint32_t ph = (it / P_STAGES) & 1;
+        const int s = it % PC::STAGES;
+        const uint32_t ph = (it / PC::STAGES) & 1;
         bool ok = true;
         if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), ph ^ 1, abort_flag);
         if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
@@ -637,24 +662,24 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         }
         const uint32_t fb_leader = map_to_rank(smem_u32(&full[s]), 0);
         const uint32_t dA = smem_u32(sA + s * P_STAGE_A), dB = smem_u32(sB + s * P_STAGE_B);
-        const uint32_t dSA = smem_u32(sSFA + s * P_STAGE_SFA), dSB = smem_u32(sSFB + s * P_STAGE_SFB);
+        const uint32_t dSA = smem_u32(sSFA + s * PC::SFA), dSB = smem_u32(sSFB + s * PC::SFB);
         // scale atoms viewed as rows of 256 bytes: a stage is 8 rows per 128 operand rows
-        const int ysa = ((tile_m * 2 + static_cast<int>(rank)) * kblocks64 + KB_PER_STAGE * kt) * 2;
-        const int ysb = ((tile_n * 2) * kblocks64 + KB_PER_STAGE * kt) * 2;
+        const int ysa = ((tile_m * 2 + static_cast<int>(rank)) * katoms + PC::ATOMS * kt) * 2;
+        const int ysb = ((tile_n * 2) * katoms + PC::ATOMS * kt) * 2;
         if (elect_one()) {
-          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * P_STAGE);
+          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * PC::STAGE);
           tma_load_2d_pair(dA, &tmap_a, kt * BK_BYTES, tile_m * 256 + 128 * rank, fb_leader);
           tma_load_2d_pair(dB, &tmap_b, kt * BK_BYTES, tile_n * 256 + 128 * rank, fb_leader);
           tma_load_2d_pair(dSA, &tmap_sfa, 0, ysa, fb_leader);
           tma_load_2d_pair(dSB, &tmap_sfb, 0, ysb, fb_leader);
-          tma_load_2d_pair(dSB + P_STAGE_SFA, &tmap_sfb, 0, ysb + 2 * kblocks64, fb_leader);
+          tma_load_2d_pair(dSB + PC::SFA, &tmap_sfb, 0, ysb + 2 * katoms, fb_leader);
         }
         __syncwarp();
       }
     }
     if (lane == 0 && *abort_flag && leader) {
-      for (int i = (it > P_STAGES ? it - P_STAGES : 0); i < it; ++i) {
-        const uint32_t bar = smem_u32(&full[i % P_STAGES]), ph = (i / P_STAGES) & 1;
+      for (int i = (it > PC::STAGES ? it - PC::STAGES : 0); i < it; ++i) {
+        const uint32_t bar = smem_u32(&full[i % PC::STAGES]), ph = (i / PC::STAGES) & 1;
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
         }
@@ -666,33 +691,43 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
       const int total = my_tiles * kstages;
       for (int g = 0; g < total; ++g) {
-        const int kt = g % kstages, ti = g / kstages, s = g % P_STAGES;
+        const int kt = g % kstages, ti = g / kstages, s = g % PC::STAGES;
         bool ok = true;
         if (kt == 0) {
           if (lane == 0) ok = mbar_wait(smem_u32(acc_empty), (ti & 1) ^ 1, abort_flag);
           if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
           fence_after();
         }
-        if (lane == 0) ok = mbar_wait(smem_u32(&full[s]), (g / P_STAGES) & 1, abort_flag);
+        if (lane == 0) ok = mbar_wait(smem_u32(&full[s]), (g / PC::STAGES) & 1, abort_flag);
         if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
         fence_after();
-        const uint32_t sfa_s = smem_u32(sSFA + s * P_STAGE_SFA);
-        const uint32_t sfb_s = smem_u32(sSFB + s * P_STAGE_SFB);
+        const uint32_t sfa_s = smem_u32(sSFA + s * PC::SFA);
+        const uint32_t sfb_s = smem_u32(sSFB + s * PC::SFB);
         const uint32_t set = static_cast<uint32_t>(g & 1) * KB_PER_STAGE;
         const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
         const uint64_t adesc = desc_sw128(smem_u32(sA + s * P_STAGE_A));
         const uint64_t bdesc = desc_sw128(smem_u32(sB + s * P_STAGE_B));
         if (elect_one()) {
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
-            tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * kk));
-            tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * kk));
-            tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + P_STAGE_SFA + 512 * kk));
+          // one scale atom per K = 64 MMA (NVFP4) or per two of them (MXFP4)
+          const int na = MX ? (nk + 1) / 2 : nk;
+          for (int ka = 0; ka < na; ++ka) {
+            const uint32_t col = tmem + P_SF_COL + (set + ka) * P_SF_W;
+            tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * ka));
+            tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * ka));
+            tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + PC::SFA + 512 * ka));
           }
           for (int kk = 0; kk < nk; ++kk) {
-            const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
-            mma_mxf4nvf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col,
-                              col + 4);
+            const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (MX) {
+              // MMA kk reads scale bytes 2 (kk & 1), +1 of atom kk / 2's columns
+              const uint32_t col = tmem + P_SF_COL + (set + kk / 2) * P_SF_W;
+              const uint32_t sf_id = 2u * static_cast<uint32_t>(kk & 1);
+              mma_mxf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC_MX | (sf_id << 29) | (sf_id << 4), acc,
+                            col, col + 4);
+            } else {
+              const uint32_t col = tmem + P_SF_COL + (set + kk) * P_SF_W;
+              mma_mxf4nvf4_pair(tmem, adesc + 2 * kk, bdesc + 2 * kk, P_IDESC, acc, col, col + 4);
+            }
           }
           umma_commit_pair(smem_u32(&empty[s]));
           if (kt == kstages - 1) umma_commit_pair(smem_u32(acc_full));
@@ -706,7 +741,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     // quarter, each converting and storing half of the tile's columns.
     const int q = warp & 3, h = (warp - 2) >> 2;
     uint8_t* buf = sOut + (warp - 2) * 2048;
-    const float ab = __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
+    const float ab = MX ? 1.0f : __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));   // MXFP4: no tensor scales
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
     float eq_alpha = 0.0f, epi_amax = 0.0f;
     if constexpr (QMODE != kNoEpiQuant) eq_alpha = __ldg(eq.alpha);
@@ -914,29 +949,30 @@ cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, con
 }
 
 // Scale array of an operand (GEMM layout) viewed as rows of 256 bytes:
-// 512-byte atoms -> two rows each; one stage of 4 atoms = 8 rows.
-bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K) {
+// 512-byte atoms -> two rows each; one stage of 4 atoms (NVFP4) = 8 rows, of
+// 2 atoms (MXFP4, one atom per 128 K) = 4 rows.
+bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, bool mx = false) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const int64_t bytes = (rows / 128) * (K / 64) * 512;
+  const int64_t bytes = (rows / 128) * (mx ? K / 128 : K / 64) * 512;
   const cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(bytes / 256)};
   const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {256, 8};
+  const cuuint32_t box[2] = {256, mx ? 4u : 8u};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int QMODE>
+template <int QMODE, bool MX = false>
 cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                         const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
                         int32_t* status, const EpiQuant& eq, cudaStream_t st) {
   const bool fp32 = out_dtype == NVFP4_OUT_DTYPE_FP32;
   CUtensorMap ma, mb, md, msa, msb;
   std::memset(&md, 0, sizeof(md));   // unused when the epilogue writes no D
-  if (!make_map(&ma, A, M, K / 2, 128) || !make_map(&mb, B, N, K / 2, 128) || !make_sf_map(&msa, sA, M, K) ||
-      !make_sf_map(&msb, sB, N, K))
+  if (!make_map(&ma, A, M, K / 2, 128) || !make_map(&mb, B, N, K / 2, 128) || !make_sf_map(&msa, sA, M, K, MX) ||
+      !make_sf_map(&msb, sB, N, K, MX))
     return cudaErrorInvalidValue;
   if (D && !make_out_map(&md, D, M, N, ldd, fp32)) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
@@ -944,7 +980,8 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+        cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QMODE, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairCfg<MX>::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -957,7 +994,7 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(P_THREADS);
-  cfg.dynamicSmemBytes = P_SMEM;
+  cfg.dynamicSmemBytes = PairCfg<MX>::SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -966,7 +1003,7 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE>, ma, mb, md, msa, msb, alphaA, alphaB,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE, MX>, ma, mb, md, msa, msb, alphaA, alphaB,
                                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
                                      static_cast<int>(fp32), status, eq);
   note_launch();
@@ -984,6 +1021,12 @@ cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA
   }
   if (N % 256 == 0) return launch<256>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
   return launch<128>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
+}
+
+cudaError_t mx_gemm_launch(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB, int64_t M,
+                           int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st) {
+  const EpiQuant none{nullptr, nullptr, nullptr, nullptr, 0, 1};
+  return launch_pair<kNoEpiQuant, true>(A, sA, nullptr, B, sB, nullptr, M, N, K, D, out_dtype, ldd, status, none, st);
 }
 
 cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,

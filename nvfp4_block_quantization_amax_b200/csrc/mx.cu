@@ -36,6 +36,7 @@ struct MxArgs {
   uint8_t* codes_col;
   uint8_t* scales_col;
   int32_t* status;
+  int gemm;                       // scales in the tcgen05 block-scale layout
   int64_t tiles_c;
   FastDiv tiles_c_div;
   uint32_t ntiles;
@@ -126,7 +127,8 @@ __global__ void __launch_bounds__(TNT, 3) mx_tile_kernel(const MxArgs a) {
         const uint4 c = mx_encode<ROT>(v, sc);
         const int64_t gr = r0 + row;
         *reinterpret_cast<uint4*>(a.codes_row + gr * (C / 2) + (c0 + 32 * cb) / 2) = c;
-        a.scales_row[gr * (C / 32) + (c0 / 32 + cb)] = static_cast<uint8_t>(sc);
+        const int64_t j = c0 / 32 + cb;
+        a.scales_row[a.gemm ? gemm_scale_offset(gr, j, C / 32) : gr * (C / 32) + j] = static_cast<uint8_t>(sc);
       }
     }
     if constexpr (COL) {
@@ -149,7 +151,8 @@ __global__ void __launch_bounds__(TNT, 3) mx_tile_kernel(const MxArgs a) {
         const uint4 q = mx_encode<ROT>(v, sc);
         const int64_t gc = c0 + c;
         *reinterpret_cast<uint4*>(a.codes_col + gc * (R / 2) + (r0 + 32 * h) / 2) = q;
-        a.scales_col[gc * (R / 32) + (r0 / 32 + h)] = static_cast<uint8_t>(sc);
+        const int64_t j = r0 / 32 + h;
+        a.scales_col[a.gemm ? gemm_scale_offset(gc, j, R / 32) : gc * (R / 32) + j] = static_cast<uint8_t>(sc);
       }
     }
     __syncthreads();   // the buffer is refilled by the next iteration's copies
@@ -234,6 +237,7 @@ cudaError_t mx_quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, 
   a.codes_col = codes_col;
   a.scales_col = scales_col;
   a.status = status;
+  a.gemm = (flags & kGemmScaleLayout) ? 1 : 0;
   const int64_t tiles_r = (R + TR - 1) / TR;
   a.tiles_c = (C + TC - 1) / TC;
   a.tiles_c_div = make_fastdiv(static_cast<uint32_t>(a.tiles_c > 0 ? a.tiles_c : 1));

@@ -254,6 +254,13 @@ __device__ __forceinline__ void rht16x2_presigned(float2* v) {
 // Block encoding (one 16-vector).  Codes come back packed: byte j of `lo`
 // (j < 4) holds elements 2j, 2j+1; `hi` holds elements 8..15.
 // ---------------------------------------------------------------------------
+// Byte offset of the scale of (row m, K-block j (16 elements for NVFP4, 32 for MXFP4)) in the tcgen05 block-scale
+// layout: 512-byte atoms of 128 rows x 4 K-blocks, K-atoms fastest; inside an
+// atom, row m % 32 selects a 16-byte line and (m / 32) % 4 a 4-byte word.
+__device__ __forceinline__ int64_t gemm_scale_offset(int64_t m, int64_t j, int64_t kblocks) {
+  return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
+}
+
 struct Packed16 {
   uint32_t lo, hi;
 };

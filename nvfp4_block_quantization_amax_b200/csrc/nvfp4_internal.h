@@ -65,6 +65,12 @@ cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const floa
                                  int64_t ldd, int mode, bool gemm_layout, const float* alpha_out, uint8_t* codes,
                                  uint8_t* scales, float* amax_out, int32_t* status, cudaStream_t st);
 
+// MXFP4 GEMM (gemm.cu, the CTA-pair kernel with UE8M0 block-32 scales):
+// D = sum_k (qA 2^eA)(qB 2^eB), scales in the GEMM layout with one 512-byte
+// atom per 128 rows x 128 K.  M % 256 == 0, N % 256 == 0, K % 128 == 0.
+cudaError_t mx_gemm_launch(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB, int64_t M,
+                           int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st);
+
 // MXFP4 (mx.cu): one tile kernel for rows and / or columns; dequantization.
 cudaError_t mx_quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
                                uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col, uint8_t* scales_col,

@@ -121,13 +121,6 @@ __device__ __forceinline__ uint32_t sign_bits(const PhiloxKeys& K) {
   return philox(K, 0u, 0u, 0u, kTagSigns).x & 0xFFFFu;
 }
 
-// Byte offset of the scale of (row m, K-block j) in the tcgen05 block-scale
-// layout: 512-byte atoms of 128 rows x 4 K-blocks, K-atoms fastest; inside an
-// atom, row m % 32 selects a 16-byte line and (m / 32) % 4 a 4-byte word.
-__device__ __forceinline__ int64_t gemm_scale_offset(int64_t m, int64_t j, int64_t kblocks) {
-  return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
-}
-
 // ===========================================================================
 // amax kernels.  Each CTA leaves one partial maximum (float bits, or
 // kNonFinite) per orientation; the quantize kernels reduce them.

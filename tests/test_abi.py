@@ -113,6 +113,13 @@ def test_mxfp4_host_checks_need_no_gpu(lib):
     assert q(fake, 32, 32, 36, ROW) == L.NVFP4_ERR_ALIGN                  # ld % 8
     assert q(fake, 32, 32, 32, ROW, cr=fake + 8) == L.NVFP4_ERR_ALIGN
     assert q(None, 0, 32, 32, ROW) == L.NVFP4_OK                          # empty: no-op
+    assert q(fake, 64, 128, 128, ROW | L.NVFP4_GEMM_SCALE_LAYOUT) == L.NVFP4_ERR_SHAPE   # layout: R % 128
+    g = L.mxfp4_gemm
+    assert g(fake, fake, fake, fake, 128, 256, 128, fake, 0, 256, None, 0, None) == L.NVFP4_ERR_SHAPE   # M % 256
+    assert g(fake, fake, fake, fake, 256, 256, 64, fake, 0, 256, None, 0, None) == L.NVFP4_ERR_SHAPE    # K % 128
+    assert g(fake, fake, fake, fake, 256, 256, 128, fake, 7, 256, None, 0, None) == L.NVFP4_ERR_ARG
+    assert g(None, fake, fake, fake, 256, 256, 128, fake, 0, 256, None, 0, None) == L.NVFP4_ERR_ARG
+    assert g(fake + 8, fake, fake, fake, 256, 256, 128, fake, 0, 256, None, 0, None) == L.NVFP4_ERR_ALIGN
     d = L.mxfp4_dequantize
     assert d(fake, fake, 16, 48, 0, 0, fake, None) == L.NVFP4_ERR_SHAPE
     assert d(fake, fake, 16, 32, L.NVFP4_BLOCK2D, 0, fake, None) == L.NVFP4_ERR_ARG

@@ -115,3 +115,80 @@ def test_full_size_activation_dual_rotated(api):
     assert np.array_equal(q.scales_row[:1024].cpu().numpy(), o["scales_row"])
     assert np.array_equal(q.codes_col[:, :512].cpu().numpy(), o["codes_col"])
     assert np.array_equal(q.scales_col[:, :32].cpu().numpy(), o["scales_col"])
+
+
+# ------------------------------------------------------------------ GEMM
+GEMM_LAYOUT, FP32 = 0x20, 1
+
+
+def plain_to_gemm(plain):
+    """[rows, kb] row-major scales -> the tcgen05 block-scale layout (flat)."""
+    rows, kb = plain.shape
+    m = np.arange(rows)[:, None]
+    j = np.arange(kb)[None, :]
+    off = ((m >> 7) * (kb >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3)
+    out = np.zeros(rows * kb, np.uint8)
+    out[off.ravel()] = plain.ravel()
+    return out
+
+
+def frob(D, ref):
+    return float(np.linalg.norm(D.astype(np.float64) - ref) / np.linalg.norm(ref))
+
+
+def bf16_within_one_ulp(Dbf, ref):
+    r = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).float().numpy().astype(np.float64)
+    d = Dbf.float().numpy().astype(np.float64)
+    mag = np.maximum(np.abs(r), np.finfo(np.float32).tiny)
+    ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
+    return bool(np.all(np.abs(d - r) <= ulp * 1.0000001))
+
+
+def test_quantizer_writes_the_gemm_scale_layout(api):
+    x = synthetic.normal_with_channel_outliers(256, 512, seed=21)
+    g = api.mxfp4_quantize(x.cuda(), ROW | COL | GEMM_LAYOUT, seed=4)
+    p = api.mxfp4_quantize(x.cuda(), ROW | COL, seed=4)
+    torch.cuda.synchronize()
+    assert torch.equal(g.codes_row, p.codes_row) and torch.equal(g.codes_col, p.codes_col)
+    assert np.array_equal(g.scales_row.cpu().numpy(), plain_to_gemm(p.scales_row.cpu().numpy()))
+    assert np.array_equal(g.scales_col.cpu().numpy(), plain_to_gemm(p.scales_col.cpu().numpy()))
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 128), (512, 768, 384), (1024, 512, 2048)])
+def test_mx_gemm_random_operands(api, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    A = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    B = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sA = rng.integers(118, 136, (M, K // 32), dtype=np.uint8)
+    sB = rng.integers(118, 136, (N, K // 32), dtype=np.uint8)
+    ref = oracle.mx_gemm_f64(A, sA, B, sB, M, N, K)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    args = (dev(A), dev(plain_to_gemm(sA)), dev(B), dev(plain_to_gemm(sB)))
+    D32 = api.mxfp4_gemm(*args, out_dtype=FP32)
+    Dbf = api.mxfp4_gemm(*args)
+    torch.cuda.synchronize()
+    e = frob(D32.cpu().numpy(), ref)
+    print(f"MX GEMM {M}x{N}x{K}: frob {e:.2e}")
+    assert e <= 1e-5
+    assert bf16_within_one_ulp(Dbf.cpu(), ref)
+
+
+def test_mx_gemm_of_quantized_operands(api):
+    """X-like and W-like bf16 operands through mxfp4_quantize (GEMM layout)
+    and the GEMM, against the FP64 product of the oracle's own quantization."""
+    M, N, K = 512, 512, 1024
+    x = synthetic.normal_with_channel_outliers(M, K, seed=31)
+    w = synthetic.weight(N, K, seed=32)
+    qx = api.mxfp4_quantize(x.cuda(), ROW | GEMM_LAYOUT | RHT, seed=5)
+    qw = api.mxfp4_quantize(w.cuda(), ROW | GEMM_LAYOUT | RHT, seed=5)
+    D = api.mxfp4_gemm(qx.codes_row, qx.scales_row, qw.codes_row, qw.scales_row, out_dtype=FP32)
+    torch.cuda.synchronize()
+    ox = oracle.mx_quantize(synthetic.bf16_bits(x), ROW | RHT, seed=5)
+    ow = oracle.mx_quantize(synthetic.bf16_bits(w), ROW | RHT, seed=5)
+    ref = oracle.mx_gemm_f64(ox["codes_row"], ox["scales_row"], ow["codes_row"], ow["scales_row"], M, N, K)
+    assert frob(D.cpu().numpy(), ref) <= 1e-5
+    # the shared rotation cancels in the product: close to the bf16 product
+    xf = x.float().numpy().astype(np.float64)
+    wf = w.float().numpy().astype(np.float64)
+    print("MX GEMM vs unquantized product: frob", frob(D.cpu().numpy(), xf @ wf.T))
+    assert frob(D.cpu().numpy(), xf @ wf.T) < 0.2
