@@ -10,6 +10,7 @@ Arrays: bf16 tensors are passed as ``numpy.uint16`` bit patterns, row-major
 with a row stride ``ld`` (elements).  Outputs are numpy arrays in the plain
 row-major layouts described in ``nvfp4_oracle.c``.
 """
+import contextlib
 import ctypes
 import os
 
@@ -36,68 +37,83 @@ _i64 = ctypes.c_int64
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        L.oracle_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
-        L.oracle_philox4x32_10.restype = None
-        L.oracle_sign_bits.argtypes = [ctypes.c_uint64]
-        L.oracle_sign_bits.restype = ctypes.c_uint32
-        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
-        L.oracle_e4m3_value.restype = ctypes.c_float
-        for n in ("oracle_e4m3_rne", "oracle_e4m3_ceil", "oracle_e2m1_rne"):
-            getattr(L, n).argtypes = [ctypes.c_float]
-            getattr(L, n).restype = ctypes.c_uint8
-        L.oracle_sr_hw_field.argtypes = [ctypes.c_uint32, ctypes.c_int]
-        L.oracle_sr_hw_field.restype = ctypes.c_uint32
-        for n in ("oracle_e4m3_sr", "oracle_e2m1_sr", "oracle_e2m1_sr_hw"):
-            getattr(L, n).argtypes = [ctypes.c_float, ctypes.c_uint32]
-            getattr(L, n).restype = ctypes.c_uint8
-        L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
-        L.oracle_e2m1_value.restype = ctypes.c_float
-        L.oracle_rht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
-        L.oracle_irht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
-        L.oracle_alpha_from_amax.argtypes = [ctypes.c_float]
-        L.oracle_alpha_from_amax.restype = ctypes.c_float
-        L.oracle_alpha_headroom.argtypes = [ctypes.c_float]
-        L.oracle_alpha_headroom.restype = ctypes.c_float
-        L.oracle_amax.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
-                                  ctypes.c_uint64, _f32p]
-        L.oracle_amax.restype = ctypes.c_int
-        L.oracle_quantize_1d.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_uint32, ctypes.c_uint64, ctypes.c_uint32,
-                                         ctypes.c_float, _i64, _i64, _u8p, _u8p]
-        L.oracle_quantize_1d.restype = ctypes.c_int
-        L.oracle_quantize_2d.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
-                                         _i64, _i64, _u8p, _u8p, _u8p, _u8p]
-        L.oracle_quantize_2d.restype = ctypes.c_int
-        L.oracle_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_uint32,
-                                      ctypes.c_uint64, ctypes.c_uint32, _f32p,
-                                      _u8p, _u8p, _f32p, _u8p, _u8p, _f32p, _f32p, _f32p]
-        L.oracle_quantize.restype = ctypes.c_int
-        L.oracle_dequantize.argtypes = [_u8p, _u8p, ctypes.c_float, _i64, _i64, ctypes.c_uint32,
-                                        ctypes.c_uint64, _f32p]
-        L.oracle_dequantize.restype = ctypes.c_int
-        L.oracle_gemm_f64.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
-                                      _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
-        L.oracle_gemm_f64.restype = None
-        L.oracle_quantize_block16.argtypes = [_f32p, ctypes.c_float, ctypes.c_int, ctypes.c_uint64,
-                                              ctypes.c_uint32, ctypes.c_uint64, _u8p, _u8p]
-        L.oracle_quantize_block16.restype = ctypes.c_int
-        L.oracle_block_sq_error.argtypes = [_f32p, ctypes.c_float, _u8p, ctypes.c_uint8]
-        L.oracle_block_sq_error.restype = ctypes.c_float
-        L.oracle_mx_exponent.argtypes = [ctypes.c_float]
-        L.oracle_mx_exponent.restype = ctypes.c_int
-        L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
-        L.oracle_e8m0_value.restype = ctypes.c_float
-        L.oracle_mx_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64,
-                                         _u8p, _u8p, _u8p, _u8p]
-        L.oracle_mx_quantize.restype = ctypes.c_int
-        L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64, _f32p]
-        L.oracle_mx_dequantize.restype = ctypes.c_int
-        L.oracle_mx_gemm_f64.argtypes = [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
-        L.oracle_mx_gemm_f64.restype = None
-        _lib = L
+        _lib = _configure(ctypes.CDLL(_build.build()))
     return _lib
+
+
+@contextlib.contextmanager
+def use_library(path):
+    """Run the oracle's functions against another build of its source (the
+    mutation tests' planted mistakes) inside the block."""
+    global _lib
+    saved = lib()
+    _lib = _configure(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def _configure(L):
+    L.oracle_philox4x32_10.argtypes = [_u32p, _u32p, _u32p]
+    L.oracle_philox4x32_10.restype = None
+    L.oracle_sign_bits.argtypes = [ctypes.c_uint64]
+    L.oracle_sign_bits.restype = ctypes.c_uint32
+    L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_value.restype = ctypes.c_float
+    for n in ("oracle_e4m3_rne", "oracle_e4m3_ceil", "oracle_e2m1_rne"):
+        getattr(L, n).argtypes = [ctypes.c_float]
+        getattr(L, n).restype = ctypes.c_uint8
+    L.oracle_sr_hw_field.argtypes = [ctypes.c_uint32, ctypes.c_int]
+    L.oracle_sr_hw_field.restype = ctypes.c_uint32
+    for n in ("oracle_e4m3_sr", "oracle_e2m1_sr", "oracle_e2m1_sr_hw"):
+        getattr(L, n).argtypes = [ctypes.c_float, ctypes.c_uint32]
+        getattr(L, n).restype = ctypes.c_uint8
+    L.oracle_e2m1_value.argtypes = [ctypes.c_uint8]
+    L.oracle_e2m1_value.restype = ctypes.c_float
+    L.oracle_rht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
+    L.oracle_irht16.argtypes = [_f32p, ctypes.c_uint32, _f32p]
+    L.oracle_alpha_from_amax.argtypes = [ctypes.c_float]
+    L.oracle_alpha_from_amax.restype = ctypes.c_float
+    L.oracle_alpha_headroom.argtypes = [ctypes.c_float]
+    L.oracle_alpha_headroom.restype = ctypes.c_float
+    L.oracle_amax.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_uint64, _f32p]
+    L.oracle_amax.restype = ctypes.c_int
+    L.oracle_quantize_1d.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_uint32, ctypes.c_uint64, ctypes.c_uint32,
+                                     ctypes.c_float, _i64, _i64, _u8p, _u8p]
+    L.oracle_quantize_1d.restype = ctypes.c_int
+    L.oracle_quantize_2d.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
+                                     _i64, _i64, _u8p, _u8p, _u8p, _u8p]
+    L.oracle_quantize_2d.restype = ctypes.c_int
+    L.oracle_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_uint32,
+                                  ctypes.c_uint64, ctypes.c_uint32, _f32p,
+                                  _u8p, _u8p, _f32p, _u8p, _u8p, _f32p, _f32p, _f32p]
+    L.oracle_quantize.restype = ctypes.c_int
+    L.oracle_dequantize.argtypes = [_u8p, _u8p, ctypes.c_float, _i64, _i64, ctypes.c_uint32,
+                                    ctypes.c_uint64, _f32p]
+    L.oracle_dequantize.restype = ctypes.c_int
+    L.oracle_gemm_f64.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
+                                  _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
+    L.oracle_gemm_f64.restype = None
+    L.oracle_quantize_block16.argtypes = [_f32p, ctypes.c_float, ctypes.c_int, ctypes.c_uint64,
+                                          ctypes.c_uint32, ctypes.c_uint64, _u8p, _u8p]
+    L.oracle_quantize_block16.restype = ctypes.c_int
+    L.oracle_block_sq_error.argtypes = [_f32p, ctypes.c_float, _u8p, ctypes.c_uint8]
+    L.oracle_block_sq_error.restype = ctypes.c_float
+    L.oracle_mx_exponent.argtypes = [ctypes.c_float]
+    L.oracle_mx_exponent.restype = ctypes.c_int
+    L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+    L.oracle_e8m0_value.restype = ctypes.c_float
+    L.oracle_mx_quantize.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64,
+                                     _u8p, _u8p, _u8p, _u8p]
+    L.oracle_mx_quantize.restype = ctypes.c_int
+    L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_uint32, ctypes.c_uint64, _f32p]
+    L.oracle_mx_dequantize.restype = ctypes.c_int
+    L.oracle_mx_gemm_f64.argtypes = [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
+    L.oracle_mx_gemm_f64.restype = None
+    return L
 
 
 def _p(a, t):

@@ -30,5 +30,16 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+def build_variant(source: str, out_dir: str, name: str = "liboracle_variant.so") -> str:
+    """Compile a modified copy of the oracle source (tests that plant a
+    mistake in the oracle and check that a pin catches it) into out_dir."""
+    src = os.path.join(out_dir, name.replace(".so", ".c"))
+    with open(src, "w") as f:
+        f.write(source)
+    lib = os.path.join(out_dir, name)
+    subprocess.run(["gcc", *CFLAGS, src, "-o", lib, "-lm"], check=True)
+    return lib
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))

@@ -488,6 +488,23 @@ def test_four_six_keeps_the_lower_error_candidate(pr1):
     assert n4 > 0  # the M = 4 candidate does win on some blocks
 
 
+def test_four_six_exact_tie_keeps_six():
+    """A block both candidates represent exactly (errors both 0): with
+    alpha = 1 and maximum 6, M = 6 gives Delta = 1 and M = 4 gives Delta = 1.5,
+    each mapping 6 onto the grid.  The tie keeps M = 6 (the selection rule is
+    strict: M = 4 only when its error is lower)."""
+    v = np.zeros(16, np.float32)
+    v[0], v[5] = 6.0, -3.0          # 6 and 3 on the M = 6 grid (Delta 1); 4 and 2 on M = 4's (Delta 1.5)
+    c6, s6 = oracle.quantize_block16(v, 1.0, oracle.RTN)
+    c46, s46 = oracle.quantize_block16(v, 1.0, oracle.FOUR_SIX)
+    assert oracle.e4m3_value(s6) == 1.0 and oracle.block_sq_error(v, 1.0, c6, s6) == 0.0
+    assert s46 == s6 and np.array_equal(c46, c6)
+    s4 = int(e4m3_lib_rne(1.5))
+    q4 = np.zeros(16, np.uint8)
+    q4[0], q4[5] = 6, 8 | 4          # 4 and -2 under Delta 1.5
+    assert oracle.block_sq_error(v, 1.0, q4, s4) == 0.0   # the M = 4 candidate is exact too
+
+
 def test_2d_blocks_consistent_across_orientations(pr1):
     w = pr1["w"]
     R, C = w.shape
