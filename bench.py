@@ -469,7 +469,7 @@ def cpu_baseline_line(bwd_mode):
 
 
 KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_dy_sr",
-                "quant_dy_sr_hw", "quant_w_rot", "quant_x_rot", "mx_dy")
+                "quant_dy_sr_hw", "quant_w_rot", "quant_x_rot", "mx_dy", "mx_gemm_fprop")
 
 
 def run_kernel_case(name, iters=3):
@@ -486,6 +486,10 @@ def run_kernel_case(name, iters=3):
     torch.cuda.synchronize()
     api = step.api
     qx, qw, qd, qwr, qxr = (step.out[k] for k in ("x", "w", "dy", "w_rot", "x_rot"))
+    mx = {}
+    if name == "mx_gemm_fprop":   # MXFP4 operands of the fprop GEMM (GEMM scale layout)
+        mx["x"] = api.mxfp4_quantize(x, ROW | GEMM)
+        mx["w"] = api.mxfp4_quantize(w, ROW | GEMM)
     calls = {
         "gemm_fprop": lambda: api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row,
                                              qw.scales_row, qw.alpha_row, out=step.y),
@@ -501,6 +505,8 @@ def run_kernel_case(name, iters=3):
         "quant_w_rot": lambda: step.quantize("w_rot", RTN, COL | RHT | GEMM, 7, 1),
         "quant_x_rot": lambda: step.quantize("x_rot", RTN, COL | RHT | GEMM, 7, 2),
         "mx_dy": lambda: api.mxfp4_quantize(dy, ROW | COL | RHT, seed=7),
+        "mx_gemm_fprop": lambda: api.mxfp4_gemm(mx["x"].codes_row, mx["x"].scales_row, mx["w"].codes_row,
+                                                mx["w"].scales_row, out=step.y),
     }
     for _ in range(iters):
         calls[name]()
