@@ -126,3 +126,21 @@ def test_mxfp4_host_checks_need_no_gpu(lib):
     assert d(None, fake, 16, 32, 0, 0, fake, None) == L.NVFP4_ERR_ARG
     assert d(fake + 4, fake, 16, 32, 0, 0, fake, None) == L.NVFP4_ERR_ALIGN
     assert d(None, None, 0, 32, 0, 0, None, None) == L.NVFP4_OK
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(lib, tmp_path):
+    """A C11 program (-Wall -Wextra -pedantic -Werror) includes the header,
+    links libnvfp4.so and runs the host-side checks of every entry point."""
+    import shutil
+    import subprocess
+    from nvfp4_block_quantization_amax_b200 import build
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    so = build.build()
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "helpers", "abi_from_c.c"), so, "-Wl,-rpath," + os.path.dirname(so),
+                    "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout
