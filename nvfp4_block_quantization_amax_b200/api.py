@@ -2,6 +2,7 @@
 memory and the current stream are the only things torch supplies) and call
 libnvfp4.so.  Every step of the computation runs in the library's kernels.
 """
+import math
 from dataclasses import dataclass
 from typing import Optional
 
@@ -31,6 +32,47 @@ def _p(t: Optional[torch.Tensor]):
 
 def _stream():
     return torch.cuda.current_stream().cuda_stream
+
+
+def _need(t: Optional[torch.Tensor], numel: int, dtype, what: str, device=None):
+    """Raise unless t can hold `numel` contiguous elements of `dtype` (on
+    `device`): the library writes through raw pointers and cannot check."""
+    if t is None:
+        raise ValueError(f"{what}: buffer missing")
+    if t.dtype != dtype:
+        raise TypeError(f"{what}: dtype {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{what}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{what}: {t.numel()} elements, {numel} needed")
+
+
+def _need_matrix(t: torch.Tensor, rows: int, cols: int, dtype, what: str, device=None):
+    """A row-major matrix view of at least rows x cols (row stride >= cols)."""
+    if t.dtype != dtype:
+        raise TypeError(f"{what}: dtype {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{what}: on {t.device}, expected {device}")
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] < cols or t.stride(1) != 1:
+        raise ValueError(f"{what}: shape {tuple(t.shape)} / strides {t.stride()}, need a row-major "
+                         f"[>= {rows}, >= {cols}] matrix")
+
+
+def check_outputs(q: "QTensor", R: int, C: int, flags: int, device=None):
+    """Raise unless q's buffers can take the outputs of nvfp4_quantize on an
+    [R, C] tensor with these flags."""
+    if flags & NVFP4_ROWWISE:
+        _need(q.codes_row, R * (C // 2), torch.uint8, "codes_row", device)
+        _need(q.scales_row, math.prod(scale_shape(R, C, flags)), torch.uint8, "scales_row", device)
+        _need(q.alpha_row, 1, torch.float32, "alpha_row", device)
+    if flags & NVFP4_COLWISE:
+        _need(q.codes_col, C * (R // 2), torch.uint8, "codes_col", device)
+        _need(q.scales_col, math.prod(scale_shape(C, R, flags)), torch.uint8, "scales_col", device)
+        _need(q.alpha_col, 1, torch.float32, "alpha_col", device)
+    if q.amax is not None:
+        _need(q.amax, 2, torch.float32, "amax", device)
 
 
 @dataclass
@@ -89,6 +131,10 @@ def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream
     ld = x.stride(0) if x.numel() else C
     if alpha is not None:
         flags |= NVFP4_ALPHA_PROVIDED
+    if out is not None:
+        check_outputs(out, R, C, flags, x.device)
+    if status is not None:
+        _need(status, 1, torch.int32, "status", x.device)
     q = out if out is not None else alloc_outputs(R, C, flags, x.device)
     ws = workspace if workspace is not None else workspace_for(R, C, flags, x.device)
     qt = L.nvfp4_qtensor_t(_p(q.codes_row), _p(q.scales_row), _p(q.alpha_row), _p(q.codes_col),
@@ -103,6 +149,8 @@ def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, alpha: torch.Ten
                      flags: int = 0, seed: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Decode [R, C/2] codes to fp32 (or bf16 with NVFP4_OUT_BF16)."""
     dtype = torch.bfloat16 if flags & NVFP4_OUT_BF16 else torch.float32
+    if out is not None:
+        _need(out, R * C, dtype, "out", codes.device)
     y = out if out is not None else torch.empty((R, C), dtype=dtype, device=codes.device)
     st = L.nvfp4_dequantize(_p(codes), _p(scales), _p(alpha), R, C, flags, seed, _p(y), _stream())
     _check(st, "nvfp4_dequantize")
@@ -118,6 +166,8 @@ def nvfp4_gemm(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch
     N = B.shape[0]
     K = 2 * K2
     dt = torch.bfloat16 if out_dtype == NVFP4_OUT_DTYPE_BF16 else torch.float32
+    if out is not None:
+        _need_matrix(out, M, N, dt, "out", A.device)
     D = out if out is not None else torch.empty((M, N), dtype=dt, device=A.device)
     st = L.nvfp4_gemm(_p(A), _p(sA), _p(alphaA), _p(B), _p(sB), _p(alphaB), M, N, K, _p(D), out_dtype,
                       D.stride(0), None, 0, _stream())
@@ -138,6 +188,8 @@ def nvfp4_gemm_quantize(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor,
     dev = A.device
     D = None
     if write_d:
+        if out is not None:
+            _need_matrix(out, M, N, torch.bfloat16, "out", dev)
         D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     codes = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((M, N // 16), dtype=torch.uint8, device=dev)
@@ -159,6 +211,31 @@ class MXTensor:
     scales_col: Optional[torch.Tensor] = None
 
 
+def mx_alloc_outputs(R: int, C: int, flags: int, device) -> MXTensor:
+    """Output buffers of mxfp4_quantize on an [R, C] tensor: codes [rows,
+    len/2] and UE8M0 scales [rows, len/32] (flat in the GEMM layout)."""
+    q = MXTensor()
+    u8 = dict(dtype=torch.uint8, device=device)
+    gemm = bool(flags & NVFP4_GEMM_SCALE_LAYOUT)
+    if flags & NVFP4_ROWWISE:
+        q.codes_row = torch.empty((R, C // 2), **u8)
+        q.scales_row = torch.empty((R * (C // 32),) if gemm else (R, C // 32), **u8)
+    if flags & NVFP4_COLWISE:
+        q.codes_col = torch.empty((C, R // 2), **u8)
+        q.scales_col = torch.empty((C * (R // 32),) if gemm else (C, R // 32), **u8)
+    return q
+
+
+def mx_check_outputs(q: MXTensor, R: int, C: int, flags: int, device=None):
+    """Raise unless q's buffers can take the outputs of mxfp4_quantize."""
+    if flags & NVFP4_ROWWISE:
+        _need(q.codes_row, R * (C // 2), torch.uint8, "codes_row", device)
+        _need(q.scales_row, R * (C // 32), torch.uint8, "scales_row", device)
+    if flags & NVFP4_COLWISE:
+        _need(q.codes_col, C * (R // 2), torch.uint8, "codes_col", device)
+        _need(q.scales_col, C * (R // 32), torch.uint8, "scales_col", device)
+
+
 def mxfp4_quantize(x: torch.Tensor, flags: int, seed: int = 0, status: Optional[torch.Tensor] = None,
                    out: Optional[MXTensor] = None) -> MXTensor:
     """Quantize a 2D bf16 CUDA tensor (unit column stride) to MXFP4 with the C
@@ -169,17 +246,11 @@ def mxfp4_quantize(x: torch.Tensor, flags: int, seed: int = 0, status: Optional[
         raise ValueError("x must have unit column stride")
     R, C = x.shape
     ld = x.stride(0) if x.numel() else C
-    q = out
-    if q is None:
-        q = MXTensor()
-        u8 = dict(dtype=torch.uint8, device=x.device)
-        gemm = bool(flags & NVFP4_GEMM_SCALE_LAYOUT)
-        if flags & NVFP4_ROWWISE:
-            q.codes_row = torch.empty((R, C // 2), **u8)
-            q.scales_row = torch.empty((R * (C // 32),) if gemm else (R, C // 32), **u8)
-        if flags & NVFP4_COLWISE:
-            q.codes_col = torch.empty((C, R // 2), **u8)
-            q.scales_col = torch.empty((C * (R // 32),) if gemm else (C, R // 32), **u8)
+    if out is not None:
+        mx_check_outputs(out, R, C, flags, x.device)
+    if status is not None:
+        _need(status, 1, torch.int32, "status", x.device)
+    q = out if out is not None else mx_alloc_outputs(R, C, flags, x.device)
     st = L.mxfp4_quantize(_p(x), R, C, ld, flags, seed, _p(q.codes_row), _p(q.scales_row), _p(q.codes_col),
                           _p(q.scales_col), _p(status), _stream())
     _check(st, "mxfp4_quantize")
@@ -191,6 +262,8 @@ def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, R: int, C: int, 
     """Decode MXFP4 codes [R, C/2] and scales [R, C/32] to fp32 (or bf16 with
     NVFP4_OUT_BF16)."""
     dtype = torch.bfloat16 if flags & NVFP4_OUT_BF16 else torch.float32
+    if out is not None:
+        _need(out, R * C, dtype, "out", codes.device)
     y = out if out is not None else torch.empty((R, C), dtype=dtype, device=codes.device)
     st = L.mxfp4_dequantize(_p(codes), _p(scales), R, C, flags, seed, _p(y), _stream())
     _check(st, "mxfp4_dequantize")
@@ -205,6 +278,8 @@ def mxfp4_gemm(A: torch.Tensor, sA: torch.Tensor, B: torch.Tensor, sB: torch.Ten
     N = B.shape[0]
     K = 2 * K2
     dt = torch.bfloat16 if out_dtype == NVFP4_OUT_DTYPE_BF16 else torch.float32
+    if out is not None:
+        _need_matrix(out, M, N, dt, "out", A.device)
     D = out if out is not None else torch.empty((M, N), dtype=dt, device=A.device)
     st = L.mxfp4_gemm(_p(A), _p(sA), _p(B), _p(sB), M, N, K, _p(D), out_dtype, D.stride(0), None, 0, _stream())
     _check(st, "mxfp4_gemm")
