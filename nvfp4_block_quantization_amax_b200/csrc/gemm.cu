@@ -1,6 +1,10 @@
-// gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a tensor cores.
+// gemm.cu -- block-scaled NVFP4 (and MXFP4) GEMM on the sm_100a tensor cores.
 //
 //   D[m, n] = alphaA * alphaB * sum_k (qA[m,k] DeltaA[m,k/16]) (qB[n,k] DeltaB[n,k/16])
+//
+// MXFP4 operands (UE8M0 scales per 32 K, no tensor scales) run through the
+// CTA-pair kernel with MX = true: the same pipeline, .block32 MMAs, one scale
+// atom per two MMAs.
 //
 // The NVFP4 pretraining write-up (§四) describes the Blackwell tensor cores
 // that read narrow values plus 8-bit block scales and accumulate in FP32; this
