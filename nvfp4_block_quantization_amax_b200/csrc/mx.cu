@@ -200,14 +200,8 @@ __global__ void __launch_bounds__(256) mx_dequant_kernel(const uint8_t* __restri
 
 template <bool ROT, bool ROW, bool COL>
 static cudaError_t launch_mx_tile(const MxArgs& a, cudaStream_t st) {
-  const int smem = 2 * TR * TC * 2;
+  const int smem = 2 * TR * TC * 2;   // 32 KB: within the default dynamic shared-memory limit
   auto fn = mx_tile_kernel<ROT, ROW, COL>;
-  static bool configured = false;   // the attribute is per function; setting it twice is harmless
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, TNT, smem) != cudaSuccess || n <= 0) n = 1;
   const int grid = static_cast<int>(std::min<int64_t>(a.ntiles, static_cast<int64_t>(sm_count()) * n));
