@@ -45,6 +45,7 @@ def workload(bwd_mode="eden"):
     return ("linear fwd+bwd, 8B-shaped: X 8192x4096 (4/6 1D), W 14336x4096 (4/6 2D), "
             f"dY 8192x14336 ({BWD_NAMES[bwd_mode]} rows+cols), fprop/dgrad/wgrad NVFP4 GEMMs, bf16 out")
 FP4_PER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+FP4_DATASHEET_TFLOPS = 9000.0   # B200 dense FP4, datasheet
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 ROW, COL, B2D, RHT, GEMM = 0x1, 0x2, 0x4, 0x40, 0x20
@@ -213,30 +214,48 @@ class LayerStep:
                                 workspace=self.ws[name])
 
     def run(self, step, timers=None):
-        """One step.  timers: dict name -> list of (start, end) CUDA events."""
+        """One step.  timers: dict call name -> list of (start, end) CUDA
+        events (quantize calls are named q_*, GEMMs fprop / dgrad / wgrad)."""
         api = self.api
         seed = 1000 * (step + 1)   # a new rotation and noise per step
         mark = (lambda k: _Mark(timers, k)) if timers is not None else (lambda k: _NoMark())
-        with mark("quantize"):
+        with mark("q_x"):
             self.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0)
+        with mark("q_w"):
             self.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1)
         qx, qw = self.out["x"], self.out["w"]
-        with mark("gemm"):
+        with mark("fprop"):
             api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row, qw.scales_row, qw.alpha_row,
                            out=self.y)
-        with mark("quantize"):
+        with mark("q_dy"):
             self.quantize("dy", self.bwd, ROW | COL | GEMM, seed, 0)
+        with mark("q_w_rot"):
             self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1)
         qd, qwr = self.out["dy"], self.out["w_rot"]
-        with mark("gemm"):
+        with mark("dgrad"):
             api.nvfp4_gemm(qd.codes_row, qd.scales_row, qd.alpha_row, qwr.codes_col, qwr.scales_col,
                            qwr.alpha_col, out=self.dx)
-        with mark("quantize"):
+        with mark("q_x_rot"):
             self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2)
         qxr = self.out["x_rot"]
-        with mark("gemm"):
+        with mark("wgrad"):
             api.nvfp4_gemm(qd.codes_col, qd.scales_col, qd.alpha_col, qxr.codes_col, qxr.scales_col,
                            qxr.alpha_col, out=self.dw)
+
+    def shapes(self):
+        """(name, elements, algorithmic bytes per element) of the quantize
+        calls and (name, M, N, K) of the GEMMs."""
+        T, H = self.x.shape
+        O = self.w.shape[0]
+        one = 2 + 0.5 + 1 / 16
+        quant = [("q_x", T * H, one), ("q_w", O * H, one), ("q_dy", T * O, 2 + 2 * (0.5 + 1 / 16)),
+                 ("q_w_rot", O * H, one), ("q_x_rot", T * H, one)]
+        gemms = [("fprop", T, O, H), ("dgrad", T, H, O), ("wgrad", O, H, T)]
+        return quant, gemms
+
+
+GEMM_CALLS = ("fprop", "dgrad", "wgrad")
+QUANT_CALLS = ("q_x", "q_w", "q_dy", "q_w_rot", "q_x_rot")
 
 
 class _NoMark:
@@ -278,6 +297,142 @@ def gemm_traffic_record():
     return g.get("dram_bytes_per_launch") if g.get("source_sha256_16") == h else None
 
 
+class L2Flush:
+    """Overwrites a 256 MiB buffer (twice L2) between timed calls so no
+    timed call starts with its inputs in L2."""
+
+    def __init__(self, device):
+        import torch
+        self.buf = torch.empty(64 << 20, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_call(fn, iters, flush=None, warm=1):
+    """Median device time (ms) of fn() over `iters` calls, CUDA events on the
+    current stream, L2 overwritten before every call when flush is given."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        ts.append((s, e))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ts)
+
+
+MODE_NAMES = {RTN: "rtn", FOUR_SIX: "four_six", RHT_SR: "rht_sr", MS_EDEN: "ms_eden", RHT_SR_HW: "rht_sr_hw"}
+SP, PROVIDED = 0x8, 0x10
+
+
+def quant_bytes_per_elem(flags):
+    """Algorithmic bytes per element of one quantize call: the bf16 read once,
+    codes and scales of every requested orientation."""
+    n_or = bool(flags & ROW) + bool(flags & COL)
+    if flags & B2D:
+        return 2 + 0.5 * n_or + n_or / 256
+    return 2 + n_or * (0.5 + 1 / 16)
+
+
+def quantize_modes_table(api, tensors, hbm, flush, iters=7):
+    """Every mode x orientation on the given tensors: the whole call (two
+    passes), the single-pass call, and the quantize kernel alone (alpha
+    provided); microseconds and the fraction of HBM bandwidth by algorithmic
+    bytes."""
+    import torch
+    table = {}
+    for label, t, modes, extra in tensors:
+        R, C = t.shape
+        out = api.alloc_outputs(R, C, ROW | COL | extra, t.device)
+        ws = api.workspace_for(R, C, ROW | COL | SP, t.device)
+        alpha = torch.full((1,), 1e-3, dtype=torch.float32, device=t.device)
+        entry = {}
+        for mode in modes:
+            per = {}
+            for oname, of in (("rows", ROW), ("cols", COL), ("dual", ROW | COL)):
+                flags = of | extra
+                us, frac = [], []
+                for variant in ("two_pass", "single_pass", "kernel_alone"):
+                    if variant == "two_pass":
+                        fn = lambda: api.nvfp4_quantize(t, mode, flags, seed=5, out=out, workspace=ws)
+                    elif variant == "single_pass":
+                        fn = lambda: api.nvfp4_quantize(t, mode, flags | SP, seed=5, out=out, workspace=ws)
+                    else:
+                        fn = lambda: api.nvfp4_quantize(t, mode, flags, seed=5, alpha=alpha, out=out, workspace=ws)
+                    ms = time_call(fn, iters, flush)
+                    us.append(round(ms * 1e3, 2))
+                    frac.append(round(R * C * quant_bytes_per_elem(flags) / (ms * 1e-3) / 1e9 / hbm, 4))
+                per[oname] = {"us": us, "frac_hbm": frac}
+            entry[MODE_NAMES[mode]] = per
+        table[label] = entry
+        del out, ws
+    return table
+
+
+def sweep_table(api, hbm, flush, device):
+    """BASELINE config 4: bf16 4096 x N, every mode, rows and rows + columns,
+    two-pass vs single-pass amax; Gelem/s and fraction of HBM bandwidth."""
+    import torch
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    res = {}
+    for n in synthetic.SWEEP_N:
+        x = synthetic.device_sweep(n, seed=n, device=device)
+        out = api.alloc_outputs(4096, n, ROW | COL, device)
+        ws = api.workspace_for(4096, n, ROW | COL | SP, device)
+        iters = 10 if n <= 16384 else 3
+        per = {}
+        for mode in MODE_NAMES:
+            row = {}
+            for oname, of in (("rows", ROW), ("dual", ROW | COL)):
+                g, f = [], []
+                for sp in (0, SP):
+                    ms = time_call(lambda: api.nvfp4_quantize(x, mode, of | sp, seed=3, out=out, workspace=ws),
+                                   iters, flush)
+                    g.append(round(4096 * n / (ms * 1e-3) / 1e9, 1))
+                    f.append(round(4096 * n * quant_bytes_per_elem(of) / (ms * 1e-3) / 1e9 / hbm, 4))
+                row[oname] = {"gelem_s": g, "frac_hbm": f}
+            per[MODE_NAMES[mode]] = row
+        res[f"4096x{n}"] = per
+        del x, out, ws
+        torch.cuda.empty_cache()
+    return res
+
+
+def step_breakdown(step, steps, hbm, fp4_peak):
+    """Run `steps` steps with every call timed; per call: average us and its
+    roofline fraction (quantize: algorithmic bytes vs HBM; GEMM: 2MNK vs the
+    FP4 peak)."""
+    import torch
+    timers = {}
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        step.run(100 + i, timers)
+    e.record()
+    torch.cuda.synchronize()
+    ms_step = s.elapsed_time(e) / steps
+    quant, gemms = step.shapes()
+    calls = []
+    for name, n, bpe in quant:
+        us = 1e3 * sum(a.elapsed_time(b) for a, b in timers[name]) / steps
+        calls.append({"call": name, "us": round(us, 2), "bound": "hbm",
+                      "frac": round(n * bpe / (us * 1e-6) / 1e9 / hbm, 4)})
+    flops = 0.0
+    for name, M, N, K in gemms:
+        us = 1e3 * sum(a.elapsed_time(b) for a, b in timers[name]) / steps
+        flops += 2.0 * M * N * K
+        calls.append({"call": name, "us": round(us, 2), "bound": "tensor",
+                      "frac": round(2.0 * M * N * K / (us * 1e-6) / 1e12 / fp4_peak, 4)})
+    return {"ms_per_step": ms_step, "gemm_tflops_per_step_time": flops / (ms_step * 1e-3) / 1e12, "calls": calls}
+
+
 def run_device(args, rank, world, local_rank):
     import torch
     from nvfp4_block_quantization_amax_b200 import _lib, synthetic
@@ -311,8 +466,8 @@ def run_device(args, rank, world, local_rank):
     ms_local = start.elapsed_time(end) / args.steps
     clocks = clk.summary()
     ms = max_over_ranks(ms_local, device)
-    gemm_ms = sum(s.elapsed_time(e) for s, e in timers["gemm"]) / (3 * args.steps)
-    quant_ms = sum(s.elapsed_time(e) for s, e in timers["quantize"]) / args.steps
+    gemm_ms = sum(s.elapsed_time(e) for k in GEMM_CALLS for s, e in timers[k]) / (3 * args.steps)
+    quant_ms = sum(s.elapsed_time(e) for k in QUANT_CALLS for s, e in timers[k]) / args.steps
 
     # --- end to end: pinned host inputs in, results back to pinned host ---
     hx, hw, hdy = (t.cpu().pin_memory() for t in (x, w, dy))
@@ -345,7 +500,10 @@ def run_device(args, rank, world, local_rank):
 
     total_flops = sum_over_ranks(gemm_flops(), device)
     peaks, src = load_peaks()
-    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    hbm = peaks["hbm_gbs"]
+    # the GEMM is timed inside a step of a few milliseconds repeated for well
+    # under the seconds a sustained figure needs: the burst peak applies
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
     gemm_tflops = 2.0 * TOKENS * OUT * HIDDEN / (gemm_ms * 1e-3) / 1e12
     q_elems = sum(n for _, n, _ in quant_calls())
     q_bytes = sum(n * b for _, n, b in quant_calls())
@@ -354,6 +512,8 @@ def run_device(args, rank, world, local_rank):
     traffic = gemm_traffic_record()
     h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
     d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
+    per_call = {k: round(1e3 * sum(s.elapsed_time(e) for s, e in timers[k]) / args.steps, 2)
+                for k in QUANT_CALLS + GEMM_CALLS}
     result = {
         "metric": METRIC,
         "value": total_flops / (ms * 1e-3) / 1e12,
@@ -369,21 +529,80 @@ def run_device(args, rank, world, local_rank):
         "data": "synthetic (seeded; shapes and distributions of the pages' 8B workload)",
         "config": {"workload": workload(args.bwd_mode), "tokens": TOKENS, "hidden": HIDDEN, "out_features": OUT,
                    "bwd_mode": args.bwd_mode, "parallelism": f"replicas x{world} (weak)",
-                   "l2": "inputs larger than L2: 419 MB of bf16 per step"},
+                   "l2": "inputs larger than L2: 419 MB of bf16 per step; sub-benchmarks overwrite a 256 MiB "
+                         "buffer before every timed call"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp4_peak, "traffic": traffic,
-                     "kernel": "nvfp4_gemm_kernel (avg of fprop, dgrad, wgrad)",
-                     "peak_source": f"{src} bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)"},
-        "quantize": {"gelem_s": q_gelem, "alg_gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
-                     "ms_per_step": quant_ms, "hbm_peak_gbs": peaks["hbm_gbs"],
+                     "kernel": "nvfp4_gemm_pair_kernel (avg of fprop, dgrad, wgrad)",
+                     "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/BF16 ratio)",
+                     "peak_datasheet": FP4_DATASHEET_TFLOPS,
+                     "frac_datasheet": gemm_tflops / FP4_DATASHEET_TFLOPS},
+        "quantize": {"gelem_s": q_gelem, "alg_gbs": q_gbs, "frac_hbm": q_gbs / hbm,
+                     "ms_per_step": quant_ms, "hbm_peak_gbs": hbm,
                      "note": "algorithmic bytes: bf16 read once + codes + scales per orientation"},
-        "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak, "ms_per_gemm": gemm_ms},
+        "gemm": {"tflops": gemm_tflops, "frac_fp4_peak": gemm_tflops / fp4_peak,
+                 "frac_datasheet": gemm_tflops / FP4_DATASHEET_TFLOPS, "ms_per_gemm": gemm_ms},
+        "per_call_us": per_call,
         "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    del hx, hw, hdy, hy, hdx, hdw
+    if not args.no_extras:
+        result.update(run_extras(args, step, x, w, dy, device, hbm, fp4_peak))
     return result
+
+
+def run_extras(args, step, x, w, dy, device, hbm, fp4_peak):
+    """The sub-benchmarks of the JSON line: every quantize mode on the 8B
+    tensors, the 4096 x N sweep, the 12B-shaped step, the GEMMs timed alone
+    (NVFP4 and MXFP4)."""
+    import torch
+    from nvfp4_block_quantization_amax_b200 import synthetic
+    api = step.api
+    flush = L2Flush(device)
+    extras = {}
+    all_modes = list(MODE_NAMES)
+    extras["quantize_modes"] = {
+        "columns": ["two_pass (amax + quantize)", "single_pass", "kernel_alone (alpha provided)"],
+        "timing": "CUDA events, L2 overwritten before each call, median of 7",
+        "bytes": "algorithmic: bf16 read once + codes + scales per orientation",
+        **quantize_modes_table(api, [("X 8192x4096", x, all_modes, 0), ("dY 8192x14336", dy, all_modes, 0),
+                                     ("W 14336x4096 2D", w, [RTN, FOUR_SIX], B2D)], hbm, flush)}
+    # GEMMs alone (burst): the step's NVFP4 operands, and MXFP4 ones of the fprop shape
+    qx, qw = step.out["x"], step.out["w"]
+    ms = time_call(lambda: api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row, qw.scales_row,
+                                          qw.alpha_row, out=step.y), 20, flush)
+    fl = 2.0 * TOKENS * OUT * HIDDEN
+    extras["nvfp4_gemm_alone"] = {"shape": "8192x14336x4096", "us": round(ms * 1e3, 2),
+                                  "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / fp4_peak,
+                                  "frac_datasheet": fl / (ms * 1e-3) / 1e12 / FP4_DATASHEET_TFLOPS}
+    mx_x = api.mxfp4_quantize(x, ROW | GEMM)
+    mx_w = api.mxfp4_quantize(w, ROW | GEMM)
+    ms = time_call(lambda: api.mxfp4_gemm(mx_x.codes_row, mx_x.scales_row, mx_w.codes_row, mx_w.scales_row,
+                                          out=step.y), 20, flush)
+    extras["mxfp4_gemm"] = {"shape": "8192x14336x4096", "us": round(ms * 1e3, 2),
+                            "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / fp4_peak,
+                            "frac_datasheet": fl / (ms * 1e-3) / 1e12 / FP4_DATASHEET_TFLOPS}
+    del mx_x, mx_w
+    # the 12B-hybrid-shaped step (BASELINE config 5): tokens 16384, hidden 5120, FFN 20480
+    s = synthetic.STEP_12B
+    lay = synthetic.device_layer(s["tokens"], s["hidden"], s["ffn"], seed=12, device=device)
+    st12 = LayerStep(lay["x"], lay["w"], lay["dy"], BWD_MODES[args.bwd_mode], device)
+    for i in range(3):
+        st12.run(i)
+    torch.cuda.synchronize()
+    extras["step12b"] = {"workload": "12B-hybrid-shaped linear fwd+bwd: X 16384x5120, W 20480x5120, "
+                                     f"dY 16384x20480 ({BWD_NAMES[args.bwd_mode]}), one stream",
+                         **step_breakdown(st12, 20, hbm, fp4_peak)}
+    del st12, lay
+    torch.cuda.empty_cache()
+    extras["sweep"] = {"timing": "CUDA events, L2 overwritten before each call, median of 10 (3 for N >= 65536)",
+                       "columns": ["two_pass", "single_pass"],
+                       "data": "device-drawn N(0,1) with 0.1% channel outliers x50 (torch CUDA generator)",
+                       **sweep_table(api, hbm, flush, device)}
+    return extras
 
 
 # --------------------------------------------------------------------------
@@ -433,9 +652,41 @@ def oracle_sample(budget_rows=64, gemm_rows=16, gemm_cols=16, bwd_mode="eden"):
         dt, _ = timed(lambda: oracle.gemm_f64(A, sA, 1.0, B, sB, 1.0, gemm_rows, gemm_cols, K))
         t_total += dt * (M * N) / (gemm_rows * gemm_cols)
         parts.append(f"GEMM {gemm_rows}x{gemm_cols} of {M}x{N}, K={K}")
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    desc = ("oracle timed on " + "; ".join(parts) + "; each part scaled to the full step by its element count")
+    threads = omp_threads()
+    desc = ("oracle timed on " + "; ".join(parts) + "; each part scaled to the full step by its element count "
+            "(extrapolated)")
     return t_total, desc, threads
+
+
+def _gomp():
+    import ctypes
+    import oracle
+    oracle.lib()   # loads the oracle and with it the OpenMP runtime it links
+    try:
+        return ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return None
+
+
+def omp_threads():
+    g = _gomp()
+    return int(g.omp_get_max_threads()) if g is not None else 1
+
+
+class single_threaded:
+    """Run the oracle's OpenMP regions on one thread inside the block."""
+
+    def __enter__(self):
+        self.g = _gomp()
+        self.n = omp_threads()
+        if self.g is not None:
+            self.g.omp_set_num_threads(1)
+        return self
+
+    def __exit__(self, *a):
+        if self.g is not None:
+            self.g.omp_set_num_threads(self.n)
+        return False
 
 
 def run_reference(args):
@@ -458,14 +709,22 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizer, f64 GEMM (CPU oracle)",
             "data": "synthetic", "config": {"workload": workload(args.bwd_mode), "bwd_mode": args.bwd_mode},
-            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "extrapolated": True,
+            "note": "each step times the oracle on bounded slices of the step and scales every part to the "
+                    "full step by its element count: ms_per_step is an extrapolation, not a measured run",
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+                             "extrapolated": True},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def cpu_baseline_line(bwd_mode):
     dt, desc, threads = oracle_sample(bwd_mode=bwd_mode)
+    with single_threaded():
+        dt1, desc1, _ = oracle_sample(budget_rows=16, bwd_mode=bwd_mode)
     return {"value": gemm_flops() / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": desc, "step_seconds_extrapolated": dt}
+            "sample": desc, "extrapolated": True, "step_seconds_extrapolated": dt,
+            "single_thread": {"value": gemm_flops() / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                              "sample": desc1, "extrapolated": True, "step_seconds_extrapolated": dt1}}
 
 
 KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_x", "quant_w2d", "quant_dy", "quant_dy_sr",
@@ -521,6 +780,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--bwd-mode", choices=sorted(BWD_MODES), default="eden")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sub-benchmarks (per-mode table, sweep, 12B step, GEMMs alone)")
     ap.add_argument("--kernel-case", choices=KERNEL_CASES,
                     help="run one call of the step a few times and exit (for profiler captures)")
     args = ap.parse_args(argv)

@@ -14,7 +14,9 @@
  *
  * Conventions shared by every call
  *   - All device pointers are caller-owned CUDA device memory; the library
- *     never allocates.  Scratch memory comes from the caller's workspace.
+ *     never allocates.  Scratch memory comes from the caller's workspace,
+ *     except for nvfp4_quantize_noalloc, whose scratch is a fixed array
+ *     inside the library (see that call).
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream).  Nothing synchronises the
  *     host; the tensor scale alpha stays on the device.
@@ -91,8 +93,11 @@ typedef enum {
 #define NVFP4_BLOCK2D 0x4u          /* 16x16 blocks (weights, [NV] §二); RTN/4-6 */
 #define NVFP4_SINGLE_PASS 0x8u      /* amax and quantize in one cooperative launch:
                                      * per-CTA maxima, a grid barrier (bounded:
-                                     * 1 s, then NVFP4_ERR_TIMEOUT in *status and
-                                     * no outputs), then the encoding; results
+                                     * 1 s, or the nanoseconds in the environment
+                                     * variable NVFP4_BARRIER_TIMEOUT_NS read at
+                                     * each call; then NVFP4_ERR_TIMEOUT in
+                                     * *status and unspecified outputs), then
+                                     * the encoding; results
                                      * identical to the two-pass call.  Needs 16
                                      * more workspace bytes (the barrier counter,
                                      * cleared by the call).  Pays off for small
@@ -183,15 +188,19 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int
  * run (no page defines this; it has no counterpart in the method): a plugin
  * inside another runtime that owns all device memory, or a program whose
  * memory plan is fixed at start-up.  Same arguments and results as
- * nvfp4_quantize, minus the workspace: the scratch of the amax pass lives in
+ * nvfp4_quantize, minus the workspace: the scratch (the amax pass's per-CTA
+ * partials and, with NVFP4_SINGLE_PASS, the grid barrier's counter) lives in
  * an 8192-byte array compiled into the library, which every GPU that loads
  * the library holds until the process exits.  A call that would need more
- * scratch than that returns NVFP4_ERR_WORKSPACE.  The first call on each
- * device (with that device current) looks up the array's device address;
- * make it before any stream capture starts.  All calls on a device share the
- * array, so calls whose kernels may overlap on the GPU race and can give wrong
- * results: order them on one stream.  Nothing in the array must start at
- * zero.  The function itself allocates nothing. */
+ * scratch than that returns NVFP4_ERR_WORKSPACE.  Arguments are checked
+ * first; the first accepted call on each device (with that device current)
+ * then looks up the array's device address: make it before any stream
+ * capture starts, and do not reset the device (cudaDeviceReset) between
+ * calls, since the address is kept.  All calls on a device share the array,
+ * so calls whose kernels may overlap on the GPU race and can give wrong
+ * results or a barrier timeout: order them on one stream.  The partials need
+ * no clearing; the barrier counter is cleared by each single-pass call with a
+ * stream-ordered memset.  The function itself allocates nothing. */
 NVFP4_API nvfp4_status_t nvfp4_quantize_noalloc(const void* x, int64_t R, int64_t C, int64_t ld,
                                                 nvfp4_mode_t mode, uint32_t flags, uint64_t seed,
                                                 uint32_t stream_id, const float* alpha_in,

@@ -30,6 +30,41 @@ std::atomic<uint64_t> g_launches{0};
 
 namespace nvfp4 {
 void note_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode_t mode,
+                                   uint32_t flags, uint32_t stream_id, const float* alpha_in,
+                                   const nvfp4_qtensor_t* out, bool* empty) {
+  *empty = false;
+  if (!out) return NVFP4_ERR_ARG;
+  if (static_cast<int>(mode) < NVFP4_RTN || static_cast<int>(mode) > NVFP4_RHT_SR_HW) return NVFP4_ERR_ARG;
+  if (flags & ~kQuantFlags) return NVFP4_ERR_ARG;
+  const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE, two_d = flags & NVFP4_BLOCK2D;
+  const bool gemm = flags & NVFP4_GEMM_SCALE_LAYOUT;
+  if (!row && !col) return NVFP4_ERR_ARG;
+  if (two_d && (mode == NVFP4_RHT_SR || mode == NVFP4_MS_EDEN || mode == NVFP4_RHT_SR_HW || (flags & NVFP4_RHT)))
+    return NVFP4_ERR_ARG;
+  if (stream_id >= 0x80000000u) return NVFP4_ERR_ARG;
+  if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
+  if (C % 16) return NVFP4_ERR_SHAPE;
+  if ((col || two_d) && R % 16) return NVFP4_ERR_SHAPE;
+  if (R * (C / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (gemm) {
+    if (row && (R % 128 || C % 64)) return NVFP4_ERR_SHAPE;
+    if (col && (C % 128 || R % 64)) return NVFP4_ERR_SHAPE;
+  }
+  if (R == 0 || C == 0) {  // empty tensor: nothing to write
+    *empty = true;
+    return NVFP4_OK;
+  }
+  if ((flags & NVFP4_ALPHA_PROVIDED) && !alpha_in) return NVFP4_ERR_ARG;
+  if (row && (!out->codes_row || !out->scales_row || !out->alpha_row)) return NVFP4_ERR_ARG;
+  if (col && (!out->codes_col || !out->scales_col || !out->alpha_col)) return NVFP4_ERR_ARG;
+  if (!x) return NVFP4_ERR_ARG;
+  if (!aligned(x, 16) || ld % 8) return NVFP4_ERR_ALIGN;
+  if (row && !aligned(out->codes_row, 16)) return NVFP4_ERR_ALIGN;
+  if (col && !aligned(out->codes_col, 16)) return NVFP4_ERR_ALIGN;
+  return NVFP4_OK;
+}
 }  // namespace nvfp4
 
 extern "C" {
@@ -111,31 +146,10 @@ nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, n
                               uint32_t flags, uint64_t seed, uint32_t stream_id,
                               const float* alpha_in, const nvfp4_qtensor_t* out, void* workspace,
                               size_t workspace_bytes, void* stream) {
-  if (!out) return NVFP4_ERR_ARG;
-  if (static_cast<int>(mode) < NVFP4_RTN || static_cast<int>(mode) > NVFP4_RHT_SR_HW) return NVFP4_ERR_ARG;
-  if (flags & ~kQuantFlags) return NVFP4_ERR_ARG;
-  const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE, two_d = flags & NVFP4_BLOCK2D;
-  const bool gemm = flags & NVFP4_GEMM_SCALE_LAYOUT;
-  if (!row && !col) return NVFP4_ERR_ARG;
-  if (two_d && (mode == NVFP4_RHT_SR || mode == NVFP4_MS_EDEN || mode == NVFP4_RHT_SR_HW || (flags & NVFP4_RHT)))
-    return NVFP4_ERR_ARG;
-  if (stream_id >= 0x80000000u) return NVFP4_ERR_ARG;
-  if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
-  if (C % 16) return NVFP4_ERR_SHAPE;
-  if ((col || two_d) && R % 16) return NVFP4_ERR_SHAPE;
-  if (R * (C / 16) >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
-  if (gemm) {
-    if (row && (R % 128 || C % 64)) return NVFP4_ERR_SHAPE;
-    if (col && (C % 128 || R % 64)) return NVFP4_ERR_SHAPE;
-  }
-  if (R == 0 || C == 0) return NVFP4_OK;  // empty tensor: nothing to write
-  if ((flags & NVFP4_ALPHA_PROVIDED) && !alpha_in) return NVFP4_ERR_ARG;
-  if (row && (!out->codes_row || !out->scales_row || !out->alpha_row)) return NVFP4_ERR_ARG;
-  if (col && (!out->codes_col || !out->scales_col || !out->alpha_col)) return NVFP4_ERR_ARG;
-  if (!x) return NVFP4_ERR_ARG;
-  if (!aligned(x, 16) || ld % 8) return NVFP4_ERR_ALIGN;
-  if (row && !aligned(out->codes_row, 16)) return NVFP4_ERR_ALIGN;
-  if (col && !aligned(out->codes_col, 16)) return NVFP4_ERR_ALIGN;
+  bool empty = false;
+  const nvfp4_status_t chk = nvfp4::check_quantize_args(x, R, C, ld, mode, flags, stream_id, alpha_in, out, &empty);
+  if (chk != NVFP4_OK || empty) return chk;
+  const bool row = flags & NVFP4_ROWWISE, col = flags & NVFP4_COLWISE;
   const size_t need = nvfp4::quant_workspace_bytes(R, C, flags);
   if (need && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return NVFP4_ERR_WORKSPACE;
   nvfp4::QuantOutputs o{out->codes_row, out->scales_row, out->alpha_row, out->codes_col,

@@ -4,21 +4,28 @@
 // quantizes -- a plugin hosted inside another runtime that owns all device
 // memory, or a program that fixes its memory plan at start-up and may not
 // call cudaMalloc afterwards.  Such a caller still owns x and every output
-// buffer; only the scratch of the two-pass path (one partial amax per amax
-// CTA and orientation) comes from a fixed array compiled into this library.
+// buffer; only the scratch comes from a fixed array compiled into this
+// library: the per-CTA amax partials of the amax pass and, with
+// NVFP4_SINGLE_PASS, the grid barrier's arrival counter after them.
 //
 // The array is a file-scope __device__ symbol, so every GPU that loads the
 // library holds it (kNoAllocScratchBytes bytes) until the process exits.
 // Host code cannot use the symbol's name as a device address: the first call
 // on each device, with that device current, looks the address up with
 // cudaGetSymbolAddress and keeps it for later calls.  Make that first call on
-// a device before any stream capture starts.
+// a device before any stream capture starts, and do not reset the device
+// (cudaDeviceReset) between calls: a reset reloads the module, the array may
+// move, and the kept address would then be stale.  Arguments are checked
+// before the lookup, so a call the library rejects never performs it.
 //
 // All calls on a device share the one array and it keeps whatever the last
-// call wrote.  Nothing in it has to start at zero: the amax pass writes every
-// partial that the quantize kernel then reads.  Two calls whose kernels may
-// run at the same time on the GPU (for example on two unordered streams) race
-// on the array and can produce wrong results; order such calls on one stream.
+// call wrote.  The amax partials need no clearing (the amax pass writes every
+// partial that the quantize kernel then reads); the barrier counter must
+// start at zero and each single-pass call clears it with a stream-ordered
+// memset.  Two calls whose kernels may run at the same time on the GPU (for
+// example on two unordered streams) race on the partials and on the counter
+// and can produce wrong results or a barrier that gives up (NVFP4_ERR_TIMEOUT
+// in the status word); order such calls on one stream.
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <mutex>
@@ -57,6 +64,10 @@ extern "C" {
 nvfp4_status_t nvfp4_quantize_noalloc(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode_t mode,
                                       uint32_t flags, uint64_t seed, uint32_t stream_id,
                                       const float* alpha_in, const nvfp4_qtensor_t* out, void* stream) {
+  bool empty = false;
+  const nvfp4_status_t chk =
+      nvfp4::check_quantize_args(x, R, C, ld, mode, flags, stream_id, alpha_in, out, &empty);
+  if (chk != NVFP4_OK || empty) return chk;
   const size_t need = nvfp4_workspace_size(R, C, flags);
   if (need > kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;  // more scratch than the fixed array holds
   void* scratch = nullptr;

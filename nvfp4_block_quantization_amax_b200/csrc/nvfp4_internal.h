@@ -43,6 +43,12 @@ int sm_count();
 void note_launch(int n = 1);  // count kernels launched by the library
 size_t quant_workspace_bytes(int64_t R, int64_t C, uint32_t flags);
 
+// Host-side checks of nvfp4_quantize's arguments, the workspace excepted.
+// NVFP4_OK with *empty set when the tensor has no elements (nothing to do).
+nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t ld, nvfp4_mode_t mode,
+                                   uint32_t flags, uint32_t stream_id, const float* alpha_in,
+                                   const nvfp4_qtensor_t* out, bool* empty);
+
 cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int mode,
                             uint32_t flags, uint64_t seed, uint32_t stream_id,
                             const float* alpha_in, const QuantOutputs& out, void* workspace,

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 
 #include "nvfp4_device.cuh"
 #include "nvfp4_internal.h"
@@ -891,14 +892,19 @@ __device__ __forceinline__ uint32_t load_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-constexpr uint64_t kBarrierTimeoutNs = 1000000000ull;   // 1 s
+// Default limit of the single-pass grid barrier's wait: 1 s.  The
+// environment variable NVFP4_BARRIER_TIMEOUT_NS, read at every single-pass
+// call, replaces it (the tests set it to 0 to make the wait run out).
+constexpr uint64_t kBarrierTimeoutNs = 1000000000ull;
 
 // Grid-wide barrier of a cooperative launch: every CTA's thread 0 releases
-// its writes, counts itself in, and waits (at most kBarrierTimeoutNs) until
-// all `n` CTAs are in.  The counter starts at 0 (the launcher clears it).
-// Returns false, with NVFP4_ERR_TIMEOUT in the status word, if the wait ran
-// out; the caller then returns without touching its outputs.
-__device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, int32_t* status, uint32_t* ok_smem) {
+// its writes, counts itself in, and waits (at most timeout_ns) until all `n`
+// CTAs are in.  The counter starts at 0 (the launcher clears it).  Returns
+// false, with NVFP4_ERR_TIMEOUT in the status word, if the wait ran out; the
+// caller then returns without touching its outputs (its own copies have all
+// landed: every amax body ends with no cp.async group outstanding).
+__device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, uint64_t timeout_ns, int32_t* status,
+                                             uint32_t* ok_smem) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -906,7 +912,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, int3
     const uint64_t t0 = global_ns();
     uint32_t ok = 1;
     while (load_acquire_gpu(counter) < n) {
-      if (global_ns() - t0 > kBarrierTimeoutNs) {
+      if (global_ns() - t0 >= timeout_ns) {
         ok = 0;
         break;
       }
@@ -923,7 +929,8 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, int3
 // quantization, all in one cooperative launch whose CTAs are co-resident.
 // For tensors that fit in L2 the quantize pass re-reads from L2, not HBM.
 template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
-__global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, uint32_t* counter) {
+__global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, uint32_t* counter,
+                                                              uint64_t timeout_ns) {
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
   __shared__ uint32_t pass_ok;
@@ -937,7 +944,7 @@ __global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, 
     } else {
       amax_plain_body<TNT>(a.x, a.R, a.ld, a.chunks_row, pr, cta, ncta, stg.red);
     }
-    if (!grid_barrier(counter, ncta, a.status, &pass_ok)) return;
+    if (!grid_barrier(counter, ncta, timeout_ns, a.status, &pass_ok)) return;
   }
   if constexpr (TWO_D) {
     quant_tile_2d_body<MODE, ROW, COL>(a, cta, ncta, tile_ring, stg);
@@ -1050,7 +1057,13 @@ static cudaError_t launch_single_pass(QuantArgs a, cudaStream_t st) {
   if (a.partials_col != a.partials) a.partials_col = a.partials + amax_partial_count();
   cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
-  void* args[] = {&a, &counter};
+  uint64_t timeout_ns = kBarrierTimeoutNs;
+  if (const char* env = std::getenv("NVFP4_BARRIER_TIMEOUT_NS")) {
+    char* end = nullptr;
+    const unsigned long long v = std::strtoull(env, &end, 10);
+    if (end != env && *end == '\0') timeout_ns = v;
+  }
+  void* args[] = {&a, &counter, &timeout_ns};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fn), dim3(grid), dim3(TNT), args, smem, st);
   note_launch();
   return e;

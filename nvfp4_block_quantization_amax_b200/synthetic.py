@@ -101,3 +101,50 @@ def step_12b(seed=0):
 
 def sweep(n, seed=0):
     return normal_with_channel_outliers(4096, n, seed=seed)
+
+
+# ---------------------------------------------------------------------------
+# Device-side draws with the same distributions, for timing runs whose
+# tensors are too large to draw on the host in reasonable time (torch's
+# counter-based CUDA generator, fixed seeds; bf16 by round-to-nearest-even).
+# ---------------------------------------------------------------------------
+def _gen(seed, device):
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def device_normal_with_channel_outliers(rows, cols, seed, device, frac=0.001, factor=50.0):
+    g = _gen(seed, device)
+    a = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32)
+    n = max(1, int(round(frac * cols)))
+    ch = torch.randperm(cols, generator=g, device=device)[:n]
+    a[:, ch] *= factor
+    return a.to(torch.bfloat16)
+
+
+def device_weight(rows, cols, seed, device, std=0.02):
+    g = _gen(seed, device)
+    return (torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def device_laplace_with_spikes(rows, cols, seed, device, scale=1e-4, frac=1e-4, spike=1e-2):
+    g = _gen(seed, device)
+    u = torch.rand((rows, cols), generator=g, device=device, dtype=torch.float32) - 0.5
+    # inverse CDF of Laplace(0, scale); u = -0.5 (probability 2^-24) is nudged to avoid log(0)
+    a = -scale * torch.sign(u) * torch.log1p(-2.0 * u.abs().clamp(max=0.5 - 2.0 ** -25))
+    n = max(1, int(round(frac * rows * cols)))
+    idx = torch.randint(0, rows * cols, (n,), generator=g, device=device)
+    sign = torch.where(torch.rand((n,), generator=g, device=device) < 0.5, -1.0, 1.0)
+    a.view(-1)[idx] = sign * spike
+    return a.to(torch.bfloat16)
+
+
+def device_layer(tokens, hidden, out_features, seed, device):
+    return dict(x=device_normal_with_channel_outliers(tokens, hidden, seed, device),
+                w=device_weight(out_features, hidden, seed + 1, device),
+                dy=device_laplace_with_spikes(tokens, out_features, seed + 2, device))
+
+
+def device_sweep(n, seed, device):
+    return device_normal_with_channel_outliers(4096, n, seed, device)

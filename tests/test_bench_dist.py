@@ -75,3 +75,13 @@ def test_reference_arm_sample_runs_in_every_backward_mode(mode):
     assert dt > 0 and threads >= 1
     assert "dY rows+cols: 16x14336" in desc
     assert bench.BWD_NAMES[mode] in bench.workload(mode)
+
+
+def test_quantize_bytes_per_element():
+    # bf16 read once + 0.5 B of codes and 1/16 B of scale per element and
+    # orientation (1D); 2D blocks carry one scale per 256 elements
+    assert bench.quant_bytes_per_elem(bench.ROW) == 2.5625
+    assert bench.quant_bytes_per_elem(bench.COL) == 2.5625
+    assert bench.quant_bytes_per_elem(bench.ROW | bench.COL) == 3.125
+    assert bench.quant_bytes_per_elem(bench.ROW | bench.B2D) == 2 + 0.5 + 1 / 256
+    assert bench.quant_bytes_per_elem(bench.ROW | bench.COL | bench.B2D) == 3 + 2 / 256

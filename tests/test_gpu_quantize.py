@@ -378,6 +378,29 @@ def test_single_pass_nonfinite_sets_status(api):
         assert int(status.item()) == -4, (mode, flags)
 
 
+@pytest.mark.parametrize("mode,flags", [(3, ROW | COL), (1, ROW), (1, ROW | B2D), (0, COL | RHT)])
+def test_single_pass_barrier_timeout_sets_status(api, pr1, monkeypatch, mode, flags):
+    # A barrier limit of 0 ns makes the wait run out for every CTA that is not
+    # the last to arrive (the grid always has more than one CTA): the call
+    # returns, the status word says NVFP4_ERR_TIMEOUT, and the next call with
+    # the default limit is bit-exact with the oracle again.
+    from nvfp4_block_quantization_amax_b200 import _lib as L
+    x = pr1["w"] if flags & B2D else pr1["x"]
+    xd = x.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setenv("NVFP4_BARRIER_TIMEOUT_NS", "0")
+    api.nvfp4_quantize(xd, mode, flags | SP, seed=9, stream_id=1, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == L.NVFP4_ERR_TIMEOUT
+    monkeypatch.delenv("NVFP4_BARRIER_TIMEOUT_NS")
+    status.zero_()
+    g, o, _ = run_both(api, x, mode, flags | SP, seed=9, stream_id=1)
+    assert_same(g, o, flags)
+    api.nvfp4_quantize(xd, mode, flags | SP, seed=9, stream_id=1, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
 def test_single_pass_workspace_is_scratch(api, pr1):
     # the barrier counter is cleared by the call itself: a workspace full of
     # garbage, reused call after call, gives the same result
