@@ -20,6 +20,7 @@ from . import build as _build
 
 ROWWISE, COLWISE, BLOCK2D, ALPHA_PROVIDED, RHT, INVERSE_RHT = 0x1, 0x2, 0x4, 0x10, 0x40, 0x80
 HEADROOM = 0x200
+VECTOR_SCALES = 0x400
 RTN, FOUR_SIX, RHT_SR, MS_EDEN, RHT_SR_HW = 0, 1, 2, 3, 4
 OK, ERR_ARG, ERR_SHAPE, ERR_NONFINITE = 0, -1, -2, -4
 
@@ -97,6 +98,16 @@ def _configure(L):
     L.oracle_gemm_f64.argtypes = [_u8p, _u8p, ctypes.c_float, _u8p, _u8p, ctypes.c_float,
                                   _i64, _i64, _i64, _i64p, _i64, _i64p, _i64, _f64p]
     L.oracle_gemm_f64.restype = None
+    L.oracle_amax_vectors.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                      _f32p]
+    L.oracle_amax_vectors.restype = ctypes.c_int
+    L.oracle_quantize_vector_scales.argtypes = [_u16p, _i64, _i64, _i64, ctypes.c_int, ctypes.c_uint32,
+                                                ctypes.c_uint64, ctypes.c_uint32, _u8p, _u8p, _f32p,
+                                                _u8p, _u8p, _f32p, _f32p, _f32p]
+    L.oracle_quantize_vector_scales.restype = ctypes.c_int
+    L.oracle_gemm_f64_vector_scales.argtypes = [_u8p, _u8p, _f32p, _u8p, _u8p, _f32p, _i64, _i64, _i64,
+                                                _i64p, _i64, _i64p, _i64, _f64p]
+    L.oracle_gemm_f64_vector_scales.restype = None
     L.oracle_quantize_block16.argtypes = [_f32p, ctypes.c_float, ctypes.c_int, ctypes.c_uint64,
                                           ctypes.c_uint32, ctypes.c_uint64, _u8p, _u8p]
     L.oracle_quantize_block16.restype = ctypes.c_int
@@ -228,9 +239,55 @@ def amax(x, orient=0, rot=False, seed=0, C=None):
     return float(out[0])
 
 
+def amax_vectors(x, orient=0, rot=False, seed=0, C=None):
+    """amax of every row (orient 0) or column (orient 1), over rotated
+    16-blocks when rot is set."""
+    x = _bf16_bits(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    out = np.zeros(C if orient else R, np.float32)
+    _check(lib().oracle_amax_vectors(_p(x, _u16p), R, C, ld, orient, int(rot), seed, _p(out, _f32p)))
+    return out
+
+
+def quantize_vector_scales(x, mode, flags, seed=0, stream_id=0, C=None):
+    """1D quantization with one tensor scale per row (row orientation) or per
+    column (column orientation).  alpha_row [R] / alpha_col [C] are arrays;
+    amax_row / amax_col the largest vector amax."""
+    x = _bf16_bits(x)
+    R, ld = x.shape
+    C = ld if C is None else C
+    out = {}
+    cr = sr = cc = sc = ar = ac = None
+    if flags & ROWWISE:
+        cr = np.zeros((R, C // 2), np.uint8)
+        sr = np.zeros((R, C // 16), np.uint8)
+        ar = np.zeros(max(R, 1), np.float32)
+    if flags & COLWISE:
+        cc = np.zeros((C, R // 2), np.uint8)
+        sc = np.zeros((C, R // 16), np.uint8)
+        ac = np.zeros(max(C, 1), np.float32)
+    mr = np.zeros(1, np.float32)
+    mc = np.zeros(1, np.float32)
+    _check(lib().oracle_quantize_vector_scales(_p(x, _u16p), R, C, ld, mode, flags & ~VECTOR_SCALES, seed,
+                                               stream_id, _p(cr, _u8p), _p(sr, _u8p), _p(ar, _f32p),
+                                               _p(cc, _u8p), _p(sc, _u8p), _p(ac, _f32p), _p(mr, _f32p),
+                                               _p(mc, _f32p)))
+    if flags & ROWWISE:
+        out.update(codes_row=cr, scales_row=sr, alpha_row=ar[:R], amax_row=float(mr[0]))
+    if flags & COLWISE:
+        out.update(codes_col=cc, scales_col=sc, alpha_col=ac[:C], amax_col=float(mc[0]))
+    return out
+
+
 def quantize(x, mode, flags, seed=0, stream_id=0, alpha=None, C=None):
     """Quantize a [R, ld] uint16 (bf16) array whose first C columns are the
-    tensor.  Returns a dict with the requested outputs."""
+    tensor.  Returns a dict with the requested outputs.  With VECTOR_SCALES
+    (one tensor scale per row / column) see quantize_vector_scales."""
+    if flags & VECTOR_SCALES:
+        if alpha is not None:
+            raise ValueError("VECTOR_SCALES computes its own tensor scales")
+        return quantize_vector_scales(x, mode, flags, seed=seed, stream_id=stream_id, C=C)
     x = _bf16_bits(x)
     R, ld = x.shape
     C = ld if C is None else C
@@ -300,7 +357,24 @@ def dequantize(codes, scales, alpha, R, C, flags=0, seed=0):
 
 def gemm_f64(A, sA, alphaA, B, sB, alphaB, M, N, K, rows=None, cols=None):
     """FP64 reference D = alphaA alphaB (qA DeltaA)(qB DeltaB)^T on the given
-    rows / columns (None = all)."""
+    rows / columns (None = all).  alphaA / alphaB may be per-row arrays ([M],
+    [N]: one tensor scale per operand row)."""
+    if np.ndim(alphaA) or np.ndim(alphaB):
+        aA = np.broadcast_to(np.asarray(alphaA, np.float32), (M,)).copy()
+        aB = np.broadcast_to(np.asarray(alphaB, np.float32), (N,)).copy()
+        A = _c(A, np.uint8)
+        B = _c(B, np.uint8)
+        sA = _c(sA, np.uint8)
+        sB = _c(sB, np.uint8)
+        r = None if rows is None else _c(rows, np.int64)
+        c = None if cols is None else _c(cols, np.int64)
+        nr = M if r is None else len(r)
+        nc = N if c is None else len(c)
+        D = np.zeros((nr, nc), np.float64)
+        lib().oracle_gemm_f64_vector_scales(_p(A, _u8p), _p(sA, _u8p), _p(aA, _f32p), _p(B, _u8p), _p(sB, _u8p),
+                                            _p(aB, _f32p), M, N, K, _p(r, _i64p), nr, _p(c, _i64p), nc,
+                                            _p(D, _f64p))
+        return D
     A = _c(A, np.uint8)
     B = _c(B, np.uint8)
     sA = _c(sA, np.uint8)

@@ -56,6 +56,7 @@
 #define OR_BLOCK2D 0x4u
 #define OR_ALPHA_PROVIDED 0x10u
 #define OR_HEADROOM 0x200u
+#define OR_VECTOR_SCALES 0x400u
 #define OR_RHT 0x40u
 #define OR_INVERSE_RHT 0x80u
 
@@ -660,6 +661,89 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld,
   return OR_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Finer tensor scales ([NV] §九: the single global amax is named as a       */
+/* limitation, with per-row or per-block global scales as the remedy).       */
+/* ------------------------------------------------------------------------ */
+/* READING: the pages name the remedy without defining it.  The oracle takes
+ * the plainest form: Eq. 1 applied to each vector of the quantized operand on
+ * its own -- a row of x for the row orientation, a column of x for the column
+ * orientation (the rows of the GEMM operand, one per output row or column of
+ * the product) -- alpha_i = amax_i / (6 * 448), amax_i over that vector's
+ * (rotated) values; everything else is unchanged.  A "per-block" global scale
+ * with the 16-element block as its unit would coincide with the E4M3 block
+ * scale itself, so that variant is not a separate mode. */
+int oracle_amax_vectors(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int orient,
+                        int rot, uint64_t seed, float* amax) {
+  if (R < 0 || C < 0 || ld < C) return OR_ERR_SHAPE;
+  int64_t nvec = orient ? C : R, len = orient ? R : C;
+  if (rot && len % 16) return OR_ERR_SHAPE;
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t c = 0; c < C; ++c)
+      if (!isfinite(bf16_to_f32(x[r * ld + c]))) return OR_ERR_NONFINITE;
+  uint32_t signs = oracle_sign_bits(seed);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < nvec; ++i) {
+    float m = 0.0f;
+    if (!rot) {
+      for (int64_t k = 0; k < len; ++k) {
+        int64_t r = orient ? k : i, c = orient ? i : k;
+        m = fmaxf(m, fabsf(bf16_to_f32(x[r * ld + c])));
+      }
+    } else {
+      for (int64_t b = 0; b < len / 16; ++b) {
+        float v[16];
+        gather_block(x, ld, orient, i, b, 1, signs, v);
+        m = fmaxf(m, max_abs16(v));
+      }
+    }
+    amax[i] = m;
+  }
+  return OR_OK;
+}
+
+/* 1D quantization with one tensor scale per vector (flag OR_VECTOR_SCALES):
+ * alpha[i] = Eq. 1 of vector i's amax (or the headroom form), then the
+ * vector is quantized exactly as oracle_quantize_1d would with that alpha.
+ * Outputs as oracle_quantize; alpha_row [R] and alpha_col [C] are vectors;
+ * amax_row / amax_col receive the largest vector amax of the orientation. */
+int oracle_quantize_vector_scales(const uint16_t* x, int64_t R, int64_t C, int64_t ld,
+                                  int mode, uint32_t flags, uint64_t seed, uint32_t stream_id,
+                                  uint8_t* codes_row, uint8_t* scales_row, float* alpha_row,
+                                  uint8_t* codes_col, uint8_t* scales_col, float* alpha_col,
+                                  float* amax_row, float* amax_col) {
+  int want_row = (flags & OR_ROWWISE) != 0, want_col = (flags & OR_COLWISE) != 0;
+  if (mode < OR_RTN || mode > OR_RHT_SR_HW) return OR_ERR_ARG;
+  if (!want_row && !want_col) return OR_ERR_ARG;
+  if (flags & (OR_BLOCK2D | OR_ALPHA_PROVIDED)) return OR_ERR_ARG;
+  if (R < 0 || C < 0 || ld < C) return OR_ERR_SHAPE;
+  if (want_row && C % 16) return OR_ERR_SHAPE;
+  if (want_col && R % 16) return OR_ERR_SHAPE;
+  int rot = rotated(mode, flags);
+  for (int o = 0; o < 2; ++o) {
+    if (!(o ? want_col : want_row)) continue;
+    int64_t nvec = o ? C : R, len = o ? R : C;
+    float* av = (float*)malloc(sizeof(float) * (size_t)(nvec > 0 ? nvec : 1));
+    int st = oracle_amax_vectors(x, R, C, ld, o, rot, seed, av);
+    if (st) { free(av); return st; }
+    float tmax = 0.0f;
+    uint8_t* codes = o ? codes_col : codes_row;
+    uint8_t* scales = o ? scales_col : scales_row;
+    float* alpha = o ? alpha_col : alpha_row;
+    for (int64_t i = 0; i < nvec; ++i) {
+      tmax = fmaxf(tmax, av[i]);
+      float a = (flags & OR_HEADROOM) ? oracle_alpha_headroom(av[i]) : oracle_alpha_from_amax(av[i]);
+      if (alpha) alpha[i] = a;
+      oracle_quantize_1d(x, R, C, ld, o, mode, flags, seed, stream_id, a, i, i + 1,
+                         codes ? codes + i * (len / 2) : NULL, scales ? scales + i * (len / 16) : NULL);
+    }
+    if (o == 0 && amax_row) *amax_row = tmax;
+    if (o == 1 && amax_col) *amax_col = tmax;
+    free(av);
+  }
+  return OR_OK;
+}
+
 /* Dequantization: xhat = q * (alpha * Delta), optionally rotated back
  * (inverse transform along each 16-block).  codes [R, C/2]; scales [R, C/16]
  * or, with BLOCK2D, [R/16, C/16].  Output fp32 [R, C]. */
@@ -724,6 +808,26 @@ void oracle_gemm_f64(const uint8_t* A, const uint8_t* sA, float alphaA,
       D[i * ncols + j] = acc * (double)alphaA * (double)alphaB;
     }
     free(arow);
+  }
+}
+
+/* GEMM reference in FP64 with one tensor scale per operand row:
+ * D[m, n] = alphaA[m] alphaB[n] sum_k (qA DeltaA)(qB DeltaB); operands as in
+ * oracle_gemm_f64, alphaA [M], alphaB [N]. */
+void oracle_gemm_f64_vector_scales(const uint8_t* A, const uint8_t* sA, const float* alphaA,
+                                   const uint8_t* B, const uint8_t* sB, const float* alphaB,
+                                   int64_t M, int64_t N, int64_t K, const int64_t* rows,
+                                   int64_t nrows, const int64_t* cols, int64_t ncols,
+                                   double* D) {
+  if (!rows) nrows = M;
+  if (!cols) ncols = N;
+  oracle_gemm_f64(A, sA, 1.0f, B, sB, 1.0f, M, N, K, rows, nrows, cols, ncols, D);
+  for (int64_t i = 0; i < nrows; ++i) {
+    int64_t m = rows ? rows[i] : i;
+    for (int64_t j = 0; j < ncols; ++j) {
+      int64_t n = cols ? cols[j] : j;
+      D[i * ncols + j] *= (double)alphaA[m] * (double)alphaB[n];
+    }
   }
 }
 

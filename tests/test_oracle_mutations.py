@@ -10,6 +10,7 @@ import oracle
 from oracle import build as oracle_build
 import test_oracle_mx_pins as MXP
 import test_oracle_pins as P
+import test_oracle_vector_scales as VSP
 from test_oracle_pins import aten_philox, pr1  # noqa: F401  (fixtures)
 from nvfp4_block_quantization_amax_b200 import synthetic
 
@@ -90,6 +91,13 @@ MUTATIONS = [
      lambda f: P.test_dequant_matches_library_decode(f("pr1"))),
     ("GEMM drops a tensor scale", "D[i * ncols + j] = acc * (double)alphaA * (double)alphaB;",
      "D[i * ncols + j] = acc * (double)alphaA;", lambda f: P.test_gemm_f64_matches_numpy_matmul()),
+    ("vector scales from one vector's amax",
+     "float a = (flags & OR_HEADROOM) ? oracle_alpha_headroom(av[i]) : oracle_alpha_from_amax(av[i]);",
+     "float a = (flags & OR_HEADROOM) ? oracle_alpha_headroom(av[0]) : oracle_alpha_from_amax(av[0]);",
+     lambda f: VSP.test_vector_alpha_is_eq1_per_vector(VSP.x.__wrapped__(), False)),
+    ("vector-scaled GEMM column scale", "D[i * ncols + j] *= (double)alphaA[m] * (double)alphaB[n];",
+     "D[i * ncols + j] *= (double)alphaA[m] * (double)alphaA[n];",
+     lambda f: VSP.test_gemm_f64_vector_scales_matches_numpy()),
     ("MX shared exponent", "int e = (k - 1) - 2;", "int e = (k - 1) - 1;",
      lambda f: MXP.test_shared_exponent_puts_block_max_in_4_to_8()),
     ("MX nibble order", "(uint8_t)(q[2 * k] | (q[2 * k + 1] << 4));", "(uint8_t)(q[2 * k + 1] | (q[2 * k] << 4));",
