@@ -145,7 +145,10 @@ __device__ __forceinline__ float e2m1_sr_value_nb(float y, uint32_t u16) {
   const float t = __fmul_rn(a, m);
   const float fl = floorf(t);
   const float f = __fsub_rn(t, fl);
-  const float up = (static_cast<float>(u16) < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
+  // (float) u16 from the exact float 2^23 + u16, keeping the integer
+  // conversion unit out of the per-element path
+  const float fu = __fsub_rn(__uint_as_float(0x4B000000u | u16), 8388608.0f);
+  const float up = (fu < __fmul_rn(f, 65536.0f)) ? 1.0f : 0.0f;
   const float q = (a >= 6.0f) ? 6.0f : __fmul_rn(__fadd_rn(fl, up), inv_m);
   return copysignf(q, y);
 }
@@ -277,38 +280,45 @@ __device__ __forceinline__ float scale_raw(float amax_b, float alpha, float M) {
 // Encoding rounds to nearest even with saturation at +-6 (PTX
 // cvt.rn.satfinite.e2m1x2.f32, two values per byte); decoding is exact.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t e2m1x8_rne(float y0, float y1, float y2, float y3, float y4, float y5,
-                                               float y6, float y7) {
+// Two values -> one byte of codes, y_lo in the low nibble (PTX
+// cvt.rn.satfinite.e2m1x2.f32 takes the high element first), returned
+// through a 32-bit register.
+__device__ __forceinline__ uint32_t e2m1x2_rne(float y_lo, float y_hi) {
   uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(r)
-      : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(y_lo), "f"(y_hi));
   return r;
 }
 
+__device__ __forceinline__ uint32_t e2m1x8_rne(float y0, float y1, float y2, float y3, float y4, float y5,
+                                               float y6, float y7) {
+  const uint32_t b01 = __byte_perm(e2m1x2_rne(y0, y1), e2m1x2_rne(y2, y3), 0x7740u);   // [b0, b1, 0, 0]
+  const uint32_t b23 = __byte_perm(e2m1x2_rne(y4, y5), e2m1x2_rne(y6, y7), 0x7740u);   // [b2, b3, 0, 0]
+  return __byte_perm(b01, b23, 0x5410u);
+}
+
+// Each byte is taken out of the word in C++ and handed to the convert through
+// a 32-bit register (cvt.u8.u32 inside the asm): unpacking the word into four
+// .b8 registers inside one asm block decoded bytes 2 and 3 as zeros in some
+// inlining contexts on sm_100a, so this form is used throughout.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2) : "r"(byte));
+  return h2;
+}
+
 __device__ __forceinline__ void e2m1x8_values(uint32_t w, float* q) {
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
-      ".reg .b16 l0, l1, l2, l3, u0, u1, u2, u3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %8;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
-      "mov.b32 {l0, u0}, h0;\n\t"
-      "mov.b32 {l1, u1}, h1;\n\t"
-      "mov.b32 {l2, u2}, h2;\n\t"
-      "mov.b32 {l3, u3}, h3;\n\t"
-      "cvt.f32.f16 %0, l0;\n\tcvt.f32.f16 %1, u0;\n\t"
-      "cvt.f32.f16 %2, l1;\n\tcvt.f32.f16 %3, u1;\n\t"
-      "cvt.f32.f16 %4, l2;\n\tcvt.f32.f16 %5, u2;\n\t"
-      "cvt.f32.f16 %6, l3;\n\tcvt.f32.f16 %7, u3;\n\t}"
-      : "=f"(q[0]), "=f"(q[1]), "=f"(q[2]), "=f"(q[3]), "=f"(q[4]), "=f"(q[5]), "=f"(q[6]), "=f"(q[7])
-      : "r"(w));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t h2 = e2m1x2_to_f16x2((w >> (8 * k)) & 0xFFu);
+    q[2 * k] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    q[2 * k + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+  }
 }
 
 // Sign-only codes (magnitude 0) of one lane of sixteen pairs.
@@ -435,6 +445,124 @@ __device__ __forceinline__ void quantize_pair_rne(const float2* v, float alpha, 
     pa = ta ? pa4 : pa6;
     sbb = tb ? b4 : b6;
     pb = tb ? pb4 : pb6;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Table-driven block encoding.  For a fixed tensor scale alpha the element
+// scale of Eq. 3, s = RN(alpha * Delta), and its reciprocal take one of 128
+// values (one per E4M3 byte), so each CTA tabulates them once: entry b holds
+// {s, rinv} with rinv = RN(1 / s), or 0 where s = 0 or 1 / s overflows (the
+// block then encodes as signed zeros, as Eq. 3's reading requires).  A block
+// reads one entry instead of decoding its scale byte and rounding a
+// reciprocal; the values are the same IEEE results.
+// ---------------------------------------------------------------------------
+constexpr int kScaleTab = 128;
+
+__device__ __forceinline__ float2 scale_entry(float alpha, uint32_t b) {
+  const float s = __fmul_rn(alpha, e4m3_value(b));
+  float r = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+  if (isinf(r)) r = 0.0f;
+  return make_float2(s, r);
+}
+
+// Fill tab[0..127] (shared memory) for tensor scale alpha; the caller
+// synchronises the CTA before reading it.
+template <int NT>
+__device__ __forceinline__ void build_scale_tab(float2* tab, float alpha) {
+  for (int b = threadIdx.x; b < kScaleTab; b += NT) tab[b] = scale_entry(alpha, static_cast<uint32_t>(b));
+}
+
+// Two values rounded to E4M3 (nearest even, saturating at 448) in one
+// conversion: a in the low byte, b in the next.  a, b >= 0.
+__device__ __forceinline__ uint32_t e4m3x2_rne(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Smallest E4M3 value not below each of a, b (saturating at 448).
+__device__ __forceinline__ void e4m3x2_ceil(float a, float b, uint32_t& ba, uint32_t& bb) {
+  const uint32_t r = e4m3x2_rne(a, b);
+  ba = r & 0xFFu;
+  bb = r >> 8;
+  if (ba < 0x7Eu && e4m3_value(ba) < a) ++ba;
+  if (bb < 0x7Eu && e4m3_value(bb) < b) ++bb;
+}
+
+// Per-block scale context of one tensor scale: the table, and the Eq. 2
+// denominators RN(alpha * 6) and RN(alpha * 4).
+struct ScaleCtx {
+  const float2* tab;
+  float alpha, den6, den4;
+};
+
+__device__ __forceinline__ ScaleCtx make_scale_ctx(const float2* tab, float alpha) {
+  return ScaleCtx{tab, alpha, __fmul_rn(alpha, 6.0f), __fmul_rn(alpha, 4.0f)};
+}
+
+// Eq. 2's quotient amax_b / den (0 when den is 0).
+__device__ __forceinline__ float scale_quot(float amax_b, float den) {
+  return (den == 0.0f) ? 0.0f : __fdiv_rn(amax_b, den);
+}
+
+// Codes of the two lane-paired blocks v * rinv (Eq. 3 as a reciprocal
+// multiply; rinv = 0 gives signed zeros).
+__device__ __forceinline__ void encode_x2(const float2* v, float2 rinv2, Packed16& pa, Packed16& pb) {
+  float2 y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = mul2(v[i], rinv2);
+  pa.lo = e2m1x8_rne(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
+  pa.hi = e2m1x8_rne(y[8].x, y[9].x, y[10].x, y[11].x, y[12].x, y[13].x, y[14].x, y[15].x);
+  pb.lo = e2m1x8_rne(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
+  pb.hi = e2m1x8_rne(y[8].y, y[9].y, y[10].y, y[11].y, y[12].y, y[13].y, y[14].y, y[15].y);
+}
+
+// Squared error of two encodings in the original domain (the Four Over Six
+// criterion): sum of RN((v - RN(q s))^2), s2 = (s_a, s_b) from the table.
+// Same operations as sq_error_x2: the subtraction of the rounded product and
+// the first summation level stay scalar (never merged with the products).
+__device__ __forceinline__ float2 sq_error_tab(const float2* v, float2 s2, const Packed16& pa, const Packed16& pb) {
+  float2 q[16], e[16];
+  decode16x2(pa, pb, q);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 d = sub2_exact(v[i], mul2(q[i], s2));
+    e[i] = mul2(d, d);
+  }
+  return sum16x2(e);
+}
+
+// Round-to-nearest block quantization of two lane-paired blocks from the
+// table (Four Over Six §2.1 Eq. 2-3; with FOUR_SIX the better of the M = 6
+// and M = 4 candidates by squared error, ties to M = 6, §1 Table 1).
+template <bool FOUR_SIX>
+__device__ __forceinline__ void quantize_pair_tab(const float2* v, const ScaleCtx& c, Packed16& pa, Packed16& pb,
+                                                  uint32_t& sba, uint32_t& sbb) {
+  float ma, mb;
+  max_abs16x2(v, ma, mb);
+  const uint32_t s6 = e4m3x2_rne(scale_quot(ma, c.den6), scale_quot(mb, c.den6));
+  const uint32_t a6 = s6 & 0xFFu, b6 = s6 >> 8;
+  const float2 ta6 = c.tab[a6], tb6 = c.tab[b6];
+  encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
+  sba = a6;
+  sbb = b6;
+  if constexpr (FOUR_SIX) {
+    const uint32_t s4 = e4m3x2_rne(scale_quot(ma, c.den4), scale_quot(mb, c.den4));
+    const uint32_t a4 = s4 & 0xFFu, b4 = s4 >> 8;
+    const float2 ta4 = c.tab[a4], tb4 = c.tab[b4];
+    Packed16 pa4, pb4;
+    encode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4);
+    const float2 e6 = sq_error_tab(v, make_float2(ta6.x, tb6.x), pa, pb);
+    const float2 e4 = sq_error_tab(v, make_float2(ta4.x, tb4.x), pa4, pb4);
+    if (e4.x < e6.x) {
+      sba = a4;
+      pa = pa4;
+    }
+    if (e4.y < e6.y) {
+      sbb = b4;
+      pb = pb4;
+    }
   }
 }
 

@@ -279,19 +279,23 @@ __device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t wo
 }
 
 // have_words: MS-EDEN only - wa / wb already hold the blocks' scale-SR words.
+// c: the tensor scale's table (s and 1 / s per scale byte) and the Eq. 2
+// denominators.
 template <int MODE>
-__device__ __forceinline__ void quantize_pair(const float2* v, float alpha, const PhiloxKeys& K, uint32_t c2,
+__device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c, const PhiloxKeys& K, uint32_t c2,
                                               uint64_t blka, uint64_t blkb, Packed16& pa, Packed16& pb,
                                               uint32_t& sba, uint32_t& sbb, bool have_words = false,
                                               uint32_t wa = 0u, uint32_t wb = 0u) {
   if constexpr (MODE == kModeRTN || MODE == kModeFourSix) {
-    quantize_pair_rne<MODE == kModeFourSix>(v, alpha, pa, pb, sba, sbb);
+    quantize_pair_tab<MODE == kModeFourSix>(v, c, pa, pb, sba, sbb);
   } else if constexpr (MODE == kModeMsEden) {
+    // RTN codes under the provisional scale (M = 6), then the unbiasing
+    // scale sum(r^2) / (alpha sum(r q)), stochastically rounded to E4M3
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    const uint32_t prova = e4m3_rne(scale_raw(ma, alpha, 6.0f));
-    const uint32_t provb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
-    encode_rne_x2(v, alpha, prova, provb, pa, pb);
+    const uint32_t prov = e4m3x2_rne(scale_quot(ma, c.den6), scale_quot(mb, c.den6));
+    const float2 ta = c.tab[prov & 0xFFu], tb = c.tab[prov >> 8];
+    encode_x2(v, make_float2(ta.y, tb.y), pa, pb);
     float2 q[16], rr[16], rq[16];
     decode16x2(pa, pb, q);
 #pragma unroll
@@ -300,7 +304,7 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
       rq[i] = mul2(v[i], q[i]);
     }
     const float2 num = sum16x2(rr);
-    const float2 den = mul2(make_float2(alpha, alpha), sum16x2(rq));
+    const float2 den = mul2(make_float2(c.alpha, c.alpha), sum16x2(rq));
     if (!have_words) {
       const uint64_t ua = blka >> 2, ub = blkb >> 2;
       const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagScaleSR);
@@ -318,64 +322,56 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
     // handed over last element first so that nibble j holds element 4g + j.
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    sba = e4m3_ceil(scale_raw(ma, alpha, 6.0f));
-    sbb = e4m3_ceil(scale_raw(mb, alpha, 6.0f));
-    const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
-    const float rb = __frcp_rn(__fmul_rn(alpha, e4m3_value(sbb)));
+    e4m3x2_ceil(scale_quot(ma, c.den6), scale_quot(mb, c.den6), sba, sbb);
+    const float2 r2 = make_float2(c.tab[sba].y, c.tab[sbb].y);
     const uint4 da = philox(K, static_cast<uint32_t>(blka), static_cast<uint32_t>(blka >> 32), c2, kTagValueSRHw);
     const uint4 db = philox(K, static_cast<uint32_t>(blkb), static_cast<uint32_t>(blkb >> 32), c2, kTagValueSRHw);
-    const uint32_t wa[4] = {da.x, da.y, da.z, da.w}, wb[4] = {db.x, db.y, db.z, db.w};
-    const float2 r2 = make_float2(ra, rb);
+    const uint32_t wa4[4] = {da.x, da.y, da.z, da.w}, wb4[4] = {db.x, db.y, db.z, db.w};
     float2 y[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = mul2(v[i], r2);
     uint32_t ca[4], cb[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      ca[g] = e2m1x4_sr_hw(y[4 * g + 3].x, y[4 * g + 2].x, y[4 * g + 1].x, y[4 * g].x, wa[g]);
-      cb[g] = e2m1x4_sr_hw(y[4 * g + 3].y, y[4 * g + 2].y, y[4 * g + 1].y, y[4 * g].y, wb[g]);
+      ca[g] = e2m1x4_sr_hw(y[4 * g + 3].x, y[4 * g + 2].x, y[4 * g + 1].x, y[4 * g].x, wa4[g]);
+      cb[g] = e2m1x4_sr_hw(y[4 * g + 3].y, y[4 * g + 2].y, y[4 * g + 1].y, y[4 * g].y, wb4[g]);
     }
-    // the sign nibble follows the input's sign bit, zeros included
+    // the sign nibble follows the input's sign bit, zeros included (a zero
+    // reciprocal leaves magnitude 0 and the sign alone)
     const Packed16 sa = sign_codes16<false>(v), sb = sign_codes16<true>(v);
     pa.lo = (ca[0] | (ca[1] << 16)) | sa.lo;
     pa.hi = (ca[2] | (ca[3] << 16)) | sa.hi;
     pb.lo = (cb[0] | (cb[1] << 16)) | sb.lo;
     pb.hi = (cb[2] | (cb[3] << 16)) | sb.hi;
-    if (isinf(ra)) pa = sa;
-    if (isinf(rb)) pb = sb;
   } else {  // RHT + stochastic rounding of the values
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    sba = e4m3_ceil(scale_raw(ma, alpha, 6.0f));
-    sbb = e4m3_ceil(scale_raw(mb, alpha, 6.0f));
-    const float ra = __frcp_rn(__fmul_rn(alpha, e4m3_value(sba)));
-    const float rb = __frcp_rn(__fmul_rn(alpha, e4m3_value(sbb)));
+    e4m3x2_ceil(scale_quot(ma, c.den6), scale_quot(mb, c.den6), sba, sbb);
+    const float2 r2 = make_float2(c.tab[sba].y, c.tab[sbb].y);
     // element i uses half (i & 1) of word (i >> 1) & 3 of draw i >> 3 (unit 2 blk + draw)
-    uint32_t wa[8], wb[8];
+    uint32_t wa8[8], wb8[8];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const uint64_t ua = 2 * blka + j, ub = 2 * blkb + j;
       const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagValueSR);
       const uint4 db = philox(K, static_cast<uint32_t>(ub), static_cast<uint32_t>(ub >> 32), c2, kTagValueSR);
-      wa[4 * j] = da.x; wa[4 * j + 1] = da.y; wa[4 * j + 2] = da.z; wa[4 * j + 3] = da.w;
-      wb[4 * j] = db.x; wb[4 * j + 1] = db.y; wb[4 * j + 2] = db.z; wb[4 * j + 3] = db.w;
+      wa8[4 * j] = da.x; wa8[4 * j + 1] = da.y; wa8[4 * j + 2] = da.z; wa8[4 * j + 3] = da.w;
+      wb8[4 * j] = db.x; wb8[4 * j + 1] = db.y; wb8[4 * j + 2] = db.z; wb8[4 * j + 3] = db.w;
     }
-    const float2 r2 = make_float2(ra, rb);
     float qa[16], qb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 y = mul2(v[i], r2);
       const int w = ((i >> 3) << 2) | ((i >> 1) & 3), sh = 16 * (i & 1);
-      qa[i] = e2m1_sr_value_nb(y.x, (wa[w] >> sh) & 0xFFFFu);
-      qb[i] = e2m1_sr_value_nb(y.y, (wb[w] >> sh) & 0xFFFFu);
+      qa[i] = e2m1_sr_value_nb(y.x, (wa8[w] >> sh) & 0xFFFFu);
+      qb[i] = e2m1_sr_value_nb(y.y, (wb8[w] >> sh) & 0xFFFFu);
     }
-    // the rounded values lie on the grid, so their encoding is exact
+    // the rounded values lie on the grid, so their encoding is exact (a zero
+    // reciprocal gives signed zeros)
     pa.lo = e2m1x8_rne(qa[0], qa[1], qa[2], qa[3], qa[4], qa[5], qa[6], qa[7]);
     pa.hi = e2m1x8_rne(qa[8], qa[9], qa[10], qa[11], qa[12], qa[13], qa[14], qa[15]);
     pb.lo = e2m1x8_rne(qb[0], qb[1], qb[2], qb[3], qb[4], qb[5], qb[6], qb[7]);
     pb.hi = e2m1x8_rne(qb[8], qb[9], qb[10], qb[11], qb[12], qb[13], qb[14], qb[15]);
-    if (isinf(ra)) pa = sign_codes16<false>(v);
-    if (isinf(rb)) pb = sign_codes16<true>(v);
   }
 }
 
@@ -386,9 +382,13 @@ __device__ __forceinline__ void quantize_pair(const float2* v, float alpha, cons
 // unit k / 2, so one draw serves the pair.
 // ===========================================================================
 template <int MODE, bool ROT, int NT>
-__device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint32_t* red) {
+__device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint32_t* red,
+                                                float2* tab) {
   float alpha, alpha_unused;
   resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red, cta);
+  build_scale_tab<NT>(tab, alpha);
+  __syncthreads();
+  const ScaleCtx sc = make_scale_ctx(tab, alpha);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -401,17 +401,34 @@ __device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta
   const uint32_t nb = a.nb_row.d;
   const uint32_t total = static_cast<uint32_t>(a.R) * nb;
   const uint32_t npairs = (total + 1) / 2;
+  const uint32_t stride = ncta * NT;
   const bool gemm = (a.flags & kGemmScaleLayout) != 0;
   const bool check = (a.flags & kAlphaProvided) != 0;
-  for (uint32_t pk = cta * NT + threadIdx.x; pk < npairs; pk += ncta * NT) {
+  // Pair pk holds blocks 2 pk and 2 pk + 1 (64 contiguous bytes when they
+  // share a row).  The next pair's loads are issued before this pair is
+  // encoded, so every thread keeps a pair in flight while it computes.
+  auto load_pair = [&](uint32_t pk, uint4& a0, uint4& a1, uint4& b0, uint4& b1) {
+    const uint32_t ka = 2 * pk, kb = ka + 1 < total ? ka + 1 : ka;
+    const uint32_t ra = fastdiv(ka, a.nb_row), cba = ka - ra * nb;
+    const uint32_t rb = fastdiv(kb, a.nb_row), cbb = kb - rb * nb;
+    const uint4* pa = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(ra) * a.ld + 16 * cba);
+    const uint4* pb = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(rb) * a.ld + 16 * cbb);
+    a0 = __ldcs(pa);
+    a1 = __ldcs(pa + 1);
+    b0 = __ldcs(pb);
+    b1 = __ldcs(pb + 1);
+  };
+  uint32_t pk = cta * NT + threadIdx.x;
+  uint4 n0, n1, n2, n3;
+  if (pk < npairs) load_pair(pk, n0, n1, n2, n3);
+  for (; pk < npairs; pk += stride) {
+    const uint4 a0 = n0, a1 = n1, b0 = n2, b1 = n3;
+    if (pk + stride < npairs) load_pair(pk + stride, n0, n1, n2, n3);
     const uint32_t ka = 2 * pk, kb = ka + 1;
     const bool vb = kb < total;
     const uint32_t ra = fastdiv(ka, a.nb_row), cba = ka - ra * nb;
     const uint32_t kk = vb ? kb : ka;
     const uint32_t rb = fastdiv(kk, a.nb_row), cbb = kk - rb * nb;
-    const uint4* pa = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(ra) * a.ld + 16 * cba);
-    const uint4* pb = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(rb) * a.ld + 16 * cbb);
-    const uint4 a0 = __ldcs(pa), a1 = __ldcs(pa + 1), b0 = __ldcs(pb), b1 = __ldcs(pb + 1);
     if (check) {
       uint32_t hin = 0;
       const uint32_t w[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
@@ -425,14 +442,19 @@ __device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta
     if constexpr (ROT) rht16x2_presigned(v);
     Packed16 qa, qb;
     uint32_t sa, sb;
-    quantize_pair<MODE>(v, alpha, K, c2, ka, kb, qa, qb, sa, sb);
-    *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(ra) * (a.C / 2) + 8 * cba) = make_uint2(qa.lo, qa.hi);
-    if (a.scales_row)
+    quantize_pair<MODE>(v, sc, K, c2, ka, kb, qa, qb, sa, sb);
+    uint8_t* ca = a.codes_row + static_cast<int64_t>(ra) * (a.C / 2) + 8 * cba;
+    if (vb && rb == ra && (reinterpret_cast<uintptr_t>(ca) & 15u) == 0) {
+      *reinterpret_cast<uint4*>(ca) = make_uint4(qa.lo, qa.hi, qb.lo, qb.hi);
+    } else {
+      *reinterpret_cast<uint2*>(ca) = make_uint2(qa.lo, qa.hi);
+      if (vb)
+        *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(rb) * (a.C / 2) + 8 * cbb) =
+            make_uint2(qb.lo, qb.hi);
+    }
+    if (a.scales_row) {
       a.scales_row[gemm ? gemm_scale_offset(ra, cba, nb) : static_cast<int64_t>(ka)] = static_cast<uint8_t>(sa);
-    if (vb) {
-      *reinterpret_cast<uint2*>(a.codes_row + static_cast<int64_t>(rb) * (a.C / 2) + 8 * cbb) =
-          make_uint2(qb.lo, qb.hi);
-      if (a.scales_row)
+      if (vb)
         a.scales_row[gemm ? gemm_scale_offset(rb, cbb, nb) : static_cast<int64_t>(kb)] = static_cast<uint8_t>(sb);
     }
   }
@@ -463,6 +485,8 @@ struct TileStaging {
   uint8_t colscale[TC][TR / 16];     // their scales (2D: unused)
   uint8_t scale2d[TR / 16][TC / 16]; // chosen 16x16 scales (2D)
   uint32_t red[TNT / 32];
+  float2 tab_r[kScaleTab];           // {s, 1 / s} per scale byte, row orientation
+  float2 tab_c[kScaleTab];           // the same for the column orientation
 };
 
 template <int MODE, bool ROT, bool ROW, bool COL>
@@ -474,6 +498,10 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   uint32_t* red = stg.red;
   float alpha_r, alpha_c;
   resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
+  if constexpr (ROW) build_scale_tab<TNT>(stg.tab_r, alpha_r);
+  if constexpr (COL) build_scale_tab<TNT>(stg.tab_c, alpha_c);
+  __syncthreads();
+  const ScaleCtx scr = make_scale_ctx(stg.tab_r, alpha_r), scc = make_scale_ctx(stg.tab_c, alpha_c);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -585,7 +613,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         const uint64_t blkb = static_cast<uint64_t>(grb) * (C / 16) + gcb;
         Packed16 pa, pb;
         uint32_t sa, sb;
-        quantize_pair<MODE>(v, alpha_r, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+        quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
         if (va) {
           *reinterpret_cast<uint2*>(a.codes_row + gra * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
           if (a.scales_row)
@@ -617,7 +645,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
         Packed16 qa, qb;
         uint32_t sa, sb;
-        quantize_pair<MODE>(v, alpha_c, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
+        quantize_pair<MODE>(v, scc, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
                             static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
@@ -670,6 +698,9 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
   // one tensor scale for both orientations: the plain amax, whose partials
   // both orientations read (alpha_c == alpha; it is computed to publish it)
   resolve_alpha<TNT>(a, true, COL, ROW, COL, alpha, alpha_c, red, cta);
+  build_scale_tab<TNT>(stg.tab_r, alpha);
+  __syncthreads();
+  const ScaleCtx sc = make_scale_ctx(stg.tab_r, alpha);
   const bool gemm = (a.flags & kGemmScaleLayout) != 0;
   const bool check = (a.flags & kAlphaProvided) != 0;
   const int t = threadIdx.x;
@@ -742,15 +773,19 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
         ma = fmaxf(ma, __shfl_xor_sync(0xFFFFFFFFu, ma, o));
         mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
       }
-      uint32_t sa = e4m3_rne(scale_raw(ma, alpha, 6.0f)), sb = e4m3_rne(scale_raw(mb, alpha, 6.0f));
+      const uint32_t s6 = e4m3x2_rne(scale_quot(ma, sc.den6), scale_quot(mb, sc.den6));
+      uint32_t sa = s6 & 0xFFu, sb = s6 >> 8;
+      const float2 ta6 = sc.tab[sa], tb6 = sc.tab[sb];
       Packed16 pa, pb;
-      encode_rne_x2(v, alpha, sa, sb, pa, pb);
+      encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
       if constexpr (MODE == kModeFourSix) {
-        const uint32_t sa4 = e4m3_rne(scale_raw(ma, alpha, 4.0f)), sb4 = e4m3_rne(scale_raw(mb, alpha, 4.0f));
+        const uint32_t s4 = e4m3x2_rne(scale_quot(ma, sc.den4), scale_quot(mb, sc.den4));
+        const uint32_t sa4 = s4 & 0xFFu, sb4 = s4 >> 8;
+        const float2 ta4 = sc.tab[sa4], tb4 = sc.tab[sb4];
         Packed16 pa4, pb4;
-        encode_rne_x2(v, alpha, sa4, sb4, pa4, pb4);
-        float2 e6 = sq_error_x2(v, alpha, sa, sb, pa, pb);
-        float2 e4 = sq_error_x2(v, alpha, sa4, sb4, pa4, pb4);
+        encode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4);
+        float2 e6 = sq_error_tab(v, make_float2(ta6.x, tb6.x), pa, pb);
+        float2 e4 = sq_error_tab(v, make_float2(ta4.x, tb4.x), pa4, pb4);
         // block error = the half-warp's row errors summed in butterfly order
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) {
@@ -807,7 +842,8 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
         }
         const uint32_t sbyte = scale2d[rb][cp >> 3];
         Packed16 qa, qb;
-        encode_rne_x2(v, alpha, sbyte, sbyte, qa, qb);
+        const float r = sc.tab[sbyte].y;
+        encode_x2(v, make_float2(r, r), qa, qb);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
       }
@@ -863,7 +899,8 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
 template <int MODE, bool ROT, int NT>
 __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
   __shared__ uint32_t red[NT / 32];
-  quant_rows_body<MODE, ROT, NT>(a, blockIdx.x, gridDim.x, red);
+  __shared__ float2 tab[kScaleTab];
+  quant_rows_body<MODE, ROT, NT>(a, blockIdx.x, gridDim.x, red, tab);
 }
 
 template <int MODE, bool ROT, bool ROW, bool COL>
@@ -949,7 +986,7 @@ __global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, 
   if constexpr (TWO_D) {
     quant_tile_2d_body<MODE, ROW, COL>(a, cta, ncta, tile_ring, stg);
   } else if constexpr (ROW && !COL) {
-    quant_rows_body<MODE, ROT, TNT>(a, cta, ncta, stg.red);
+    quant_rows_body<MODE, ROT, TNT>(a, cta, ncta, stg.red, stg.tab_r);
   } else {
     quant_tile_1d_body<MODE, ROT, ROW, COL>(a, cta, ncta, tile_ring, stg);
   }
