@@ -592,13 +592,28 @@ __device__ __forceinline__ int64_t gemm_scale_byte(int64_t m, int64_t j, int64_t
   return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
 }
 
+// Tile order of the CTA-pair kernel: groups of `gm` M-tiles (the whole N
+// range each), M fastest inside a group.  A wave of pairs then touches only
+// one group's A panels and its B panels, which stay in L2 while the group is
+// worked through, instead of every A panel per wave (the M-fastest order
+// over the full M range re-read A from DRAM on the K = 14336 / 8192 shapes).
+__device__ __forceinline__ void pair_tile_coords(int tile, int m_tiles, int n_tiles, int gm, int& tile_m,
+                                                 int& tile_n) {
+  const int group = tile / (gm * n_tiles);
+  const int local = tile - group * gm * n_tiles;
+  const int m0 = group * gm;
+  const int rows = min(gm, m_tiles - m0);
+  tile_m = m0 + local % rows;
+  tile_n = local / rows;
+}
+
 template <int QMODE, bool MX = false>
 __global__ void __launch_bounds__(P_THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
                            const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
                            const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status,
-                           const EpiQuant eq) {
+                           const EpiQuant eq, int group_m) {
   using PC = PairCfg<MX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -655,7 +670,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       int it = 0;
       bool stop = false;
       for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
-        const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+        int tile_m, tile_n;
+        pair_tile_coords(tile, m_tiles, N / 256, group_m, tile_m, tile_n);
         for (int kt = 0; kt < kstages; ++kt, ++it) {
           const int s = it % PC::STAGES;
           const uint32_t ph = (it / PC::STAGES) & 1;
@@ -762,13 +778,17 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     if constexpr (QMODE != kNoEpiQuant) eq_alpha = __ldg(eq.alpha);
     int ti = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++ti) {
-      const int tile_m = tile % m_tiles, tile_n = tile / m_tiles;
+      int tile_m, tile_n;
+      pair_tile_coords(tile, m_tiles, N / 256, group_m, tile_m, tile_n);
       if (!mbar_wait(smem_u32(acc_full), ti & 1, abort_flag)) break;
       fence_after();
       const int row0 = tile_m * 256 + 128 * static_cast<int>(rank) + 32 * q;
       const int col0 = tile_n * 256 + 128 * h;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + 128 * h;
       if (!out_fp32) {
+        // two rounds of 64 columns: load, wait, convert to packed bf16; the
+        // accumulator is handed back once the whole row is in registers
+        // (measured faster than loading all 128 columns before one wait)
         uint32_t packed[64];
 #pragma unroll
         for (int c = 0; c < 128; c += 64) {
@@ -1018,9 +1038,16 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // M-tiles per raster group: as many as keep the group's A panels plus all
+  // of B within about 64 MB of L2 (operand bytes per 256-row panel: K / 2
+  // codes + K / 16 scales)
+  const int64_t panel = 256 * (K / 2 + K / 16);
+  const int64_t m_tiles = M / 256, n_tiles = N / 256;
+  int64_t gm = (int64_t(64) << 20) / panel - n_tiles;
+  gm = gm < 1 ? 1 : (gm > m_tiles ? m_tiles : gm);
   cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE, MX>, ma, mb, md, msa, msb, alphaA, alphaB,
                                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                                     static_cast<int>(fp32), status, eq);
+                                     static_cast<int>(fp32), status, eq, static_cast<int>(gm));
   note_launch();
   return e;
 }
