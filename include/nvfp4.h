@@ -108,6 +108,19 @@ typedef enum {
 #define NVFP4_HEADROOM 0x200u       /* alpha = amax / (4 * 448) instead of Eq. 1's
                                      * amax / (6 * 448): the M = 4 candidate of
                                      * Four Over Six then never saturates        */
+#define NVFP4_VECTOR_SCALES 0x400u  /* one tensor scale per row of the quantized
+                                     * operand ([NV] §九 names finer-than-tensor
+                                     * global scales as the remedy for one global
+                                     * amax; READING: Eq. 1 applied to each vector
+                                     * on its own): alpha_i = amax_i / (6 * 448)
+                                     * over row i of x (rowwise) or column i of x
+                                     * (columnwise), rotated values in rotating
+                                     * modes.  alpha_row then points to R floats,
+                                     * alpha_col to C floats; amax_out receives
+                                     * the largest vector amax per orientation.
+                                     * 1D blocks only (not with BLOCK2D,
+                                     * SINGLE_PASS or ALPHA_PROVIDED).  The
+                                     * workspace holds the R + C vector maxima. */
 /* nvfp4_dequantize flags (NVFP4_BLOCK2D and NVFP4_GEMM_SCALE_LAYOUT also apply) */
 #define NVFP4_INVERSE_RHT 0x80u     /* undo the rotation after decoding          */
 #define NVFP4_OUT_BF16 0x100u       /* write bf16 instead of fp32                */
@@ -233,6 +246,20 @@ NVFP4_API nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const f
                           int64_t M, int64_t N, int64_t K, void* D, int out_dtype,
                           int64_t ldd, void* workspace, size_t workspace_bytes,
                           void* stream);
+
+/* nvfp4_gemm for operands quantized with NVFP4_VECTOR_SCALES (one tensor
+ * scale per operand row; [NV] §九, READING as at that flag):
+ *     D[m, n] = alphaA[m] * alphaB[n] * sum_k (qA DeltaA)(qB DeltaB)
+ * alphaA: device floats [M] (the alpha_row vector of A's quantization, or
+ * alpha_col when A is a column-orientation output), alphaB: [N] likewise.
+ * D = RN(RN(acc * alphaA[m]) * alphaB[n]) in FP32, then bf16 or fp32 as for
+ * nvfp4_gemm.  M % 256 == 0, N % 256 == 0, K % 128 == 0; operands and D
+ * 16-byte aligned.  The workspace is optional as for nvfp4_gemm. */
+NVFP4_API nvfp4_status_t nvfp4_gemm_vector_scales(const uint8_t* A, const uint8_t* sA, const float* alphaA,
+                                                  const uint8_t* B, const uint8_t* sB, const float* alphaB,
+                                                  int64_t M, int64_t N, int64_t K, void* D, int out_dtype,
+                                                  int64_t ldd, void* workspace, size_t workspace_bytes,
+                                                  void* stream);
 
 /* nvfp4_gemm whose epilogue also quantizes the output for the next layer
  * ([NV] §九 counts the separate amax and quantize passes over an activation

@@ -21,6 +21,7 @@ NVFP4_COLWISE = 0x2
 NVFP4_BLOCK2D = 0x4
 NVFP4_SINGLE_PASS = 0x8
 NVFP4_HEADROOM = 0x200
+NVFP4_VECTOR_SCALES = 0x400
 NVFP4_ALPHA_PROVIDED = 0x10
 NVFP4_GEMM_SCALE_LAYOUT = 0x20
 NVFP4_RHT = 0x40
@@ -31,7 +32,7 @@ NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
 EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
-            "nvfp4_gemm", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "nvfp4_launch_count",
+            "nvfp4_gemm", "nvfp4_gemm_vector_scales", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "nvfp4_launch_count",
             "nvfp4_status_string", "nvfp4_version")
 
 
@@ -67,6 +68,8 @@ def load(path=LIB_PATH):
     L.nvfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
     L.nvfp4_gemm.restype = ctypes.c_int
+    L.nvfp4_gemm_vector_scales.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
+    L.nvfp4_gemm_vector_scales.restype = ctypes.c_int
     L.nvfp4_gemm_quantize.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i64, ctypes.c_int, u32, vp,
                                       vp, vp, vp, vp, sz, vp]
     L.nvfp4_gemm_quantize.restype = ctypes.c_int
@@ -113,6 +116,12 @@ def nvfp4_gemm(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, workspa
                workspace_bytes, stream):
     return int(load().nvfp4_gemm(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd,
                                  workspace, workspace_bytes, stream))
+
+
+def nvfp4_gemm_vector_scales(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, workspace,
+                             workspace_bytes, stream):
+    return int(load().nvfp4_gemm_vector_scales(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd,
+                                               workspace, workspace_bytes, stream))
 
 
 def nvfp4_gemm_quantize(A, sA, alphaA, B, sB, alphaB, M, N, K, D, ldd, mode, flags, alpha_out, codes, scales,

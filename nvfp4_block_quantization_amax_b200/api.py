@@ -12,7 +12,7 @@ from . import _lib as L
 from ._lib import (NVFP4_ALPHA_PROVIDED, NVFP4_BLOCK2D, NVFP4_COLWISE, NVFP4_FOUR_SIX,  # noqa: F401
                    NVFP4_GEMM_SCALE_LAYOUT, NVFP4_INVERSE_RHT, NVFP4_MS_EDEN, NVFP4_OUT_BF16,
                    NVFP4_OUT_DTYPE_BF16, NVFP4_OUT_DTYPE_FP32, NVFP4_RHT, NVFP4_RHT_SR, NVFP4_RHT_SR_HW,
-                   NVFP4_ROWWISE, NVFP4_RTN, NVFP4_SINGLE_PASS)
+                   NVFP4_ROWWISE, NVFP4_RTN, NVFP4_SINGLE_PASS, NVFP4_VECTOR_SCALES)
 
 
 class NVFP4Error(RuntimeError):
@@ -63,14 +63,15 @@ def _need_matrix(t: torch.Tensor, rows: int, cols: int, dtype, what: str, device
 def check_outputs(q: "QTensor", R: int, C: int, flags: int, device=None):
     """Raise unless q's buffers can take the outputs of nvfp4_quantize on an
     [R, C] tensor with these flags."""
+    vec = bool(flags & NVFP4_VECTOR_SCALES)
     if flags & NVFP4_ROWWISE:
         _need(q.codes_row, R * (C // 2), torch.uint8, "codes_row", device)
         _need(q.scales_row, math.prod(scale_shape(R, C, flags)), torch.uint8, "scales_row", device)
-        _need(q.alpha_row, 1, torch.float32, "alpha_row", device)
+        _need(q.alpha_row, R if vec else 1, torch.float32, "alpha_row", device)
     if flags & NVFP4_COLWISE:
         _need(q.codes_col, C * (R // 2), torch.uint8, "codes_col", device)
         _need(q.scales_col, math.prod(scale_shape(C, R, flags)), torch.uint8, "scales_col", device)
-        _need(q.alpha_col, 1, torch.float32, "alpha_col", device)
+        _need(q.alpha_col, C if vec else 1, torch.float32, "alpha_col", device)
     if q.amax is not None:
         _need(q.amax, 2, torch.float32, "amax", device)
 
@@ -100,14 +101,15 @@ def scale_shape(rows: int, cols: int, flags: int):
 def alloc_outputs(R: int, C: int, flags: int, device) -> QTensor:
     q = QTensor()
     u8 = dict(dtype=torch.uint8, device=device)
+    vec = bool(flags & NVFP4_VECTOR_SCALES)   # one tensor scale per row / column
     if flags & NVFP4_ROWWISE:
         q.codes_row = torch.empty((R, C // 2), **u8)
         q.scales_row = torch.empty(scale_shape(R, C, flags), **u8)
-        q.alpha_row = torch.empty(1, dtype=torch.float32, device=device)
+        q.alpha_row = torch.empty(max(R, 1) if vec else 1, dtype=torch.float32, device=device)
     if flags & NVFP4_COLWISE:
         q.codes_col = torch.empty((C, R // 2), **u8)
         q.scales_col = torch.empty(scale_shape(C, R, flags), **u8)
-        q.alpha_col = torch.empty(1, dtype=torch.float32, device=device)
+        q.alpha_col = torch.empty(max(C, 1) if vec else 1, dtype=torch.float32, device=device)
     q.amax = torch.zeros(2, dtype=torch.float32, device=device)
     return q
 
@@ -172,6 +174,26 @@ def nvfp4_gemm(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch
     st = L.nvfp4_gemm(_p(A), _p(sA), _p(alphaA), _p(B), _p(sB), _p(alphaB), M, N, K, _p(D), out_dtype,
                       D.stride(0), None, 0, _stream())
     _check(st, "nvfp4_gemm")
+    return D
+
+
+def nvfp4_gemm_vector_scales(A: torch.Tensor, sA: torch.Tensor, alphaA: torch.Tensor, B: torch.Tensor,
+                             sB: torch.Tensor, alphaB: torch.Tensor, out_dtype: int = NVFP4_OUT_DTYPE_BF16,
+                             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """nvfp4_gemm for operands quantized with NVFP4_VECTOR_SCALES: alphaA
+    holds one tensor scale per row of A ([M]), alphaB one per row of B ([N])."""
+    M, K2 = A.shape
+    N = B.shape[0]
+    K = 2 * K2
+    _need(alphaA, M, torch.float32, "alphaA", A.device)
+    _need(alphaB, N, torch.float32, "alphaB", A.device)
+    dt = torch.bfloat16 if out_dtype == NVFP4_OUT_DTYPE_BF16 else torch.float32
+    if out is not None:
+        _need_matrix(out, M, N, dt, "out", A.device)
+    D = out if out is not None else torch.empty((M, N), dtype=dt, device=A.device)
+    st = L.nvfp4_gemm_vector_scales(_p(A), _p(sA), _p(alphaA), _p(B), _p(sB), _p(alphaB), M, N, K, _p(D),
+                                    out_dtype, D.stride(0), None, 0, _stream())
+    _check(st, "nvfp4_gemm_vector_scales")
     return D
 
 

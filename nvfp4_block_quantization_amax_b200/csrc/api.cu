@@ -10,7 +10,7 @@
 namespace {
 
 constexpr uint32_t kQuantFlags = NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_BLOCK2D | NVFP4_SINGLE_PASS | NVFP4_HEADROOM |
-                                 NVFP4_ALPHA_PROVIDED | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_RHT;
+                                 NVFP4_ALPHA_PROVIDED | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_RHT | NVFP4_VECTOR_SCALES;
 constexpr uint32_t kDequantFlags = NVFP4_BLOCK2D | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_INVERSE_RHT | NVFP4_OUT_BF16;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -44,6 +44,8 @@ nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t 
   if (two_d && (mode == NVFP4_RHT_SR || mode == NVFP4_MS_EDEN || mode == NVFP4_RHT_SR_HW || (flags & NVFP4_RHT)))
     return NVFP4_ERR_ARG;
   if (stream_id >= 0x80000000u) return NVFP4_ERR_ARG;
+  if ((flags & NVFP4_VECTOR_SCALES) && (flags & (NVFP4_BLOCK2D | NVFP4_SINGLE_PASS | NVFP4_ALPHA_PROVIDED)))
+    return NVFP4_ERR_ARG;
   if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (C % 16) return NVFP4_ERR_SHAPE;
   if ((col || two_d) && R % 16) return NVFP4_ERR_SHAPE;
@@ -195,6 +197,26 @@ nvfp4_status_t nvfp4_gemm(const uint8_t* A, const uint8_t* sA, const float* alph
                         : nullptr;
   return launch_status(nvfp4::gemm_launch(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status_t nvfp4_gemm_vector_scales(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                                        const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K,
+                                        void* D, int out_dtype, int64_t ldd, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  if (out_dtype != NVFP4_OUT_DTYPE_BF16 && out_dtype != NVFP4_OUT_DTYPE_FP32) return NVFP4_ERR_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return NVFP4_ERR_SHAPE;
+  if (M % 256 || N % 256 || K % 128 || ldd < N) return NVFP4_ERR_SHAPE;
+  if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+  if (!A || !sA || !alphaA || !B || !sB || !alphaB || !D) return NVFP4_ERR_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(sA, 16) || !aligned(sB, 16) || !aligned(D, 16))
+    return NVFP4_ERR_ALIGN;
+  if (!aligned(alphaA, 4) || !aligned(alphaB, 4)) return NVFP4_ERR_ALIGN;
+  if ((ldd * (out_dtype == NVFP4_OUT_DTYPE_BF16 ? 2 : 4)) % 16) return NVFP4_ERR_ALIGN;
+  int32_t* status = (workspace && workspace_bytes >= sizeof(int32_t) && aligned(workspace, 4))
+                        ? static_cast<int32_t*>(workspace)
+                        : nullptr;
+  return launch_status(nvfp4::gemm_vs_launch(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status_t nvfp4_gemm_quantize(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,

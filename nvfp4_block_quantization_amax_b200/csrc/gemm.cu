@@ -607,7 +607,10 @@ __device__ __forceinline__ void pair_tile_coords(int tile, int m_tiles, int n_ti
   tile_n = local / rows;
 }
 
-template <int QMODE, bool MX = false>
+// VS (vector scales): alpha_a holds one tensor scale per row of A ([M]) and
+// alpha_b one per row of B ([N]); the epilogue scales D[m, n] by
+// alpha_a[m] then alpha_b[n].
+template <int QMODE, bool MX = false, bool VS = false>
 __global__ void __launch_bounds__(P_THREADS, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
@@ -772,7 +775,9 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     // quarter, each converting and storing half of the tile's columns.
     const int q = warp & 3, h = (warp - 2) >> 2;
     uint8_t* buf = sOut + (warp - 2) * 2048;
-    const float ab = MX ? 1.0f : __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));   // MXFP4: no tensor scales
+    // one factor for the whole product (MXFP4: no tensor scales), or per-row
+    // and per-column factors (VS)
+    const float ab = (MX || VS) ? 1.0f : __fmul_rn(__ldg(alpha_a), __ldg(alpha_b));
     const uint32_t acc_empty_leader = map_to_rank(smem_u32(acc_empty), 0);
     float eq_alpha = 0.0f, epi_amax = 0.0f;
     if constexpr (QMODE != kNoEpiQuant) eq_alpha = __ldg(eq.alpha);
@@ -785,6 +790,12 @@ __global__ void __launch_bounds__(P_THREADS, 1)
       const int row0 = tile_m * 256 + 128 * static_cast<int>(rank) + 32 * q;
       const int col0 = tile_n * 256 + 128 * h;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + 128 * h;
+      // VS: D = RN(RN(acc * alpha_a[m]) * alpha_b[n])
+      const float am = VS ? __ldg(alpha_a + row0 + lane) : 1.0f;
+      auto scale = [&](uint32_t acc_bits, int col) -> float {
+        if constexpr (VS) return __fmul_rn(__fmul_rn(__uint_as_float(acc_bits), am), __ldg(alpha_b + col0 + col));
+        return __fmul_rn(__uint_as_float(acc_bits), ab);
+      };
       if (!out_fp32) {
         // two rounds of 64 columns: load, wait, convert to packed bf16; the
         // accumulator is handed back once the whole row is in registers
@@ -798,8 +809,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), ab),
-                                                            __fmul_rn(__uint_as_float(r[2 * j + 1]), ab));
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale(r[2 * j], c + 2 * j), scale(r[2 * j + 1], c + 2 * j + 1));
             packed[c / 2 + j] = *reinterpret_cast<const uint32_t*>(&b2);
           }
         }
@@ -878,10 +888,10 @@ __global__ void __launch_bounds__(P_THREADS, 1)
 #pragma unroll
               for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
-                    make_uint4(__float_as_uint(__fmul_rn(__uint_as_float(r[4 * j]), ab)),
-                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 1]), ab)),
-                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 2]), ab)),
-                               __float_as_uint(__fmul_rn(__uint_as_float(r[4 * j + 3]), ab)));
+                    make_uint4(__float_as_uint(scale(r[4 * j], c + 4 * j)),
+                               __float_as_uint(scale(r[4 * j + 1], c + 4 * j + 1)),
+                               __float_as_uint(scale(r[4 * j + 2], c + 4 * j + 2)),
+                               __float_as_uint(scale(r[4 * j + 3], c + 4 * j + 3)));
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -999,7 +1009,7 @@ bool make_sf_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, bo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int QMODE, bool MX = false>
+template <int QMODE, bool MX = false, bool VS = false>
 cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B, const uint8_t* sB,
                         const float* alphaB, int64_t M, int64_t N, int64_t K, void* D, int out_dtype, int64_t ldd,
                         int32_t* status, const EpiQuant& eq, cudaStream_t st) {
@@ -1015,7 +1025,7 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QMODE, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(nvfp4_gemm_pair_kernel<QMODE, MX, VS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PairCfg<MX>::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -1045,7 +1055,7 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   const int64_t m_tiles = M / 256, n_tiles = N / 256;
   int64_t gm = (int64_t(64) << 20) / panel - n_tiles;
   gm = gm < 1 ? 1 : (gm > m_tiles ? m_tiles : gm);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE, MX>, ma, mb, md, msa, msb, alphaA, alphaB,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE, MX, VS>, ma, mb, md, msa, msb, alphaA, alphaB,
                                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
                                      static_cast<int>(fp32), status, eq, static_cast<int>(gm));
   note_launch();
@@ -1063,6 +1073,14 @@ cudaError_t gemm_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA
   }
   if (N % 256 == 0) return launch<256>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
   return launch<128>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status, st);
+}
+
+cudaError_t gemm_vs_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                           const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
+                           int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st) {
+  const EpiQuant none{nullptr, nullptr, nullptr, nullptr, 0, 1};
+  return launch_pair<kNoEpiQuant, false, true>(A, sA, alphaA, B, sB, alphaB, M, N, K, D, out_dtype, ldd, status,
+                                               none, st);
 }
 
 cudaError_t mx_gemm_launch(const uint8_t* A, const uint8_t* sA, const uint8_t* B, const uint8_t* sB, int64_t M,

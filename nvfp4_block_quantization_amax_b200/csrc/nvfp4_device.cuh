@@ -490,15 +490,39 @@ __device__ __forceinline__ void e4m3x2_ceil(float a, float b, uint32_t& ba, uint
   if (bb < 0x7Eu && e4m3_value(bb) < b) ++bb;
 }
 
-// Per-block scale context of one tensor scale: the table, and the Eq. 2
-// denominators RN(alpha * 6) and RN(alpha * 4).
-struct ScaleCtx {
+// Scale contexts of the block encoders.  A context gives, for the two
+// lane-paired blocks (x: block a, y: block b), their tensor scales alpha2,
+// the Eq. 2 denominators RN(alpha * 6) and RN(alpha * 4), and the entry
+// {s, rinv} of a scale byte.
+// TabScales: one tensor scale for both blocks, entries from the CTA's table.
+struct TabScales {
   const float2* tab;
   float alpha, den6, den4;
+  __device__ __forceinline__ float2 alpha2() const { return make_float2(alpha, alpha); }
+  __device__ __forceinline__ float2 d6() const { return make_float2(den6, den6); }
+  __device__ __forceinline__ float2 d4() const { return make_float2(den4, den4); }
+  __device__ __forceinline__ float2 ent_a(uint32_t b) const { return tab[b]; }
+  __device__ __forceinline__ float2 ent_b(uint32_t b) const { return tab[b]; }
 };
 
-__device__ __forceinline__ ScaleCtx make_scale_ctx(const float2* tab, float alpha) {
-  return ScaleCtx{tab, alpha, __fmul_rn(alpha, 6.0f), __fmul_rn(alpha, 4.0f)};
+__device__ __forceinline__ TabScales make_scale_ctx(const float2* tab, float alpha) {
+  return TabScales{tab, alpha, __fmul_rn(alpha, 6.0f), __fmul_rn(alpha, 4.0f)};
+}
+
+// VecScales: a tensor scale per block (one per row or column of the tensor);
+// entries are computed per block.
+struct VecScales {
+  float2 alpha, den6, den4;
+  __device__ __forceinline__ float2 alpha2() const { return alpha; }
+  __device__ __forceinline__ float2 d6() const { return den6; }
+  __device__ __forceinline__ float2 d4() const { return den4; }
+  __device__ __forceinline__ float2 ent_a(uint32_t b) const { return scale_entry(alpha.x, b); }
+  __device__ __forceinline__ float2 ent_b(uint32_t b) const { return scale_entry(alpha.y, b); }
+};
+
+__device__ __forceinline__ VecScales make_vec_scales(float alpha_a, float alpha_b) {
+  return VecScales{make_float2(alpha_a, alpha_b), make_float2(__fmul_rn(alpha_a, 6.0f), __fmul_rn(alpha_b, 6.0f)),
+                   make_float2(__fmul_rn(alpha_a, 4.0f), __fmul_rn(alpha_b, 4.0f))};
 }
 
 // Eq. 2's quotient amax_b / den (0 when den is 0).
@@ -536,21 +560,23 @@ __device__ __forceinline__ float2 sq_error_tab(const float2* v, float2 s2, const
 // Round-to-nearest block quantization of two lane-paired blocks from the
 // table (Four Over Six §2.1 Eq. 2-3; with FOUR_SIX the better of the M = 6
 // and M = 4 candidates by squared error, ties to M = 6, §1 Table 1).
-template <bool FOUR_SIX>
-__device__ __forceinline__ void quantize_pair_tab(const float2* v, const ScaleCtx& c, Packed16& pa, Packed16& pb,
+template <bool FOUR_SIX, class S>
+__device__ __forceinline__ void quantize_pair_tab(const float2* v, const S& c, Packed16& pa, Packed16& pb,
                                                   uint32_t& sba, uint32_t& sbb) {
   float ma, mb;
   max_abs16x2(v, ma, mb);
-  const uint32_t s6 = e4m3x2_rne(scale_quot(ma, c.den6), scale_quot(mb, c.den6));
+  const float2 d6 = c.d6();
+  const uint32_t s6 = e4m3x2_rne(scale_quot(ma, d6.x), scale_quot(mb, d6.y));
   const uint32_t a6 = s6 & 0xFFu, b6 = s6 >> 8;
-  const float2 ta6 = c.tab[a6], tb6 = c.tab[b6];
+  const float2 ta6 = c.ent_a(a6), tb6 = c.ent_b(b6);
   encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
   sba = a6;
   sbb = b6;
   if constexpr (FOUR_SIX) {
-    const uint32_t s4 = e4m3x2_rne(scale_quot(ma, c.den4), scale_quot(mb, c.den4));
+    const float2 d4 = c.d4();
+    const uint32_t s4 = e4m3x2_rne(scale_quot(ma, d4.x), scale_quot(mb, d4.y));
     const uint32_t a4 = s4 & 0xFFu, b4 = s4 >> 8;
-    const float2 ta4 = c.tab[a4], tb4 = c.tab[b4];
+    const float2 ta4 = c.ent_a(a4), tb4 = c.ent_b(b4);
     Packed16 pa4, pb4;
     encode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4);
     const float2 e6 = sq_error_tab(v, make_float2(ta6.x, tb6.x), pa, pb);

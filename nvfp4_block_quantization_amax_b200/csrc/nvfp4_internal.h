@@ -18,6 +18,7 @@ constexpr uint32_t kColwise = NVFP4_COLWISE;
 constexpr uint32_t kBlock2D = NVFP4_BLOCK2D;
 constexpr uint32_t kSinglePass = NVFP4_SINGLE_PASS;
 constexpr uint32_t kHeadroom = NVFP4_HEADROOM;
+constexpr uint32_t kVectorScales = NVFP4_VECTOR_SCALES;
 constexpr uint32_t kAlphaProvided = NVFP4_ALPHA_PROVIDED;
 constexpr uint32_t kGemmScaleLayout = NVFP4_GEMM_SCALE_LAYOUT;
 constexpr uint32_t kRht = NVFP4_RHT;
@@ -70,6 +71,12 @@ cudaError_t gemm_quantize_launch(const uint8_t* A, const uint8_t* sA, const floa
                                  const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
                                  int64_t ldd, int mode, bool gemm_layout, const float* alpha_out, uint8_t* codes,
                                  uint8_t* scales, float* amax_out, int32_t* status, cudaStream_t st);
+
+// NVFP4 GEMM with one tensor scale per operand row: alphaA [M], alphaB [N]
+// (the CTA-pair kernel; M % 256 == 0, N % 256 == 0, K % 128 == 0).
+cudaError_t gemm_vs_launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, const uint8_t* B,
+                           const uint8_t* sB, const float* alphaB, int64_t M, int64_t N, int64_t K, void* D,
+                           int out_dtype, int64_t ldd, int32_t* status, cudaStream_t st);
 
 // MXFP4 GEMM (gemm.cu, the CTA-pair kernel with UE8M0 block-32 scales):
 // D = sum_k (qA 2^eA)(qB 2^eB), scales in the GEMM layout with one 512-byte

@@ -52,7 +52,16 @@ struct QuantArgs {
   int64_t tiles_r, tiles_c;       // tile grid (tile kernels)
   FastDiv tiles_c_div;            // divides a tile index by tiles_c
   FastDiv chunks_row;             // C / 8: 16-byte chunks per row (plain amax)
+  uint32_t* vmax_r;               // NVFP4_VECTOR_SCALES: per-row maxima [R] (float bits)
+  uint32_t* vmax_c;               // and per-column maxima [C]
 };
+
+// Tensor scale of one vector from its maximum (Eq. 1 per vector; the
+// headroom form with NVFP4_HEADROOM).
+__device__ __forceinline__ float vector_alpha(const QuantArgs& a, const uint32_t* vmax, int64_t i) {
+  const float den = (a.flags & kHeadroom) ? 1792.0f : 2688.0f;
+  return __fdiv_rn(__uint_as_float(__ldcg(vmax + i)), den);
+}
 
 constexpr uint32_t kNonFinite = 0xFFFFFFFFu;   // partial marker: a NaN / Inf was read
 
@@ -281,8 +290,8 @@ __device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t wo
 // have_words: MS-EDEN only - wa / wb already hold the blocks' scale-SR words.
 // c: the tensor scale's table (s and 1 / s per scale byte) and the Eq. 2
 // denominators.
-template <int MODE>
-__device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c, const PhiloxKeys& K, uint32_t c2,
+template <int MODE, class S>
+__device__ __forceinline__ void quantize_pair(const float2* v, const S& c, const PhiloxKeys& K, uint32_t c2,
                                               uint64_t blka, uint64_t blkb, Packed16& pa, Packed16& pb,
                                               uint32_t& sba, uint32_t& sbb, bool have_words = false,
                                               uint32_t wa = 0u, uint32_t wb = 0u) {
@@ -293,8 +302,9 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c
     // scale sum(r^2) / (alpha sum(r q)), stochastically rounded to E4M3
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    const uint32_t prov = e4m3x2_rne(scale_quot(ma, c.den6), scale_quot(mb, c.den6));
-    const float2 ta = c.tab[prov & 0xFFu], tb = c.tab[prov >> 8];
+    const float2 d6 = c.d6();
+    const uint32_t prov = e4m3x2_rne(scale_quot(ma, d6.x), scale_quot(mb, d6.y));
+    const float2 ta = c.ent_a(prov & 0xFFu), tb = c.ent_b(prov >> 8);
     encode_x2(v, make_float2(ta.y, tb.y), pa, pb);
     float2 q[16], rr[16], rq[16];
     decode16x2(pa, pb, q);
@@ -304,7 +314,7 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c
       rq[i] = mul2(v[i], q[i]);
     }
     const float2 num = sum16x2(rr);
-    const float2 den = mul2(make_float2(c.alpha, c.alpha), sum16x2(rq));
+    const float2 den = mul2(c.alpha2(), sum16x2(rq));
     if (!have_words) {
       const uint64_t ua = blka >> 2, ub = blkb >> 2;
       const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagScaleSR);
@@ -322,8 +332,9 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c
     // handed over last element first so that nibble j holds element 4g + j.
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    e4m3x2_ceil(scale_quot(ma, c.den6), scale_quot(mb, c.den6), sba, sbb);
-    const float2 r2 = make_float2(c.tab[sba].y, c.tab[sbb].y);
+    const float2 d6 = c.d6();
+    e4m3x2_ceil(scale_quot(ma, d6.x), scale_quot(mb, d6.y), sba, sbb);
+    const float2 r2 = make_float2(c.ent_a(sba).y, c.ent_b(sbb).y);
     const uint4 da = philox(K, static_cast<uint32_t>(blka), static_cast<uint32_t>(blka >> 32), c2, kTagValueSRHw);
     const uint4 db = philox(K, static_cast<uint32_t>(blkb), static_cast<uint32_t>(blkb >> 32), c2, kTagValueSRHw);
     const uint32_t wa4[4] = {da.x, da.y, da.z, da.w}, wb4[4] = {db.x, db.y, db.z, db.w};
@@ -346,8 +357,9 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c
   } else {  // RHT + stochastic rounding of the values
     float ma, mb;
     max_abs16x2(v, ma, mb);
-    e4m3x2_ceil(scale_quot(ma, c.den6), scale_quot(mb, c.den6), sba, sbb);
-    const float2 r2 = make_float2(c.tab[sba].y, c.tab[sbb].y);
+    const float2 d6 = c.d6();
+    e4m3x2_ceil(scale_quot(ma, d6.x), scale_quot(mb, d6.y), sba, sbb);
+    const float2 r2 = make_float2(c.ent_a(sba).y, c.ent_b(sbb).y);
     // element i uses half (i & 1) of word (i >> 1) & 3 of draw i >> 3 (unit 2 blk + draw)
     uint32_t wa8[8], wb8[8];
 #pragma unroll
@@ -381,14 +393,16 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const ScaleCtx& c
 // share a row) and quantizes them lane-paired.  Both lie in MS-EDEN draw
 // unit k / 2, so one draw serves the pair.
 // ===========================================================================
-template <int MODE, bool ROT, int NT>
+template <int MODE, bool ROT, int NT, bool VEC = false>
 __device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint32_t* red,
                                                 float2* tab) {
-  float alpha, alpha_unused;
-  resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red, cta);
-  build_scale_tab<NT>(tab, alpha);
-  __syncthreads();
-  const ScaleCtx sc = make_scale_ctx(tab, alpha);
+  float alpha = 0.0f, alpha_unused;
+  if constexpr (!VEC) {
+    resolve_alpha<NT>(a, true, false, true, false, alpha, alpha_unused, red, cta);
+    build_scale_tab<NT>(tab, alpha);
+    __syncthreads();
+  }
+  const TabScales sc = make_scale_ctx(tab, alpha);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -442,7 +456,17 @@ __device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta
     if constexpr (ROT) rht16x2_presigned(v);
     Packed16 qa, qb;
     uint32_t sa, sb;
-    quantize_pair<MODE>(v, sc, K, c2, ka, kb, qa, qb, sa, sb);
+    if constexpr (VEC) {
+      // one tensor scale per row; the thread holding a row's first block
+      // publishes it
+      const float aa = vector_alpha(a, a.vmax_r, ra);
+      const float ab = (rb == ra) ? aa : vector_alpha(a, a.vmax_r, rb);
+      quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2, ka, kb, qa, qb, sa, sb);
+      if (cba == 0) a.alpha_row[ra] = aa;
+      if (vb && cbb == 0) a.alpha_row[rb] = ab;
+    } else {
+      quantize_pair<MODE>(v, sc, K, c2, ka, kb, qa, qb, sa, sb);
+    }
     uint8_t* ca = a.codes_row + static_cast<int64_t>(ra) * (a.C / 2) + 8 * cba;
     if (vb && rb == ra && (reinterpret_cast<uintptr_t>(ca) & 15u) == 0) {
       *reinterpret_cast<uint4*>(ca) = make_uint4(qa.lo, qa.hi, qb.lo, qb.hi);
@@ -489,19 +513,21 @@ struct TileStaging {
   float2 tab_c[kScaleTab];           // the same for the column orientation
 };
 
-template <int MODE, bool ROT, bool ROW, bool COL>
+template <int MODE, bool ROT, bool ROW, bool COL, bool VEC = false>
 __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint8_t* ring,
                                                    TileStaging& stg) {
   auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);
   auto& colcodes = stg.colcodes;
   auto& colscale = stg.colscale;
   uint32_t* red = stg.red;
-  float alpha_r, alpha_c;
-  resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
-  if constexpr (ROW) build_scale_tab<TNT>(stg.tab_r, alpha_r);
-  if constexpr (COL) build_scale_tab<TNT>(stg.tab_c, alpha_c);
-  __syncthreads();
-  const ScaleCtx scr = make_scale_ctx(stg.tab_r, alpha_r), scc = make_scale_ctx(stg.tab_c, alpha_c);
+  float alpha_r = 0.0f, alpha_c = 0.0f;
+  if constexpr (!VEC) {
+    resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
+    if constexpr (ROW) build_scale_tab<TNT>(stg.tab_r, alpha_r);
+    if constexpr (COL) build_scale_tab<TNT>(stg.tab_c, alpha_c);
+    __syncthreads();
+  }
+  const TabScales scr = make_scale_ctx(stg.tab_r, alpha_r), scc = make_scale_ctx(stg.tab_c, alpha_c);
   const PhiloxKeys K = philox_keys(a.seed);
   SignMasks sm;
   if constexpr (ROT) {
@@ -613,7 +639,19 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         const uint64_t blkb = static_cast<uint64_t>(grb) * (C / 16) + gcb;
         Packed16 pa, pb;
         uint32_t sa, sb;
-        quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+        if constexpr (VEC) {
+          // tensor scales of rows gra and grb; the tiles of the first tile
+          // column publish them
+          const float aa = va ? vector_alpha(a, a.vmax_r, gra) : 0.0f;
+          const float ab = vb ? vector_alpha(a, a.vmax_r, grb) : aa;
+          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+          if (tc == 0 && cb == 0) {
+            if (va) a.alpha_row[gra] = aa;
+            if (vb) a.alpha_row[grb] = ab;
+          }
+        } else {
+          quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+        }
         if (va) {
           *reinterpret_cast<uint2*>(a.codes_row + gra * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
           if (a.scales_row)
@@ -645,8 +683,19 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
         Packed16 qa, qb;
         uint32_t sa, sb;
-        quantize_pair<MODE>(v, scc, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
-                            static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+        if constexpr (VEC) {
+          // tensor scales of columns gc, gc + 1; the first tile row publishes them
+          const float aa = vector_alpha(a, a.vmax_c, gc), ab = vector_alpha(a, a.vmax_c, gc + 1);
+          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
+                              static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+          if (tr == 0 && rb == 0) {
+            a.alpha_col[gc] = aa;
+            a.alpha_col[gc + 1] = ab;
+          }
+        } else {
+          quantize_pair<MODE>(v, scc, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
+                              static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+        }
         *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
         colscale[2 * cp][rb] = static_cast<uint8_t>(sa);
@@ -700,7 +749,7 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
   resolve_alpha<TNT>(a, true, COL, ROW, COL, alpha, alpha_c, red, cta);
   build_scale_tab<TNT>(stg.tab_r, alpha);
   __syncthreads();
-  const ScaleCtx sc = make_scale_ctx(stg.tab_r, alpha);
+  const TabScales sc = make_scale_ctx(stg.tab_r, alpha);
   const bool gemm = (a.flags & kGemmScaleLayout) != 0;
   const bool check = (a.flags & kAlphaProvided) != 0;
   const int t = threadIdx.x;
@@ -896,18 +945,143 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
   amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, part_r, part_c, blockIdx.x, gridDim.x, ring, red);
 }
 
-template <int MODE, bool ROT, int NT>
+template <int MODE, bool ROT, int NT, bool VEC>
 __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
   __shared__ uint32_t red[NT / 32];
   __shared__ float2 tab[kScaleTab];
-  quant_rows_body<MODE, ROT, NT>(a, blockIdx.x, gridDim.x, red, tab);
+  quant_rows_body<MODE, ROT, NT, VEC>(a, blockIdx.x, gridDim.x, red, tab);
 }
 
-template <int MODE, bool ROT, bool ROW, bool COL>
+template <int MODE, bool ROT, bool ROW, bool COL, bool VEC>
 __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
-  quant_tile_1d_body<MODE, ROT, ROW, COL>(a, blockIdx.x, gridDim.x, tile_ring, stg);
+  quant_tile_1d_body<MODE, ROT, ROW, COL, VEC>(a, blockIdx.x, gridDim.x, tile_ring, stg);
+}
+
+// Per-vector maxima for NVFP4_VECTOR_SCALES: max |x| (over rotated 16-blocks
+// with ROT, scaled by the transform's 1/4 at the end, which commutes with
+// the maximum) of every row (ROW) and / or column (COL), folded into
+// vmax_r / vmax_c (float bits, zeroed by the launcher) with atomicMax; the
+// largest of each orientation goes to amax_out[0] / [1] the same way.  An
+// Inf or NaN sets NVFP4_ERR_NONFINITE.
+template <bool ROW, bool COL, bool ROT>
+__global__ void __launch_bounds__(TNT) amax_vec_kernel(const QuantArgs a) {
+  __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
+  __shared__ uint32_t colmax[TC];
+  __shared__ uint32_t red[TNT / 32];
+  auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);
+  SignMasks sm;
+  if constexpr (ROT) {
+    sm = sign_masks(sign_bits(philox_keys(a.seed)));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sm.m[i] = 0u;
+  }
+  const float post = ROT ? 0.25f : 1.0f;
+  const int t = threadIdx.x;
+  const int64_t R = a.R, C = a.C;
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  const uint32_t ncta = gridDim.x;
+  uint32_t hin = 0, trmax = 0, tcmax = 0;
+  if (COL && t < TC) colmax[t] = 0u;
+  uint32_t tile = blockIdx.x;
+  int buf = 0;
+  if (tile < ntiles) load_tile_async(tiles[0], a.x, R, C, a.ld, a.tiles_c_div, tile);
+  for (; tile < ntiles; tile += ncta, buf ^= 1) {
+    const uint32_t next = tile + ncta;
+    if (next < ntiles) {
+      load_tile_async(tiles[buf ^ 1], a.x, R, C, a.ld, a.tiles_c_div, next);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint4 (*sv)[TC / 8] = tiles[buf];
+    int64_t tr, tc;
+    tile_coords(tile, a.tiles_c_div, tr, tc);
+    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
+    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
+    if constexpr (ROW) {
+      // blocks (row, cb) and (row + 32, cb); the 8 lanes of a row then combine
+      const int row = t >> 3, cb = t & 7;
+      const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
+      const uint4 a0 = sv[row][tile_chunk(row, 2 * cb)], a1 = sv[row][tile_chunk(row, 2 * cb + 1)];
+      const uint4 b0 = sv[row + 32][tile_chunk(row + 32, 2 * cb)];
+      const uint4 b1 = sv[row + 32][tile_chunk(row + 32, 2 * cb + 1)];
+      const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (va) hin = __vmaxu2(hin, wa[i] & 0x7FFF7FFFu);
+        if (vb) hin = __vmaxu2(hin, wb[i] & 0x7FFF7FFFu);
+      }
+      float2 v[16];
+      unpack16x2_signed(a0, a1, b0, b1, sm, v);
+      if constexpr (ROT) hadamard16x2(v);
+      float ma, mb;
+      max_abs16x2(v, ma, mb);
+      if (!va) ma = 0.0f;
+      if (!vb) mb = 0.0f;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        ma = fmaxf(ma, __shfl_xor_sync(0xFFFFFFFFu, ma, o));
+        mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+      }
+      const uint32_t ba = __float_as_uint(__fmul_rn(ma, post)), bb = __float_as_uint(__fmul_rn(mb, post));
+      if (cb == 0) {
+        if (row < rows) atomicMax(a.vmax_r + r0 + row, ba);
+        if (row + 32 < rows) atomicMax(a.vmax_r + r0 + row + 32, bb);
+      }
+      trmax = max(trmax, max(ba, bb));
+    }
+    if constexpr (COL) {
+      // columns (2 cp, 2 cp + 1) of row block rb, combined in shared memory
+      const int cp = t & 63, rb = t >> 6;
+      if (16 * rb < rows && 2 * cp < cols) {
+        const uint32_t* base = reinterpret_cast<const uint32_t*>(&sv[16 * rb][0]);
+        const int wofs = tile_word(16 * rb, cp);
+        float2 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = base[i * (TC / 2) + wofs];
+          if constexpr (!ROW) hin = __vmaxu2(hin, w & 0x7FFF7FFFu);
+          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+        }
+        if constexpr (ROT) hadamard16x2(v);
+        float mx = 0.0f, my = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          mx = fmaxf(mx, fabsf(v[i].x));
+          my = fmaxf(my, fabsf(v[i].y));
+        }
+        atomicMax(&colmax[2 * cp], __float_as_uint(__fmul_rn(mx, post)));
+        atomicMax(&colmax[2 * cp + 1], __float_as_uint(__fmul_rn(my, post)));
+      }
+      __syncthreads();
+      if (t < TC) {
+        const uint32_t m = colmax[t];
+        if (t < cols) {
+          atomicMax(a.vmax_c + c0 + t, m);
+          tcmax = max(tcmax, m);
+        }
+        colmax[t] = 0u;
+      }
+    }
+    __syncthreads();   // buf and colmax are reused
+  }
+  if (max(hin & 0xFFFFu, hin >> 16) >= 0x7F80u && a.status) *a.status = kStatusNonFinite;
+  if (a.amax_out) {
+    if constexpr (ROW) {
+      const uint32_t m = block_max_u32<TNT>(trmax, red);
+      if (t == 0) atomicMax(reinterpret_cast<uint32_t*>(a.amax_out), m);
+    }
+    if constexpr (COL) {
+      const uint32_t m = block_max_u32<TNT>(tcmax, red);
+      if (t == 0) atomicMax(reinterpret_cast<uint32_t*>(a.amax_out) + 1, m);
+    }
+  }
 }
 
 template <int MODE, bool ROW, bool COL>
@@ -986,9 +1160,9 @@ __global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, 
   if constexpr (TWO_D) {
     quant_tile_2d_body<MODE, ROW, COL>(a, cta, ncta, tile_ring, stg);
   } else if constexpr (ROW && !COL) {
-    quant_rows_body<MODE, ROT, TNT>(a, cta, ncta, stg.red, stg.tab_r);
+    quant_rows_body<MODE, ROT, TNT, false>(a, cta, ncta, stg.red, stg.tab_r);
   } else {
-    quant_tile_1d_body<MODE, ROT, ROW, COL>(a, cta, ncta, tile_ring, stg);
+    quant_tile_1d_body<MODE, ROT, ROW, COL, false>(a, cta, ncta, tile_ring, stg);
   }
 }
 
@@ -1013,17 +1187,23 @@ int amax_partial_count() { return 4 * 148; }
 
 // Workspace: the amax partials of both orientations, then (single pass) the
 // grid barrier's counter in its own 16-byte slot.
-size_t quant_workspace_bytes(int64_t, int64_t, uint32_t flags) {
+// NVFP4_VECTOR_SCALES: R maxima (rounded up to 4) then C maxima.
+size_t vec_workspace_bytes(int64_t R, int64_t C) {
+  return static_cast<size_t>(((R + 3) & ~int64_t(3)) + ((C + 3) & ~int64_t(3))) * sizeof(uint32_t);
+}
+
+size_t quant_workspace_bytes(int64_t R, int64_t C, uint32_t flags) {
+  if (flags & kVectorScales) return vec_workspace_bytes(R, C);
   if (flags & kAlphaProvided) return 0;
   const size_t partials = static_cast<size_t>(2 * amax_partial_count()) * sizeof(uint32_t);
   return (flags & kSinglePass) ? partials + 16 : partials;
 }
 
-template <int MODE, bool ROT>
+template <int MODE, bool ROT, bool VEC = false>
 static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
   const uint32_t pairs = (static_cast<uint32_t>(a.R) * a.nb_row.d + 1) / 2;
   const int blocks = static_cast<int>(std::min<int64_t>((pairs + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
-  quant_rows_kernel<MODE, ROT, 256><<<std::max(blocks, 1), 256, 0, st>>>(a);
+  quant_rows_kernel<MODE, ROT, 256, VEC><<<std::max(blocks, 1), 256, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1048,31 +1228,66 @@ static cudaError_t launch_tile_2d(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int MODE, bool ROT, bool ROW, bool COL>
+template <int MODE, bool ROT, bool ROW, bool COL, bool VEC = false>
 static cudaError_t launch_tile_1d(const QuantArgs& a, cudaStream_t st) {
   constexpr size_t smem = static_cast<size_t>(kTileStages) * kTileBytes;
+  auto fn = quant_tile_1d_kernel<MODE, ROT, ROW, COL, VEC>;
   static int per_sm = 0;
   if (per_sm == 0) {
     int n = 0;
-    cudaFuncSetAttribute(quant_tile_1d_kernel<MODE, ROT, ROW, COL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_tile_1d_kernel<MODE, ROT, ROW, COL>, TNT, smem) !=
-            cudaSuccess || n <= 0)
-      n = 1;
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, TNT, smem) != cudaSuccess || n <= 0) n = 1;
     per_sm = n;
   }
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
-  quant_tile_1d_kernel<MODE, ROT, ROW, COL><<<std::max(blocks, 1), TNT, smem, st>>>(a);
+  fn<<<std::max(blocks, 1), TNT, smem, st>>>(a);
   note_launch();
   return cudaGetLastError();
 }
 
-template <int MODE, bool ROT>
+template <int MODE, bool ROT, bool VEC = false>
 static cudaError_t dispatch_1d(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
-  if (row && !col) return launch_rows<MODE, ROT>(a, st);
-  if (row && col) return launch_tile_1d<MODE, ROT, true, true>(a, st);
-  return launch_tile_1d<MODE, ROT, false, true>(a, st);
+  if (row && !col) return launch_rows<MODE, ROT, VEC>(a, st);
+  if (row && col) return launch_tile_1d<MODE, ROT, true, true, VEC>(a, st);
+  return launch_tile_1d<MODE, ROT, false, true, VEC>(a, st);
+}
+
+// NVFP4_VECTOR_SCALES: clear the vector maxima (and amax_out), fold them in,
+// then quantize with one tensor scale per row / column.
+template <bool ROT>
+static cudaError_t launch_amax_vec(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
+  const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 4));
+  if (row && col) amax_vec_kernel<true, true, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  else if (row) amax_vec_kernel<true, false, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  else amax_vec_kernel<false, true, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+static cudaError_t quantize_vector_scales(QuantArgs a, int mode, bool row, bool col, bool rot, cudaStream_t st) {
+  a.vmax_r = const_cast<uint32_t*>(a.partials);
+  a.vmax_c = a.vmax_r + ((a.R + 3) & ~int64_t(3));
+  cudaError_t e = cudaMemsetAsync(a.vmax_r, 0, vec_workspace_bytes(a.R, a.C), st);
+  if (e == cudaSuccess && a.amax_out) e = cudaMemsetAsync(a.amax_out, 0, 2 * sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  e = rot ? launch_amax_vec<true>(a, row, col, st) : launch_amax_vec<false>(a, row, col, st);
+  if (e != cudaSuccess) return e;
+  switch (mode) {
+    case kModeRTN:
+      return rot ? dispatch_1d<kModeRTN, true, true>(a, row, col, st)
+                 : dispatch_1d<kModeRTN, false, true>(a, row, col, st);
+    case kModeFourSix:
+      return rot ? dispatch_1d<kModeFourSix, true, true>(a, row, col, st)
+                 : dispatch_1d<kModeFourSix, false, true>(a, row, col, st);
+    case kModeRhtSR:
+      return dispatch_1d<kModeRhtSR, true, true>(a, row, col, st);
+    case kModeRhtSRHw:
+      return dispatch_1d<kModeRhtSRHw, true, true>(a, row, col, st);
+    default:
+      return dispatch_1d<kModeMsEden, true, true>(a, row, col, st);
+  }
 }
 
 template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
@@ -1168,6 +1383,7 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || mode == kModeRhtSRHw || (flags & kRht)) && !two_d;
   if (rot) a.partials_col = a.partials + a.npart;
   if (R == 0 || C == 0) return cudaSuccess;
+  if (flags & kVectorScales) return quantize_vector_scales(a, mode, row, col, rot, st);
 
   if ((flags & kSinglePass) && !(flags & kAlphaProvided)) {
     if (two_d) {
