@@ -130,6 +130,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait for the first phase of `bar` (used only after an abort, where
+// the abort flag is already up).
+__device__ __forceinline__ void mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kTimeoutNs) {
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
@@ -316,7 +324,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* acc_empty = bars + 2 * STAGES + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  uint64_t* drain = bars + 2 * STAGES + 2;   // tensor-op drain after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -332,6 +341,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(acc_empty), 4);  // one arrival per epilogue warp
+    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -383,9 +393,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // the CTA exits (each wait again bounded).
         for (int i = (it > STAGES ? it - STAGES : 0); i < it; ++i) {
           const uint32_t bar = smem_u32(&full[i % STAGES]), ph = (i / STAGES) & 1;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
-          }
+          mbar_wait_bounded(bar, ph);
         }
       }
     }
@@ -426,6 +434,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         umma_commit(smem_u32(&empty[s]));
         if (kt == kstages - 1) umma_commit(smem_u32(acc_full));
+      }
+      if (*abort_flag) {
+        // a wait gave up: the copies and MMAs already issued may still run;
+        // let them finish (bounded) before TMEM is freed
+        umma_commit(smem_u32(drain));
+        mbar_wait_bounded(smem_u32(drain), 0);
       }
     }
   } else {
@@ -628,7 +642,8 @@ __global__ void __launch_bounds__(P_THREADS, 1)
   uint64_t* empty = bars + PC::STAGES;
   uint64_t* acc_full = bars + 2 * PC::STAGES;
   uint64_t* acc_empty = bars + 2 * PC::STAGES + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PC::STAGES + 2);
+  uint64_t* drain = bars + 2 * PC::STAGES + 2;   // tensor-op drain after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PC::STAGES + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -648,6 +663,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(acc_empty), 2 * P_EPI_WARPS);  // every epilogue warp of both CTAs
+    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -699,9 +715,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         // before the CTA exits (each wait again bounded)
         for (int i = (it > PC::STAGES ? it - PC::STAGES : 0); i < it; ++i) {
           const uint32_t bar = smem_u32(&full[i % PC::STAGES]), ph = (i / PC::STAGES) & 1;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(bar, ph) && globaltimer() - t0 < kTimeoutNs) {
-          }
+          mbar_wait_bounded(bar, ph);
         }
       }
     }
@@ -776,6 +790,13 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           full_ph ^= 1;
         }
         if (++kt == kstages) kt = 0;
+      }
+      if (*abort_flag) {
+        // a wait gave up: the copies and MMAs already issued (into both
+        // CTAs' TMEM) may still run; let them finish (bounded) before the
+        // pair frees TMEM
+        umma_commit_pair(smem_u32(drain));
+        mbar_wait_bounded(smem_u32(drain), 0);
       }
     }
   } else {
