@@ -80,10 +80,11 @@ __device__ __forceinline__ void unpack8(const uint4 u, float* v) {
 // ---------------------------------------------------------------------------
 // E4M3 block scales (OCP E4M3FN, non-negative): 127 finite codes, max 448.
 // ---------------------------------------------------------------------------
+// Normal codes (b >= 8): exponent and mantissa bits move up as one field and
+// the exponent is rebiased from 7 to 127 (+120 << 3 before the shift).
 __device__ __forceinline__ float e4m3_value(uint32_t b) {
-  const uint32_t e = b >> 3, m = b & 7u;
-  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
-           : __fmul_rn(static_cast<float>(m), 0.001953125f);  // m * 2^-9, exact
+  return (b >= 8u) ? __uint_as_float((b + (120u << 3)) << 20)
+                   : __fmul_rn(static_cast<float>(b), 0.001953125f);  // b * 2^-9, exact
 }
 
 // Round to nearest even, saturating at 448 (hardware conversion; PTX
@@ -102,18 +103,23 @@ __device__ __forceinline__ uint32_t e4m3_ceil(float v) {
 }
 
 // Stochastic rounding to E4M3 with a 24-bit uniform: up iff u24 < f * 2^24,
-// f the position of v between its neighbours.  v >= 0.
+// f the position of v between its lower neighbour lo and the next value.
+// v >= 0 (saturating at 448).
+//   E4M3 normal range [2^-6, 448): the FP32 value truncated to 3 mantissa
+//   bits is lo, so lo's code is the top bits of v, (exponent << 3 | m3)
+//   rebiased from 127 to 7, and f * 2^24 is the 20 dropped mantissa bits
+//   times 16 (an exact integer).
+//   Subnormal range [0, 2^-6): the grid step is 2^-9, so with t = 512 v
+//   (exact) lo = floor(t) and f = t - lo, both exact.
 __device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t u24) {
   if (!(v < 448.0f)) return 0x7Eu;
-  uint32_t lo = e4m3_rne(v);
-  if (e4m3_value(lo) > v) --lo;
-  const float vlo = e4m3_value(lo);
-  if (vlo == v) return lo;
-  // gap is a normal power of two, so 1/gap is exact (exponent 254 - e) and
-  // the product below equals the exact quotient (v - vlo) / gap.
-  const float gap = __fsub_rn(e4m3_value(lo + 1), vlo);
-  const float f = __fmul_rn(__fsub_rn(v, vlo), __uint_as_float(0x7F000000u - __float_as_uint(gap)));
-  return (static_cast<float>(u24) < __fmul_rn(f, 16777216.0f)) ? lo + 1 : lo;
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t lo_n = (b >> 20) - (120u << 3);
+  const uint32_t up_n = (u24 < ((b & 0xFFFFFu) << 4)) ? 1u : 0u;
+  const float t = __fmul_rn(v, 512.0f);
+  const float fl = floorf(t);
+  const uint32_t up_s = (static_cast<float>(u24) < __fmul_rn(__fsub_rn(t, fl), 16777216.0f)) ? 1u : 0u;
+  return (v >= 0.015625f) ? lo_n + up_n : static_cast<uint32_t>(fl) + up_s;
 }
 
 // ---------------------------------------------------------------------------
@@ -292,11 +298,22 @@ __device__ __forceinline__ uint32_t e2m1x2_rne(float y_lo, float y_hi) {
   return r;
 }
 
+// Eight values -> one word: four conversions whose bytes are packed inside
+// the asm block (a vector mov that builds the word from four .b8 registers;
+// only the opposite direction, splitting a word into .b8 registers, is
+// avoided, see e2m1x2_to_f16x2).
 __device__ __forceinline__ uint32_t e2m1x8_rne(float y0, float y1, float y2, float y3, float y4, float y5,
                                                float y6, float y7) {
-  const uint32_t b01 = __byte_perm(e2m1x2_rne(y0, y1), e2m1x2_rne(y2, y3), 0x7740u);   // [b0, b1, 0, 0]
-  const uint32_t b23 = __byte_perm(e2m1x2_rne(y4, y5), e2m1x2_rne(y6, y7), 0x7740u);   // [b2, b3, 0, 0]
-  return __byte_perm(b01, b23, 0x5410u);
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+  return r;
 }
 
 // Each byte is taken out of the word in C++ and handed to the convert through
@@ -397,26 +414,36 @@ __device__ __forceinline__ float2 sq_error_x2(const float2* v, float alpha, uint
   return sum16x2(e);
 }
 
-// Block maxima of |v| for two lane-paired blocks.  Tree-shaped (depth 4) so
-// the two chains of dependent max operations stay
-// short; max is exact, so the order does not matter.
+// max(|a|, |b|, |c|) and max(a, b, c) in one instruction each (the sm_100
+// three-input max.f32; the absolute values are operand modifiers).
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float r;
+  asm("{\n\t.reg .f32 x, y, z;\n\t"
+      "abs.f32 x, %1;\n\tabs.f32 y, %2;\n\tabs.f32 z, %3;\n\t"
+      "max.f32 %0, x, y, z;\n\t}"
+      : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Block maxima of |v| for two lane-paired blocks: 16 values in three levels
+// of three-input maxima (5 + 2 + 1 instructions per block); max is exact, so
+// the order does not matter.
 __device__ __forceinline__ void max_abs16x2(const float2* v, float& ma, float& mb) {
-  float a[8], b[8];
+  float a[6], b[6];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    a[i] = fmaxf(fabsf(v[i].x), fabsf(v[i + 8].x));
-    b[i] = fmaxf(fabsf(v[i].y), fabsf(v[i + 8].y));
+  for (int i = 0; i < 5; ++i) {
+    a[i] = max3_abs(v[3 * i].x, v[3 * i + 1].x, v[3 * i + 2].x);
+    b[i] = max3_abs(v[3 * i].y, v[3 * i + 1].y, v[3 * i + 2].y);
   }
-#pragma unroll
-  for (int w = 4; w > 0; w >>= 1) {
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      a[i] = fmaxf(a[i], a[i + w]);
-      b[i] = fmaxf(b[i], b[i + w]);
-    }
-  }
-  ma = a[0];
-  mb = b[0];
+  a[5] = max3_abs(a[3], a[4], v[15].x);
+  b[5] = max3_abs(b[3], b[4], v[15].y);
+  ma = fmaxf(max3(a[0], a[1], a[2]), a[5]);
+  mb = fmaxf(max3(b[0], b[1], b[2]), b[5]);
 }
 
 // Round-to-nearest block quantization of two lane-paired blocks (Four Over
