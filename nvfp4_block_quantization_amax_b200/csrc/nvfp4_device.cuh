@@ -269,6 +269,29 @@ __device__ __forceinline__ void rht16x2_presigned(float2* v) {
 __device__ __forceinline__ int64_t gemm_scale_offset(int64_t m, int64_t j, int64_t kblocks) {
   return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3);
 }
+// The same in 32-bit arithmetic, for scale arrays below 4 GB.
+__device__ __forceinline__ uint32_t gemm_scale_offset32(uint32_t m, uint32_t j, uint32_t kblocks) {
+  return ((m >> 7) * (kblocks >> 2) + (j >> 2)) * 512u + (m & 31u) * 16u + ((m >> 5) & 3u) * 4u + (j & 3u);
+}
+
+// The layout split over a 64 x 128 tile (r0 = 64 tr, c0 = 128 tc).  Row
+// orientation (kb = C / 16 blocks per row), the block of tile row r < 32 and
+// tile block column cb: tile part + thread part, and row r + 32 is 4 bytes
+// further on; column orientation (kb = R / 16), tile column c: the four
+// scale bytes of row blocks 0..3 are the 4-byte word at tile part + thread
+// part.
+__device__ __forceinline__ int64_t gemm_scale_tile_row(int64_t tr, int64_t tc, int64_t kb) {
+  return ((tr >> 1) * (kb >> 2) + 2 * tc) * 512 + (tr & 1) * 8;
+}
+__device__ __forceinline__ uint32_t gemm_scale_thread_row(int r, int cb) {
+  return static_cast<uint32_t>((cb >> 2) * 512 + (cb & 3) + (r & 31) * 16);
+}
+__device__ __forceinline__ int64_t gemm_scale_tile_col(int64_t tr, int64_t tc, int64_t kb) {
+  return (tc * (kb >> 2) + tr) * 512;
+}
+__device__ __forceinline__ uint32_t gemm_scale_thread_col(int c) {
+  return static_cast<uint32_t>((c & 31) * 16 + ((c >> 5) & 3) * 4);
+}
 
 struct Packed16 {
   uint32_t lo, hi;

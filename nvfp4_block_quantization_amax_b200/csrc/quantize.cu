@@ -273,7 +273,7 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   }
 }
 
-constexpr int kColPitch = 40;   // bytes per staged column of codes (32 used)
+constexpr int kColPitch = 48;   // bytes per staged column of codes (32 used; rows 16-byte aligned)
 
 // ---------------------------------------------------------------------------
 // One mode's quantization of two lane-paired 16-element blocks (x: block a,
@@ -477,9 +477,9 @@ __device__ __forceinline__ void quant_rows_body(const QuantArgs& a, uint32_t cta
             make_uint2(qb.lo, qb.hi);
     }
     if (a.scales_row) {
-      a.scales_row[gemm ? gemm_scale_offset(ra, cba, nb) : static_cast<int64_t>(ka)] = static_cast<uint8_t>(sa);
-      if (vb)
-        a.scales_row[gemm ? gemm_scale_offset(rb, cbb, nb) : static_cast<int64_t>(kb)] = static_cast<uint8_t>(sb);
+      // R * C / 16 < 2^32 blocks here, so 32-bit offsets suffice
+      a.scales_row[gemm ? gemm_scale_offset32(ra, cba, nb) : ka] = static_cast<uint8_t>(sa);
+      if (vb) a.scales_row[gemm ? gemm_scale_offset32(rb, cbb, nb) : kb] = static_cast<uint8_t>(sb);
     }
   }
 }
@@ -550,6 +550,9 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   // transpose hands the words out.
   const bool share = MODE == kModeMsEden && (!ROW || C % 64 == 0) && (!COL || R % 64 == 0);
   const int lane = t & 31, j4 = t & 3;
+  // whole tiles write columns as 16-byte code pieces and 4-byte scale words
+  // (R % 64 == 0 keeps both aligned)
+  const bool col_words = R % 64 == 0 && (reinterpret_cast<uintptr_t>(a.scales_col) & 3u) == 0;
 
   // prologue: the first kTileStages - 1 tiles (an empty copy group when a
   // tile does not exist keeps the group count in step)
@@ -652,17 +655,16 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         } else {
           quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
         }
-        if (va) {
-          *reinterpret_cast<uint2*>(a.codes_row + gra * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
-          if (a.scales_row)
-            a.scales_row[gemm ? gemm_scale_offset(gra, gcb, C / 16) : static_cast<int64_t>(blka)] =
-                static_cast<uint8_t>(sa);
-        }
-        if (vb) {
-          *reinterpret_cast<uint2*>(a.codes_row + grb * (C / 2) + 8 * gcb) = make_uint2(pb.lo, pb.hi);
-          if (a.scales_row)
-            a.scales_row[gemm ? gemm_scale_offset(grb, gcb, C / 16) : static_cast<int64_t>(blkb)] =
-                static_cast<uint8_t>(sb);
+        // row gra's 8 code bytes, row grb's 32 rows further on; the scale
+        // offsets split into a tile part and a thread part
+        uint8_t* crow = a.codes_row + gra * (C / 2) + 8 * gcb;
+        if (va) *reinterpret_cast<uint2*>(crow) = make_uint2(pa.lo, pa.hi);
+        if (vb) *reinterpret_cast<uint2*>(crow + 32 * (C / 2)) = make_uint2(pb.lo, pb.hi);
+        if (a.scales_row) {
+          uint8_t* srow = a.scales_row + (gemm ? gemm_scale_tile_row(tr, tc, C / 16) + gemm_scale_thread_row(row, cb)
+                                               : static_cast<int64_t>(blka));
+          if (va) srow[0] = static_cast<uint8_t>(sa);
+          if (vb) srow[gemm ? 4 : 32 * (C / 16)] = static_cast<uint8_t>(sb);
         }
       }
     }
@@ -702,24 +704,37 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         colscale[2 * cp + 1][rb] = static_cast<uint8_t>(sb);
       }
       __syncthreads();
-      {
+      if (rows == TR && cols == TC && col_words) {
+        // whole tile: thread t copies 16 code bytes of column t / 2 and
+        // threads 0..127 the 4-byte word of column t's four scales
         const int c = t >> 1, h = t & 1;
-        const int nbytes = rows / 2;
-        if (c < cols && 16 * h < nbytes) {
-          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
-          const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
-          reinterpret_cast<uint2*>(dst)[0] = src[0];
-          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+        *reinterpret_cast<uint4*>(a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h) =
+            *reinterpret_cast<const uint4*>(&colcodes[c][16 * h]);
+        if (a.scales_col && t < TC) {
+          const int64_t off = gemm ? gemm_scale_tile_col(tr, tc, R / 16) + gemm_scale_thread_col(t)
+                                   : (c0 + t) * (R / 16) + r0 / 16;
+          *reinterpret_cast<uint32_t*>(a.scales_col + off) = *reinterpret_cast<const uint32_t*>(&colscale[t][0]);
         }
-      }
-      if (a.scales_col) {
-        const int c = t >> 1;
-        if (c < cols) {
-          for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
-            const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
-            const uint8_t sbyte = colscale[c][rb2];
-            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
-            else a.scales_col[gc * (R / 16) + grb] = sbyte;
+      } else {
+        {
+          const int c = t >> 1, h = t & 1;
+          const int nbytes = rows / 2;
+          if (c < cols && 16 * h < nbytes) {
+            uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
+            const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
+            reinterpret_cast<uint2*>(dst)[0] = src[0];
+            if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+          }
+        }
+        if (a.scales_col) {
+          const int c = t >> 1;
+          if (c < cols) {
+            for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
+              const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
+              const uint8_t sbyte = colscale[c][rb2];
+              if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
+              else a.scales_col[gc * (R / 16) + grb] = sbyte;
+            }
           }
         }
       }
@@ -755,6 +770,8 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
   const int t = threadIdx.x;
   const int64_t R = a.R, C = a.C;
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
+  // whole tiles write columns as 16-byte code pieces and 4-byte scale words
+  const bool col_words = R % 64 == 0 && (reinterpret_cast<uintptr_t>(a.scales_col) & 3u) == 0;
 
   uint32_t tile = cta;
 #pragma unroll
@@ -853,26 +870,23 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
         }
       }
       const int64_t gcb = c0 / 16 + cbb;
-      if (va) {
-        const int64_t grow = r0 + rowa;
-        if (lr == 0) scale2d[rb][cbb] = static_cast<uint8_t>(sa);
-        if constexpr (ROW) {
-          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(pa.lo, pa.hi);
-          if (a.scales_row) {
-            if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sa);
-            else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sa);
-          }
-        }
+      if (lr == 0) {
+        if (va) scale2d[rb][cbb] = static_cast<uint8_t>(sa);
+        if (vb) scale2d[rb + 2][cbb] = static_cast<uint8_t>(sb);
       }
-      if (vb) {
-        const int64_t grow = r0 + rowb;
-        if (lr == 0) scale2d[rb + 2][cbb] = static_cast<uint8_t>(sb);
-        if constexpr (ROW) {
-          *reinterpret_cast<uint2*>(a.codes_row + grow * (C / 2) + 8 * gcb) = make_uint2(pb.lo, pb.hi);
-          if (a.scales_row) {
-            if (gemm) a.scales_row[gemm_scale_offset(grow, gcb, C / 16)] = static_cast<uint8_t>(sb);
-            else if (lr == 0) a.scales_row[(grow / 16) * (C / 16) + gcb] = static_cast<uint8_t>(sb);
-          }
+      if constexpr (ROW) {
+        // row rowa's 8 code bytes, row rowb = rowa + 32 further on; in the
+        // GEMM layout every row of a 2D block carries its scale (rowa < 32:
+        // tile part + thread part, rowb 4 bytes further on), in the plain
+        // layout one byte per 16 x 16 block
+        uint8_t* crow = a.codes_row + (r0 + rowa) * (C / 2) + 8 * gcb;
+        if (va) *reinterpret_cast<uint2*>(crow) = make_uint2(pa.lo, pa.hi);
+        if (vb) *reinterpret_cast<uint2*>(crow + 32 * (C / 2)) = make_uint2(pb.lo, pb.hi);
+        if (a.scales_row && (gemm || lr == 0)) {
+          uint8_t* srow = a.scales_row + (gemm ? gemm_scale_tile_row(tr, tc, C / 16) + gemm_scale_thread_row(rowa, cbb)
+                                               : (r0 / 16 + rb) * (C / 16) + gcb);
+          if (va) srow[0] = static_cast<uint8_t>(sa);
+          if (vb) srow[gemm ? 4 : 2 * (C / 16)] = static_cast<uint8_t>(sb);
         }
       }
     }
@@ -897,24 +911,44 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
       }
       __syncthreads();
-      {
+      if (rows == TR && cols == TC && col_words) {
+        // whole tile: 16 code bytes per thread; in the GEMM layout threads
+        // 0..127 write column t's four scale bytes as one word
         const int c = t >> 1, h = t & 1;
-        const int nbytes = rows / 2;
-        if (c < cols && 16 * h < nbytes) {
-          uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
-          const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
-          reinterpret_cast<uint2*>(dst)[0] = src[0];
-          if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+        *reinterpret_cast<uint4*>(a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h) =
+            *reinterpret_cast<const uint4*>(&colcodes[c][16 * h]);
+        if (a.scales_col && t < TC) {
+          const int cb = t >> 4;
+          if (gemm) {
+            const uint32_t w = static_cast<uint32_t>(scale2d[0][cb]) | (static_cast<uint32_t>(scale2d[1][cb]) << 8) |
+                               (static_cast<uint32_t>(scale2d[2][cb]) << 16) |
+                               (static_cast<uint32_t>(scale2d[3][cb]) << 24);
+            *reinterpret_cast<uint32_t*>(a.scales_col + gemm_scale_tile_col(tr, tc, R / 16) +
+                                         gemm_scale_thread_col(t)) = w;
+          } else if ((t & 15) == 0) {
+            for (int rb2 = 0; rb2 < 4; ++rb2) a.scales_col[((c0 + t) / 16) * (R / 16) + r0 / 16 + rb2] = scale2d[rb2][cb];
+          }
         }
-      }
-      if (a.scales_col) {
-        const int c = t >> 1;
-        if (c < cols) {
-          for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
-            const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
-            const uint8_t sbyte = scale2d[rb2][c >> 4];
-            if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
-            else if ((c & 15) == 0) a.scales_col[(gc / 16) * (R / 16) + grb] = sbyte;
+      } else {
+        {
+          const int c = t >> 1, h = t & 1;
+          const int nbytes = rows / 2;
+          if (c < cols && 16 * h < nbytes) {
+            uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
+            const uint2* src = reinterpret_cast<const uint2*>(&colcodes[c][16 * h]);
+            reinterpret_cast<uint2*>(dst)[0] = src[0];
+            if (16 * h + 8 < nbytes) reinterpret_cast<uint2*>(dst)[1] = src[1];
+          }
+        }
+        if (a.scales_col) {
+          const int c = t >> 1;
+          if (c < cols) {
+            for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
+              const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
+              const uint8_t sbyte = scale2d[rb2][c >> 4];
+              if (gemm) a.scales_col[gemm_scale_offset(gc, grb, R / 16)] = sbyte;
+              else if ((c & 15) == 0) a.scales_col[(gc / 16) * (R / 16) + grb] = sbyte;
+            }
           }
         }
       }
