@@ -230,12 +230,8 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
       float2 v[16];
       unpack16x2_signed(a0, a1, b0, b1, sm, v);
       hadamard16x2(v);
-      float ma = 0.0f, mb = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        ma = fmaxf(ma, fabsf(v[i].x));
-        mb = fmaxf(mb, fabsf(v[i].y));
-      }
+      float ma, mb;
+      max_abs16x2(v, ma, mb);
       if (va) mr = fmaxf(mr, ma);
       if (vb) mr = fmaxf(mr, mb);
     }
@@ -253,8 +249,9 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
           v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
         }
         hadamard16x2(v);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mc = fmaxf(mc, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        float ma, mb;
+        max_abs16x2(v, ma, mb);
+        mc = max3(mc, ma, mb);
       }
     }
     __syncthreads();   // buf is refilled two iterations from now
