@@ -8,6 +8,7 @@
 #include <cstdint>
 
 #include "nvfp4_device.cuh"
+#include "launch.cuh"
 #include "nvfp4_internal.h"
 
 namespace nvfp4 {
@@ -18,6 +19,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
                                                       const float* __restrict__ alpha_p,
                                                       int64_t R, int64_t C, FastDiv nb,
                                                       uint64_t seed, void* __restrict__ y) {
+  pdl_entry();
   const float alpha = __ldg(alpha_p);
   uint32_t signs = 0;
   if constexpr (INV) signs = philox(philox_keys(seed), 0u, 0u, 0u, kTagSigns).x & 0xFFFFu;
@@ -64,9 +66,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 template <bool INV, bool BF16>
 static void launch_dq(int sc, dim3 g, const uint8_t* codes, const uint8_t* scales, const float* alpha,
                       int64_t R, int64_t C, FastDiv nb, uint64_t seed, void* y, cudaStream_t st) {
-  if (sc == 0) { dequant_kernel<INV, BF16, 0><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
-  else if (sc == 1) { dequant_kernel<INV, BF16, 1><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
-  else { dequant_kernel<INV, BF16, 2><<<g, 256, 0, st>>>(codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
+  if (sc == 0) { launch_k(dequant_kernel<INV, BF16, 0>, dim3(g), dim3(256), 0, st, 1u, codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
+  else if (sc == 1) { launch_k(dequant_kernel<INV, BF16, 1>, dim3(g), dim3(256), 0, st, 1u, codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
+  else { launch_k(dequant_kernel<INV, BF16, 2>, dim3(g), dim3(256), 0, st, 1u, codes, scales, alpha, R, C, nb, seed, y); note_launch(); }
 }
 
 cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* scales, const float* alpha,

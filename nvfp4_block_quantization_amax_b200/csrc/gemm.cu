@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "nvfp4_device.cuh"
+#include "launch.cuh"
 #include "nvfp4_internal.h"
 
 namespace nvfp4 {
@@ -310,6 +311,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tmap_d, const uint8_t* __restrict__ sfa,
                       const uint8_t* __restrict__ sfb, const float* __restrict__ alpha_a,
                       const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status) {
+  pdl_entry();
   using G = Cfg<BN>;
   constexpr int STAGES = G::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -629,6 +631,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
                            const __grid_constant__ CUtensorMap tmap_sfb, const float* __restrict__ alpha_a,
                            const float* __restrict__ alpha_b, int M, int N, int K, int out_fp32, int32_t* status,
                            const EpiQuant eq, int group_m) {
+  pdl_entry();
   using PC = PairCfg<MX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1018,7 +1021,7 @@ cudaError_t launch(const uint8_t* A, const uint8_t* sA, const float* alphaA, con
   }
   const int64_t tiles = (M / BM) * (N / BN);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());  // persistent: one CTA per SM
-  nvfp4_gemm_kernel<BN><<<grid, NUM_THREADS, G::SMEM, st>>>(ma, mb, md, sA, sB, alphaA, alphaB, static_cast<int>(M),
+  launch_k(nvfp4_gemm_kernel<BN>, dim3(grid), dim3(NUM_THREADS), G::SMEM, st, 1u, ma, mb, md, sA, sB, alphaA, alphaB, static_cast<int>(M),
                                                             static_cast<int>(N), static_cast<int>(K), fp32, status);
   note_launch();
   return cudaGetLastError();
@@ -1067,18 +1070,6 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   }
   const int64_t tiles = (M / 256) * (N / 256);
   const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;  // persistent: one pair per TPC
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(P_THREADS);
-  cfg.dynamicSmemBytes = PairCfg<MX>::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   // M-tiles per raster group: as many as keep the group's A panels plus all
   // of B within about 64 MB of L2 (operand bytes per 256-row panel: K / 2
   // codes + K / 16 scales)
@@ -1086,9 +1077,10 @@ cudaError_t launch_pair(const uint8_t* A, const uint8_t* sA, const float* alphaA
   const int64_t m_tiles = M / 256, n_tiles = N / 256;
   int64_t gm = (int64_t(64) << 20) / panel - n_tiles;
   gm = gm < 1 ? 1 : (gm > m_tiles ? m_tiles : gm);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_pair_kernel<QMODE, MX, VS>, ma, mb, md, msa, msb, alphaA, alphaB,
-                                     static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                                     static_cast<int>(fp32), status, eq, static_cast<int>(gm));
+  cudaError_t e = launch_k(nvfp4_gemm_pair_kernel<QMODE, MX, VS>, dim3(static_cast<unsigned>(2 * pairs)),
+                           dim3(P_THREADS), PairCfg<MX>::SMEM, st, 2u, ma, mb, md, msa, msb, alphaA, alphaB,
+                           static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(fp32),
+                           status, eq, static_cast<int>(gm));
   note_launch();
   return e;
 }

@@ -22,6 +22,7 @@
 #include <cstdint>
 
 #include "nvfp4_device.cuh"
+#include "launch.cuh"
 #include "nvfp4_internal.h"
 #include "tile.cuh"
 
@@ -84,6 +85,7 @@ __device__ __forceinline__ uint4 mx_encode(float2* v, uint32_t& scale) {
 
 template <bool ROT, bool ROW, bool COL>
 __global__ void __launch_bounds__(TNT, 3) mx_tile_kernel(const MxArgs a) {
+  pdl_entry();
   extern __shared__ __align__(128) uint8_t mx_ring[];
   auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(mx_ring);
   SignMasks sm;
@@ -167,6 +169,7 @@ template <bool INV, bool BF16>
 __global__ void __launch_bounds__(256) mx_dequant_kernel(const uint8_t* __restrict__ codes,
                                                          const uint8_t* __restrict__ scales, int64_t R, int64_t C,
                                                          uint64_t seed, void* __restrict__ y) {
+  pdl_entry();
   const int64_t halves = R * (C / 16);
   const uint32_t signs = INV ? (philox(philox_keys(seed), 0u, 0u, 0u, kTagSigns).x & 0xFFFFu) : 0u;
   for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < halves;
@@ -205,7 +208,7 @@ static cudaError_t launch_mx_tile(const MxArgs& a, cudaStream_t st) {
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, TNT, smem) != cudaSuccess || n <= 0) n = 1;
   const int grid = static_cast<int>(std::min<int64_t>(a.ntiles, static_cast<int64_t>(sm_count()) * n));
-  fn<<<grid, TNT, smem, st>>>(a);
+  launch_k(fn, dim3(grid), dim3(TNT), smem, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -247,10 +250,10 @@ cudaError_t mx_dequantize_launch(const uint8_t* codes, const uint8_t* scales, in
   if (halves == 0) return cudaSuccess;
   const int blocks = static_cast<int>(std::min<int64_t>((halves + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
   const bool inv = flags & kInverseRht, bf16 = flags & kOutBf16;
-  if (inv && bf16) mx_dequant_kernel<true, true><<<blocks, 256, 0, st>>>(codes, scales, R, C, seed, y);
-  else if (inv) mx_dequant_kernel<true, false><<<blocks, 256, 0, st>>>(codes, scales, R, C, seed, y);
-  else if (bf16) mx_dequant_kernel<false, true><<<blocks, 256, 0, st>>>(codes, scales, R, C, seed, y);
-  else mx_dequant_kernel<false, false><<<blocks, 256, 0, st>>>(codes, scales, R, C, seed, y);
+  if (inv && bf16) launch_k(mx_dequant_kernel<true, true>, dim3(blocks), dim3(256), 0, st, 1u, codes, scales, R, C, seed, y);
+  else if (inv) launch_k(mx_dequant_kernel<true, false>, dim3(blocks), dim3(256), 0, st, 1u, codes, scales, R, C, seed, y);
+  else if (bf16) launch_k(mx_dequant_kernel<false, true>, dim3(blocks), dim3(256), 0, st, 1u, codes, scales, R, C, seed, y);
+  else launch_k(mx_dequant_kernel<false, false>, dim3(blocks), dim3(256), 0, st, 1u, codes, scales, R, C, seed, y);
   note_launch();
   return cudaGetLastError();
 }

@@ -22,6 +22,7 @@
 #include <cstdlib>
 
 #include "nvfp4_device.cuh"
+#include "launch.cuh"
 #include "nvfp4_internal.h"
 #include "tile.cuh"
 
@@ -962,6 +963,7 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
 template <int NT>
 __global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t ld,
                                                         FastDiv cpr, uint32_t* __restrict__ partial) {
+  pdl_entry();
   __shared__ uint32_t red[NT / 32];
   amax_plain_body<NT>(x, R, ld, cpr, partial, blockIdx.x, gridDim.x, red);
 }
@@ -971,6 +973,7 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
                                                         int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
                                                         uint32_t* __restrict__ part_r,
                                                         uint32_t* __restrict__ part_c) {
+  pdl_entry();
   __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
   __shared__ uint32_t red[TNT / 32];
   amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, part_r, part_c, blockIdx.x, gridDim.x, ring, red);
@@ -978,6 +981,7 @@ __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restri
 
 template <int MODE, bool ROT, int NT, bool VEC>
 __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
+  pdl_entry();
   __shared__ uint32_t red[NT / 32];
   __shared__ float2 tab[kScaleTab];
   quant_rows_body<MODE, ROT, NT, VEC>(a, blockIdx.x, gridDim.x, red, tab);
@@ -985,6 +989,7 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
 
 template <int MODE, bool ROT, bool ROW, bool COL, bool VEC>
 __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
+  pdl_entry();
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
   quant_tile_1d_body<MODE, ROT, ROW, COL, VEC>(a, blockIdx.x, gridDim.x, tile_ring, stg);
@@ -998,6 +1003,7 @@ __global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d
 // Inf or NaN sets NVFP4_ERR_NONFINITE.
 template <bool ROW, bool COL, bool ROT>
 __global__ void __launch_bounds__(TNT) amax_vec_kernel(const QuantArgs a) {
+  pdl_entry();
   __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
   __shared__ uint32_t colmax[TC];
   __shared__ uint32_t red[TNT / 32];
@@ -1117,6 +1123,7 @@ __global__ void __launch_bounds__(TNT) amax_vec_kernel(const QuantArgs a) {
 
 template <int MODE, bool ROW, bool COL>
 __global__ void __launch_bounds__(TNT, 3) quant_tile_2d_kernel(const QuantArgs a) {
+  pdl_entry();
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
   quant_tile_2d_body<MODE, ROW, COL>(a, blockIdx.x, gridDim.x, tile_ring, stg);
@@ -1173,6 +1180,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t n, uint
 template <int MODE, bool ROT, bool ROW, bool COL, bool TWO_D>
 __global__ void __launch_bounds__(TNT, 2) single_pass_kernel(const QuantArgs a, uint32_t* counter,
                                                               uint64_t timeout_ns) {
+  pdl_entry();
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
   __shared__ uint32_t pass_ok;
@@ -1234,7 +1242,7 @@ template <int MODE, bool ROT, bool VEC = false>
 static cudaError_t launch_rows(const QuantArgs& a, cudaStream_t st) {
   const uint32_t pairs = (static_cast<uint32_t>(a.R) * a.nb_row.d + 1) / 2;
   const int blocks = static_cast<int>(std::min<int64_t>((pairs + 255) / 256, static_cast<int64_t>(sm_count()) * 8));
-  quant_rows_kernel<MODE, ROT, 256, VEC><<<std::max(blocks, 1), 256, 0, st>>>(a);
+  launch_k(quant_rows_kernel<MODE, ROT, 256, VEC>, dim3(std::max(blocks, 1)), dim3(256), 0, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1254,7 +1262,7 @@ static cudaError_t launch_tile_2d(const QuantArgs& a, cudaStream_t st) {
   }
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
-  quant_tile_2d_kernel<MODE, ROW, COL><<<std::max(blocks, 1), TNT, smem, st>>>(a);
+  launch_k(quant_tile_2d_kernel<MODE, ROW, COL>, dim3(std::max(blocks, 1)), dim3(TNT), smem, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1272,7 +1280,7 @@ static cudaError_t launch_tile_1d(const QuantArgs& a, cudaStream_t st) {
   }
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
-  fn<<<std::max(blocks, 1), TNT, smem, st>>>(a);
+  launch_k(fn, dim3(std::max(blocks, 1)), dim3(TNT), smem, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1290,9 +1298,9 @@ template <bool ROT>
 static cudaError_t launch_amax_vec(const QuantArgs& a, bool row, bool col, cudaStream_t st) {
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * 4));
-  if (row && col) amax_vec_kernel<true, true, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
-  else if (row) amax_vec_kernel<true, false, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
-  else amax_vec_kernel<false, true, ROT><<<std::max(blocks, 1), TNT, 0, st>>>(a);
+  if (row && col) launch_k(amax_vec_kernel<true, true, ROT>, dim3(std::max(blocks, 1)), dim3(TNT), 0, st, 1u, a);
+  else if (row) launch_k(amax_vec_kernel<true, false, ROT>, dim3(std::max(blocks, 1)), dim3(TNT), 0, st, 1u, a);
+  else launch_k(amax_vec_kernel<false, true, ROT>, dim3(std::max(blocks, 1)), dim3(TNT), 0, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
@@ -1367,16 +1375,16 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   uint32_t* pr = const_cast<uint32_t*>(a.partials);
   uint32_t* pc = const_cast<uint32_t*>(a.partials_col);
   if (!rot) {
-    amax_plain_kernel<256><<<np, 256, 0, st>>>(a.x, a.R, a.ld, a.chunks_row, pr);
+    launch_k(amax_plain_kernel<256>, dim3(np), dim3(256), 0, st, 1u, a.x, a.R, a.ld, a.chunks_row, pr);
   } else {
     const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
     const FastDiv tcd = a.tiles_c_div;
     if (row && col)
-      amax_tile_kernel<true, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<true, true>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else if (row)
-      amax_tile_kernel<true, false><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<true, false>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else
-      amax_tile_kernel<false, true><<<np, TNT, 0, st>>>(a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<false, true>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
   }
   note_launch();
   return cudaGetLastError();
