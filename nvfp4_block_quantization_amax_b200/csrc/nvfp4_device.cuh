@@ -394,6 +394,54 @@ __device__ __forceinline__ void encode_rne_x2(const float2* v, float alpha, uint
   if (isinf(rb)) pb = sign_codes16<true>(v);
 }
 
+// Eight values -> one word of codes and their grid values: each converted
+// byte is decoded from its .b8 register in the same asm block
+// (cvt.rn.f16x2.e2m1x2, exact), so the word is never taken apart again.
+// h[k] holds the values of elements 2k, 2k + 1 as f16x2.
+__device__ __forceinline__ uint32_t e2m1x8_rne_dec(float y0, float y1, float y2, float y3, float y4, float y5,
+                                                   float y6, float y7, uint32_t* h) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %8, %7;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %10, %9;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %12, %11;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, t0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, t1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, t2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %4, t3;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+  return r;
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t h2) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t h2) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// Codes of two lane-paired blocks v * rinv (as encode_x2) and their grid
+// values q, lane-paired.
+__device__ __forceinline__ void encode_decode_x2(const float2* v, float2 rinv2, Packed16& pa, Packed16& pb,
+                                                 float2* q) {
+  float2 y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = mul2(v[i], rinv2);
+  uint32_t ha[8], hb[8];
+  pa.lo = e2m1x8_rne_dec(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x, ha);
+  pa.hi = e2m1x8_rne_dec(y[8].x, y[9].x, y[10].x, y[11].x, y[12].x, y[13].x, y[14].x, y[15].x, ha + 4);
+  pb.lo = e2m1x8_rne_dec(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y, hb);
+  pb.hi = e2m1x8_rne_dec(y[8].y, y[9].y, y[10].y, y[11].y, y[12].y, y[13].y, y[14].y, y[15].y, hb + 4);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    q[2 * k] = make_float2(f16_lo(ha[k]), f16_lo(hb[k]));
+    q[2 * k + 1] = make_float2(f16_hi(ha[k]), f16_hi(hb[k]));
+  }
+}
+
 // Grid values of two blocks' codes, lane-paired.
 __device__ __forceinline__ void decode16x2(const Packed16& pa, const Packed16& pb, float2* q) {
   float a[16], b[16];
@@ -607,6 +655,18 @@ __device__ __forceinline__ float2 sq_error_tab(const float2* v, float2 s2, const
   return sum16x2(e);
 }
 
+// Squared error of one encoding whose grid values q are known (the Four
+// Over Six criterion): sum of RN((v - RN(q s))^2), as sq_error_tab.
+__device__ __forceinline__ float2 sq_error_q(const float2* v, float2 s2, const float2* q) {
+  float2 e[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 d = sub2_exact(v[i], mul2(q[i], s2));
+    e[i] = mul2(d, d);
+  }
+  return sum16x2(e);
+}
+
 // Round-to-nearest block quantization of two lane-paired blocks from the
 // table (Four Over Six §2.1 Eq. 2-3; with FOUR_SIX the better of the M = 6
 // and M = 4 candidates by squared error, ties to M = 6, §1 Table 1).
@@ -619,18 +679,23 @@ __device__ __forceinline__ void quantize_pair_tab(const float2* v, const S& c, P
   const uint32_t s6 = e4m3x2_rne(scale_quot(ma, d6.x), scale_quot(mb, d6.y));
   const uint32_t a6 = s6 & 0xFFu, b6 = s6 >> 8;
   const float2 ta6 = c.ent_a(a6), tb6 = c.ent_b(b6);
-  encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
   sba = a6;
   sbb = b6;
-  if constexpr (FOUR_SIX) {
+  if constexpr (!FOUR_SIX) {
+    encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
+  } else {
+    // each candidate's grid values come out of its encoding and feed its
+    // error at once
+    float2 q[16];
+    encode_decode_x2(v, make_float2(ta6.y, tb6.y), pa, pb, q);
+    const float2 e6 = sq_error_q(v, make_float2(ta6.x, tb6.x), q);
     const float2 d4 = c.d4();
     const uint32_t s4 = e4m3x2_rne(scale_quot(ma, d4.x), scale_quot(mb, d4.y));
     const uint32_t a4 = s4 & 0xFFu, b4 = s4 >> 8;
     const float2 ta4 = c.ent_a(a4), tb4 = c.ent_b(b4);
     Packed16 pa4, pb4;
-    encode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4);
-    const float2 e6 = sq_error_tab(v, make_float2(ta6.x, tb6.x), pa, pb);
-    const float2 e4 = sq_error_tab(v, make_float2(ta4.x, tb4.x), pa4, pb4);
+    encode_decode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4, q);
+    const float2 e4 = sq_error_q(v, make_float2(ta4.x, tb4.x), q);
     if (e4.x < e6.x) {
       sba = a4;
       pa = pa4;

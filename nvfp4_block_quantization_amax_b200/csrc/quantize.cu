@@ -303,9 +303,8 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const S& c, const
     const float2 d6 = c.d6();
     const uint32_t prov = e4m3x2_rne(scale_quot(ma, d6.x), scale_quot(mb, d6.y));
     const float2 ta = c.ent_a(prov & 0xFFu), tb = c.ent_b(prov >> 8);
-    encode_x2(v, make_float2(ta.y, tb.y), pa, pb);
     float2 q[16], rr[16], rq[16];
-    decode16x2(pa, pb, q);
+    encode_decode_x2(v, make_float2(ta.y, tb.y), pa, pb, q);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       rr[i] = mul2(v[i], v[i]);
@@ -841,15 +840,18 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
       uint32_t sa = s6 & 0xFFu, sb = s6 >> 8;
       const float2 ta6 = sc.tab[sa], tb6 = sc.tab[sb];
       Packed16 pa, pb;
-      encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
+      if constexpr (MODE != kModeFourSix) encode_x2(v, make_float2(ta6.y, tb6.y), pa, pb);
       if constexpr (MODE == kModeFourSix) {
+        // each candidate's grid values come out of its encoding
+        float2 q[16];
+        encode_decode_x2(v, make_float2(ta6.y, tb6.y), pa, pb, q);
+        float2 e6 = sq_error_q(v, make_float2(ta6.x, tb6.x), q);
         const uint32_t s4 = e4m3x2_rne(scale_quot(ma, sc.den4), scale_quot(mb, sc.den4));
         const uint32_t sa4 = s4 & 0xFFu, sb4 = s4 >> 8;
         const float2 ta4 = sc.tab[sa4], tb4 = sc.tab[sb4];
         Packed16 pa4, pb4;
-        encode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4);
-        float2 e6 = sq_error_tab(v, make_float2(ta6.x, tb6.x), pa, pb);
-        float2 e4 = sq_error_tab(v, make_float2(ta4.x, tb4.x), pa4, pb4);
+        encode_decode_x2(v, make_float2(ta4.y, tb4.y), pa4, pb4, q);
+        float2 e4 = sq_error_q(v, make_float2(ta4.x, tb4.x), q);
         // block error = the half-warp's row errors summed in butterfly order
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) {
