@@ -297,6 +297,38 @@ def gemm_traffic_record():
     return g.get("dram_bytes_per_launch") if g.get("source_sha256_16") == h else None
 
 
+QUANT_SOURCES = ("quantize.cu", "nvfp4_device.cuh", "tile.cuh", "launch.cuh")
+
+
+def quantizer_issue_record():
+    """Per-kernel instruction counts of the step's quantizer launches from the
+    committed ncu summary, if it was taken on the current quantizer sources
+    (else None)."""
+    p = os.path.join(ROOT, "profiles", "quantizer_issue.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    csrc = os.path.join(ROOT, "nvfp4_block_quantization_amax_b200", "csrc")
+    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in QUANT_SOURCES)).hexdigest()[:16]
+    return d if d.get("source_sha256_16") == h else None
+
+
+def quantize_roofline(rec, quant_ms, sm_mhz, n_sm, hbm_gbs):
+    """The quantizer against its floors: per kernel the larger of its issue
+    time (warp instructions / (SMs x 4 schedulers x the sampled SM clock))
+    and its HBM time (algorithmic bytes / HBM peak), summed over the step's
+    kernels, against the step's measured quantizer time."""
+    rate = n_sm * 4 * sm_mhz * 1e6
+    issue = [k["warp_instructions"] / rate for k in rec["kernels"]]
+    mem = [k["algorithmic_bytes"] / (hbm_gbs * 1e9) for k in rec["kernels"]]
+    floor = sum(max(a, b) for a, b in zip(issue, mem))
+    return {"bound": "per kernel max(issue, hbm)", "floor_us": round(floor * 1e6, 1),
+            "achieved_us": round(quant_ms * 1e3, 1), "frac": floor / (quant_ms * 1e-3),
+            "issue_floor_us": round(sum(issue) * 1e6, 1), "hbm_floor_us": round(sum(mem) * 1e6, 1),
+            "sm_mhz": sm_mhz, "kernels": len(issue),
+            "instructions": "ncu smsp__inst_executed.sum per kernel, profiles/quantizer_issue.json"}
+
+
 class L2Flush:
     """Overwrites a 256 MiB buffer (twice L2) between timed calls so no
     timed call starts with its inputs in L2."""
@@ -548,6 +580,12 @@ def run_device(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    qrec = quantizer_issue_record()
+    if qrec is not None and clocks.get("sm_mhz"):
+        n_sm = torch.cuda.get_device_properties(device).multi_processor_count
+        result["quantize_roofline"] = quantize_roofline(qrec, quant_ms, clocks["sm_mhz"], n_sm, hbm)
+    else:
+        result["quantize_roofline"] = None
     del hx, hw, hdy, hy, hdx, hdw
     if not args.no_extras:
         result.update(run_extras(args, step, x, w, dy, device, hbm, fp4_peak))

@@ -85,3 +85,33 @@ def test_quantize_bytes_per_element():
     assert bench.quant_bytes_per_elem(bench.ROW | bench.COL) == 3.125
     assert bench.quant_bytes_per_elem(bench.ROW | bench.B2D) == 2 + 0.5 + 1 / 256
     assert bench.quant_bytes_per_elem(bench.ROW | bench.COL | bench.B2D) == 3 + 2 / 256
+
+
+def test_quantize_roofline_takes_the_larger_floor_per_kernel():
+    # kernel 1: 592e6 warp instructions at 1000 MHz on 148 SMs = 1000 us of
+    # issue against 1 us of HBM; kernel 2: 665e6 bytes at 6650 GB/s = 100 us
+    # of HBM against ~0 us of issue
+    rec = {"kernels": [{"warp_instructions": 592_000_000, "algorithmic_bytes": 6_650_000},
+                       {"warp_instructions": 1, "algorithmic_bytes": 665_000_000}]}
+    r = bench.quantize_roofline(rec, quant_ms=2.2, sm_mhz=1000.0, n_sm=148, hbm_gbs=6650.0)
+    assert r["floor_us"] == pytest.approx(1100.0, abs=0.2)
+    assert r["issue_floor_us"] == pytest.approx(1000.0, abs=0.2)
+    assert r["hbm_floor_us"] == pytest.approx(101.0, abs=0.2)
+    assert r["frac"] == pytest.approx(0.5, rel=1e-3)
+
+
+def test_quantizer_issue_record_checks_the_sources(tmp_path, monkeypatch):
+    import json
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "quantizer_issue.json").write_text(json.dumps({"source_sha256_16": "0" * 16, "kernels": []}))
+    csrc = tmp_path / "nvfp4_block_quantization_amax_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in bench.QUANT_SOURCES:
+        (csrc / f).write_text(f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.quantizer_issue_record() is None   # taken on other sources
+    import hashlib
+    h = hashlib.sha256(b"".join(f.encode() for f in bench.QUANT_SOURCES)).hexdigest()[:16]
+    (prof / "quantizer_issue.json").write_text(json.dumps({"source_sha256_16": h, "kernels": []}))
+    assert bench.quantizer_issue_record() == {"source_sha256_16": h, "kernels": []}
