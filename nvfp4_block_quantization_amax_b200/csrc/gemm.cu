@@ -830,6 +830,17 @@ __global__ void __launch_bounds__(P_THREADS, 1)
         if constexpr (VS) return __fmul_rn(__fmul_rn(__uint_as_float(acc_bits), am), __ldg(alpha_b + col0 + col));
         return __fmul_rn(__uint_as_float(acc_bits), ab);
       };
+      // two adjacent columns as packed bf16 (one packed multiply without VS)
+      auto scale_bf16x2 = [&](uint32_t acc0, uint32_t acc1, int col) -> uint32_t {
+        __nv_bfloat162 b2;
+        if constexpr (VS) {
+          b2 = __floats2bfloat162_rn(scale(acc0, col), scale(acc1, col + 1));
+        } else {
+          const float2 p = __fmul2_rn(make_float2(__uint_as_float(acc0), __uint_as_float(acc1)), make_float2(ab, ab));
+          b2 = __floats2bfloat162_rn(p.x, p.y);
+        }
+        return *reinterpret_cast<const uint32_t*>(&b2);
+      };
       if (!out_fp32) {
         // two rounds of 64 columns: load, wait, convert to packed bf16; the
         // accumulator is handed back once the whole row is in registers
@@ -842,10 +853,7 @@ __global__ void __launch_bounds__(P_THREADS, 1)
           tmem_ld32_nowait(taddr + c + 32, r + 32);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(scale(r[2 * j], c + 2 * j), scale(r[2 * j + 1], c + 2 * j + 1));
-            packed[c / 2 + j] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
+          for (int j = 0; j < 32; ++j) packed[c / 2 + j] = scale_bf16x2(r[2 * j], r[2 * j + 1], c + 2 * j);
         }
         fence_before();
         __syncwarp();
