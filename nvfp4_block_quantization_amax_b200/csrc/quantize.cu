@@ -736,7 +736,11 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         }
       }
     }
-    __syncthreads();   // buf and the staging are reused
+    // With the column pass no barrier is needed here: every read of this
+    // tile's buffer happens before the barrier ahead of the write-out, and
+    // every read of the staging before the next tile's first barrier, which
+    // the next writes of the staging follow.
+    if constexpr (!COL) __syncthreads();
   }
   cp_async_wait<0>();
 }
