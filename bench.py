@@ -181,12 +181,17 @@ class ClockSampler:
 class LayerStep:
     """Pre-allocated buffers and the C-ABI call sequence of one step."""
 
-    def __init__(self, x, w, dy, bwd_mode, device):
+    def __init__(self, x, w, dy, bwd_mode, device, shared_amax=True):
         import torch
         from nvfp4_block_quantization_amax_b200 import api
         self.api = api
         self.x, self.w, self.dy = x, w, dy
         self.bwd = bwd_mode
+        # shared_amax: one nvfp4_amax pass per weight / activation gives the
+        # plain amax of its forward quantization and the rotated-column amax
+        # of its backward partner; otherwise each call runs its own amax pass
+        self.shared_amax = shared_amax
+        self.amax = {k: torch.zeros(3, dtype=torch.float32, device=device) for k in ("x", "w")}
         T, H = x.shape
         O = w.shape[0]
         self.plan = [  # (tensor, mode, flags)
@@ -209,9 +214,9 @@ class LayerStep:
         self.dw = torch.empty((O, H), dtype=torch.bfloat16, device=device)
         self.ev = None
 
-    def quantize(self, name, mode, flags, seed, sid):
+    def quantize(self, name, mode, flags, seed, sid, amax=None):
         self.api.nvfp4_quantize(self.src[name], mode, flags, seed=seed, stream_id=sid, out=self.out[name],
-                                workspace=self.ws[name])
+                                workspace=self.ws[name], amax=amax)
 
     def run(self, step, timers=None):
         """One step.  timers: dict call name -> list of (start, end) CUDA
@@ -219,10 +224,16 @@ class LayerStep:
         api = self.api
         seed = 1000 * (step + 1)   # a new rotation and noise per step
         mark = (lambda k: _Mark(timers, k)) if timers is not None else (lambda k: _NoMark())
+        sa = self.shared_amax
+        ax, aw = self.amax["x"], self.amax["w"]
         with mark("q_x"):
-            self.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0)
+            if sa:
+                api.nvfp4_amax(self.x, COL | RHT, seed=seed, out=ax)
+            self.quantize("x", FOUR_SIX, ROW | GEMM, 0, 0, amax=ax if sa else None)
         with mark("q_w"):
-            self.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1)
+            if sa:
+                api.nvfp4_amax(self.w, COL | RHT, seed=seed, out=aw)
+            self.quantize("w", FOUR_SIX, ROW | B2D | GEMM, 0, 1, amax=aw if sa else None)
         qx, qw = self.out["x"], self.out["w"]
         with mark("fprop"):
             api.nvfp4_gemm(qx.codes_row, qx.scales_row, qx.alpha_row, qw.codes_row, qw.scales_row, qw.alpha_row,
@@ -230,13 +241,13 @@ class LayerStep:
         with mark("q_dy"):
             self.quantize("dy", self.bwd, ROW | COL | GEMM, seed, 0)
         with mark("q_w_rot"):
-            self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1)
+            self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1, amax=aw[1:] if sa else None)
         qd, qwr = self.out["dy"], self.out["w_rot"]
         with mark("dgrad"):
             api.nvfp4_gemm(qd.codes_row, qd.scales_row, qd.alpha_row, qwr.codes_col, qwr.scales_col,
                            qwr.alpha_col, out=self.dx)
         with mark("q_x_rot"):
-            self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2)
+            self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2, amax=ax[1:] if sa else None)
         qxr = self.out["x_rot"]
         with mark("wgrad"):
             api.nvfp4_gemm(qd.codes_col, qd.scales_col, qd.alpha_col, qxr.codes_col, qxr.scales_col,
@@ -474,7 +485,7 @@ def run_device(args, rank, world, local_rank):
     layer = synthetic.fwd_bwd_8b(seed=17 * rank)
     x, w, dy = (layer[k].to(device) for k in ("x", "w", "dy"))
     bwd = BWD_MODES[args.bwd_mode]
-    step = LayerStep(x, w, dy, bwd, device)
+    step = LayerStep(x, w, dy, bwd, device, shared_amax=not args.amax_per_call)
 
     # --- device-resident timing ---
     for i in range(args.warmup):
@@ -561,6 +572,9 @@ def run_device(args, rank, world, local_rank):
         "data": "synthetic (seeded; shapes and distributions of the pages' 8B workload)",
         "config": {"workload": workload(args.bwd_mode), "tokens": TOKENS, "hidden": HIDDEN, "out_features": OUT,
                    "bwd_mode": args.bwd_mode, "parallelism": f"replicas x{world} (weak)",
+                   "amax": "per call" if args.amax_per_call else
+                           "one nvfp4_amax pass per X and W (plain + rotated columns) shared by their forward "
+                           "and backward quantize calls; dY's own two-pass call",
                    "l2": "inputs larger than L2: 419 MB of bf16 per step; sub-benchmarks overwrite a 256 MiB "
                          "buffer before every timed call"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
@@ -627,7 +641,8 @@ def run_extras(args, step, x, w, dy, device, hbm, fp4_peak):
     # the 12B-hybrid-shaped step (BASELINE config 5): tokens 16384, hidden 5120, FFN 20480
     s = synthetic.STEP_12B
     lay = synthetic.device_layer(s["tokens"], s["hidden"], s["ffn"], seed=12, device=device)
-    st12 = LayerStep(lay["x"], lay["w"], lay["dy"], BWD_MODES[args.bwd_mode], device)
+    st12 = LayerStep(lay["x"], lay["w"], lay["dy"], BWD_MODES[args.bwd_mode], device,
+                     shared_amax=not args.amax_per_call)
     for i in range(3):
         st12.run(i)
     torch.cuda.synchronize()
@@ -818,6 +833,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--bwd-mode", choices=sorted(BWD_MODES), default="eden")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--amax-per-call", action="store_true",
+                    help="every quantize call runs its own amax pass (default: one nvfp4_amax pass per X and W "
+                         "serves their forward and rotated backward quantizations)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the sub-benchmarks (per-mode table, sweep, 12B step, GEMMs alone)")
     ap.add_argument("--kernel-case", choices=KERNEL_CASES,

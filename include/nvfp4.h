@@ -121,6 +121,18 @@ typedef enum {
                                      * 1D blocks only (not with BLOCK2D,
                                      * SINGLE_PASS or ALPHA_PROVIDED).  The
                                      * workspace holds the R + C vector maxima. */
+#define NVFP4_AMAX_PROVIDED 0x800u  /* skip the amax pass: alpha_in points to
+                                     * device float amax values (as written by
+                                     * nvfp4_amax), from which alpha follows by
+                                     * Eq. 1 exactly as in the two-pass path.
+                                     * Without rotation alpha_in[0] serves both
+                                     * orientations; with rotation alpha_in[0]
+                                     * is the row orientation's amax and
+                                     * alpha_in[1] the column orientation's.  A
+                                     * non-finite marker (0xFFFFFFFF) sets
+                                     * NVFP4_ERR_NONFINITE.  Not with
+                                     * ALPHA_PROVIDED, SINGLE_PASS or
+                                     * VECTOR_SCALES; needs no workspace. */
 /* nvfp4_dequantize flags (NVFP4_BLOCK2D and NVFP4_GEMM_SCALE_LAYOUT also apply) */
 #define NVFP4_INVERSE_RHT 0x80u     /* undo the rotation after decoding          */
 #define NVFP4_OUT_BF16 0x100u       /* write bf16 instead of fp32                */
@@ -170,7 +182,8 @@ NVFP4_API size_t nvfp4_workspace_size(int64_t R, int64_t C, uint32_t flags);
  * Steps ([46] §2.1 Eq. 1-3; [NV] §六):
  *   1. amax = max |x| (max over the rotated values in rotating modes,
  *      separately per orientation); alpha = amax / (6 * 448)        (Eq. 1)
- *      -- skipped with NVFP4_ALPHA_PROVIDED (alpha = *alpha_in, device).
+ *      -- skipped with NVFP4_ALPHA_PROVIDED (alpha = *alpha_in, device), or
+ *      taken from amax values computed earlier with NVFP4_AMAX_PROVIDED.
  *   2. per block: Delta = E4M3(amax_block / (alpha * M))             (Eq. 2)
  *   3. per element: q = E2M1(x / (alpha * Delta)), computed as x times the
  *      correctly rounded reciprocal of alpha * Delta                 (Eq. 3)
@@ -196,6 +209,25 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int
                               uint32_t stream_id, const float* alpha_in,
                               const nvfp4_qtensor_t* out, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* The amax values of Eq. 1 ([46] §2.1 Eq. 1; [NV] §六 step 1) of the bf16
+ * tensor x [R, C] (row stride ld), for later nvfp4_quantize calls with
+ * NVFP4_AMAX_PROVIDED: one read of x gives
+ *   amax_out[0] = max |x|                               (plain)
+ *   amax_out[1] = max |(1/4) H16 D v| over the 16-element row blocks v
+ *                 (with NVFP4_ROWWISE | NVFP4_RHT)
+ *   amax_out[2] = the same over the 16-element column blocks
+ *                 (with NVFP4_COLWISE | NVFP4_RHT; R % 16 == 0)
+ * with D the sign diagonal drawn from `seed` (as nvfp4_quantize rotates).
+ * A tensor whose plain, row or column maxima several quantize calls need is
+ * read once instead of once per call: pass amax_out to a call without
+ * rotation and amax_out + 1 to a rotating one.  Entries not requested are 0.
+ * Each value is a device float (bit pattern 0xFFFFFFFF if a NaN or Inf was
+ * read, and then NVFP4_ERR_NONFINITE in *status when status is not NULL).
+ * x 16-byte aligned, ld % 8 == 0, C % 16 == 0; amax_out 4-byte aligned (3
+ * floats, written through the stream; no workspace). */
+NVFP4_API nvfp4_status_t nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags,
+                                    uint64_t seed, float* amax_out, int32_t* status, void* stream);
 
 /* nvfp4_quantize for callers that may not allocate device memory while they
  * run (no page defines this; it has no counterpart in the method): a plugin

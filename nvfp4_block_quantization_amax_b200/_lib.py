@@ -23,6 +23,7 @@ NVFP4_SINGLE_PASS = 0x8
 NVFP4_HEADROOM = 0x200
 NVFP4_VECTOR_SCALES = 0x400
 NVFP4_ALPHA_PROVIDED = 0x10
+NVFP4_AMAX_PROVIDED = 0x800
 NVFP4_GEMM_SCALE_LAYOUT = 0x20
 NVFP4_RHT = 0x40
 NVFP4_INVERSE_RHT = 0x80
@@ -31,7 +32,7 @@ NVFP4_OUT_BF16 = 0x100
 NVFP4_OUT_DTYPE_BF16 = 0
 NVFP4_OUT_DTYPE_FP32 = 1
 
-EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_dequantize",
+EXPORTED = ("nvfp4_workspace_size", "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_amax", "nvfp4_dequantize",
             "nvfp4_gemm", "nvfp4_gemm_vector_scales", "nvfp4_gemm_quantize", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "nvfp4_launch_count",
             "nvfp4_status_string", "nvfp4_version")
 
@@ -64,6 +65,8 @@ def load(path=LIB_PATH):
     L.nvfp4_quantize_noalloc.argtypes = [vp, i64, i64, i64, ctypes.c_int, u32, u64, u32, vp,
                                          ctypes.POINTER(nvfp4_qtensor_t), vp]
     L.nvfp4_quantize_noalloc.restype = ctypes.c_int
+    L.nvfp4_amax.argtypes = [vp, i64, i64, i64, u32, u64, vp, vp, vp]
+    L.nvfp4_amax.restype = ctypes.c_int
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, u32, u64, vp, vp]
     L.nvfp4_dequantize.restype = ctypes.c_int
     L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, ctypes.c_int, i64, vp, sz, vp]
@@ -106,6 +109,10 @@ def nvfp4_quantize_noalloc(x, R, C, ld, mode, flags, seed, stream_id, alpha_in, 
     stream)."""
     return int(load().nvfp4_quantize_noalloc(x, R, C, ld, mode, flags, seed, stream_id, alpha_in,
                                              ctypes.byref(out), stream))
+
+
+def nvfp4_amax(x, R, C, ld, flags, seed, amax_out, status, stream):
+    return int(load().nvfp4_amax(x, R, C, ld, flags, seed, amax_out, status, stream))
 
 
 def nvfp4_dequantize(codes, scales, alpha, R, C, flags, seed, y, stream):

@@ -9,7 +9,7 @@ from typing import Optional
 import torch
 
 from . import _lib as L
-from ._lib import (NVFP4_ALPHA_PROVIDED, NVFP4_BLOCK2D, NVFP4_COLWISE, NVFP4_FOUR_SIX,  # noqa: F401
+from ._lib import (NVFP4_ALPHA_PROVIDED, NVFP4_AMAX_PROVIDED, NVFP4_BLOCK2D, NVFP4_COLWISE, NVFP4_FOUR_SIX,  # noqa: F401
                    NVFP4_GEMM_SCALE_LAYOUT, NVFP4_INVERSE_RHT, NVFP4_MS_EDEN, NVFP4_OUT_BF16,
                    NVFP4_OUT_DTYPE_BF16, NVFP4_OUT_DTYPE_FP32, NVFP4_RHT, NVFP4_RHT_SR, NVFP4_RHT_SR_HW,
                    NVFP4_ROWWISE, NVFP4_RTN, NVFP4_SINGLE_PASS, NVFP4_VECTOR_SCALES)
@@ -119,20 +119,53 @@ def workspace_for(R: int, C: int, flags: int, device) -> Optional[torch.Tensor]:
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
-def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream_id: int = 0,
-                   alpha: Optional[torch.Tensor] = None, out: Optional[QTensor] = None,
-                   workspace: Optional[torch.Tensor] = None,
-                   status: Optional[torch.Tensor] = None) -> QTensor:
-    """Quantize a 2D bf16 CUDA tensor (unit column stride) with the C ABI's
-    nvfp4_quantize; allocates outputs and workspace when not given."""
+def nvfp4_amax(x: torch.Tensor, flags: int = 0, seed: int = 0, out: Optional[torch.Tensor] = None,
+               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The amax values of Eq. 1 from one read of x with the C ABI's
+    nvfp4_amax: [plain, rotated rows, rotated columns] as a float32 CUDA
+    tensor of 3 (rotated entries with NVFP4_RHT and the orientation flag)."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
         raise TypeError("x must be a 2D bfloat16 CUDA tensor")
     if x.numel() and x.stride(1) != 1:
         raise ValueError("x must have unit column stride")
     R, C = x.shape
     ld = x.stride(0) if x.numel() else C
+    if out is not None:
+        _need(out, 3, torch.float32, "out", x.device)
+    if status is not None:
+        _need(status, 1, torch.int32, "status", x.device)
+    a = out if out is not None else torch.empty(3, dtype=torch.float32, device=x.device)
+    st = L.nvfp4_amax(_p(x), R, C, ld, flags, seed, _p(a), _p(status), _stream())
+    _check(st, "nvfp4_amax")
+    return a
+
+
+def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream_id: int = 0,
+                   alpha: Optional[torch.Tensor] = None, out: Optional[QTensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None) -> QTensor:
+    """Quantize a 2D bf16 CUDA tensor (unit column stride) with the C ABI's
+    nvfp4_quantize; allocates outputs and workspace when not given.  alpha
+    (a device float) replaces Eq. 1 (NVFP4_ALPHA_PROVIDED); amax (device
+    floats from nvfp4_amax: the plain entry for a call without rotation, the
+    slice from the rotated-rows entry on for a rotating one) replaces the
+    amax pass (NVFP4_AMAX_PROVIDED)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2D bfloat16 CUDA tensor")
+    if x.numel() and x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    R, C = x.shape
+    ld = x.stride(0) if x.numel() else C
+    if alpha is not None and amax is not None:
+        raise ValueError("give alpha or amax, not both")
     if alpha is not None:
         flags |= NVFP4_ALPHA_PROVIDED
+    if amax is not None:
+        if amax.dtype != torch.float32 or not amax.is_cuda or amax.device != x.device or amax.numel() < 1 \
+                or not amax.is_contiguous():
+            raise ValueError("amax must be a contiguous float32 tensor on x's device")
+        flags |= NVFP4_AMAX_PROVIDED
+        alpha = amax
     if out is not None:
         check_outputs(out, R, C, flags, x.device)
     if status is not None:

@@ -10,7 +10,8 @@
 namespace {
 
 constexpr uint32_t kQuantFlags = NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_BLOCK2D | NVFP4_SINGLE_PASS | NVFP4_HEADROOM |
-                                 NVFP4_ALPHA_PROVIDED | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_RHT | NVFP4_VECTOR_SCALES;
+                                 NVFP4_ALPHA_PROVIDED | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_RHT | NVFP4_VECTOR_SCALES |
+                                 NVFP4_AMAX_PROVIDED;
 constexpr uint32_t kDequantFlags = NVFP4_BLOCK2D | NVFP4_GEMM_SCALE_LAYOUT | NVFP4_INVERSE_RHT | NVFP4_OUT_BF16;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -46,6 +47,9 @@ nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t 
   if (stream_id >= 0x80000000u) return NVFP4_ERR_ARG;
   if ((flags & NVFP4_VECTOR_SCALES) && (flags & (NVFP4_BLOCK2D | NVFP4_SINGLE_PASS | NVFP4_ALPHA_PROVIDED)))
     return NVFP4_ERR_ARG;
+  if ((flags & NVFP4_AMAX_PROVIDED) &&
+      (flags & (NVFP4_ALPHA_PROVIDED | NVFP4_SINGLE_PASS | NVFP4_VECTOR_SCALES)))
+    return NVFP4_ERR_ARG;
   if (R < 0 || C < 0 || ld < C) return NVFP4_ERR_SHAPE;
   if (C % 16) return NVFP4_ERR_SHAPE;
   if ((col || two_d) && R % 16) return NVFP4_ERR_SHAPE;
@@ -58,7 +62,8 @@ nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t 
     *empty = true;
     return NVFP4_OK;
   }
-  if ((flags & NVFP4_ALPHA_PROVIDED) && !alpha_in) return NVFP4_ERR_ARG;
+  if ((flags & (NVFP4_ALPHA_PROVIDED | NVFP4_AMAX_PROVIDED)) && !alpha_in) return NVFP4_ERR_ARG;
+  if ((flags & NVFP4_AMAX_PROVIDED) && !aligned(alpha_in, 4)) return NVFP4_ERR_ALIGN;
   if (row && (!out->codes_row || !out->scales_row || !out->alpha_row)) return NVFP4_ERR_ARG;
   if (col && (!out->codes_col || !out->scales_col || !out->alpha_col)) return NVFP4_ERR_ARG;
   if (!x) return NVFP4_ERR_ARG;
@@ -72,6 +77,22 @@ nvfp4_status_t check_quantize_args(const void* x, int64_t R, int64_t C, int64_t 
 extern "C" {
 
 uint64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+nvfp4_status_t nvfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
+                          float* amax_out, int32_t* status, void* stream) {
+  if (flags & ~(NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_RHT)) return NVFP4_ERR_ARG;
+  if (!amax_out) return NVFP4_ERR_ARG;
+  if (R < 0 || C < 0 || ld < C || C % 16) return NVFP4_ERR_SHAPE;
+  if ((flags & NVFP4_RHT) && (flags & NVFP4_COLWISE) && R % 16) return NVFP4_ERR_SHAPE;
+  if (R * (C / 8) >= (int64_t(1) << 32)) return NVFP4_ERR_SHAPE;
+  if (!aligned(amax_out, 4) || (status && !aligned(status, 4))) return NVFP4_ERR_ALIGN;
+  if (R > 0 && C > 0) {
+    if (!x) return NVFP4_ERR_ARG;
+    if (!aligned(x, 16) || ld % 8) return NVFP4_ERR_ALIGN;
+  }
+  return launch_status(nvfp4::amax_launch(x, R, C, ld, flags, seed, amax_out, status,
+                                          static_cast<cudaStream_t>(stream)));
+}
 
 nvfp4_status_t mxfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
                               uint8_t* codes_row, uint8_t* scales_row, uint8_t* codes_col, uint8_t* scales_col,

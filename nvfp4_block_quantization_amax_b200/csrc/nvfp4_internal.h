@@ -20,6 +20,7 @@ constexpr uint32_t kSinglePass = NVFP4_SINGLE_PASS;
 constexpr uint32_t kHeadroom = NVFP4_HEADROOM;
 constexpr uint32_t kVectorScales = NVFP4_VECTOR_SCALES;
 constexpr uint32_t kAlphaProvided = NVFP4_ALPHA_PROVIDED;
+constexpr uint32_t kAmaxProvided = NVFP4_AMAX_PROVIDED;
 constexpr uint32_t kGemmScaleLayout = NVFP4_GEMM_SCALE_LAYOUT;
 constexpr uint32_t kRht = NVFP4_RHT;
 constexpr uint32_t kInverseRht = NVFP4_INVERSE_RHT;
@@ -54,6 +55,10 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
                             uint32_t flags, uint64_t seed, uint32_t stream_id,
                             const float* alpha_in, const QuantOutputs& out, void* workspace,
                             cudaStream_t st);
+
+// nvfp4_amax (quantize.cu): amax_out[0..2] = plain, rotated rows, rotated columns.
+cudaError_t amax_launch(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
+                        float* amax_out, int32_t* status, cudaStream_t st);
 
 cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* scales, const float* alpha,
                               int64_t R, int64_t C, uint32_t flags, uint64_t seed, void* y,

@@ -55,6 +55,7 @@ struct QuantArgs {
   FastDiv chunks_row;             // C / 8: 16-byte chunks per row (plain amax)
   uint32_t* vmax_r;               // NVFP4_VECTOR_SCALES: per-row maxima [R] (float bits)
   uint32_t* vmax_c;               // and per-column maxima [C]
+  int amax_rot;                   // NVFP4_AMAX_PROVIDED: rotated (per-orientation amax values)
 };
 
 // Tensor scale of one vector from its maximum (Eq. 1 per vector; the
@@ -109,8 +110,16 @@ __device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, b
     return;
   }
   uint32_t mr = 0, mc = 0;
-  if (need_r) mr = reduce_partials<NT>(a.partials, a.npart, red);
-  if (need_c) mc = reduce_partials<NT>(a.partials_col, a.npart, red);
+  if (a.flags & kAmaxProvided) {
+    // amax values from an earlier amax pass (nvfp4_amax): [0] for the row
+    // orientation (both without rotation), [1] for the columns when rotated
+    const uint32_t* am = reinterpret_cast<const uint32_t*>(a.alpha_in);
+    if (need_r) mr = __ldg(am);
+    if (need_c) mc = __ldg(am + (a.amax_rot ? 1 : 0));
+  } else {
+    if (need_r) mr = reduce_partials<NT>(a.partials, a.npart, red);
+    if (need_c) mc = reduce_partials<NT>(a.partials_col, a.npart, red);
+  }
   // Eq. 1: alpha = amax / (6 * 448); with NVFP4_HEADROOM amax / (4 * 448)
   const float amax_r = __uint_as_float(mr == kNonFinite ? 0u : mr);
   const float amax_c = __uint_as_float(mc == kNonFinite ? 0u : mc);
@@ -141,9 +150,12 @@ __device__ __forceinline__ uint32_t sign_bits(const PhiloxKeys& K) {
 // sign cleared, so two are compared at once with a per-halfword unsigned
 // max; a pattern >= 0x7F80 is an Inf or a NaN.
 template <int NT>
+// With atomic_out the CTA's maximum is folded into atomic_out[0] (zeroed by
+// the launcher) instead of being stored as a partial.
 __device__ __forceinline__ void amax_plain_body(const uint16_t* __restrict__ x, int64_t R, int64_t ld, FastDiv cpr,
                                                 uint32_t* __restrict__ partial, uint32_t cta, uint32_t ncta,
-                                                uint32_t* red) {
+                                                uint32_t* red, uint32_t* atomic_out = nullptr,
+                                                int32_t* status = nullptr) {
   const uint32_t total = static_cast<uint32_t>(R) * cpr.d;   // chunks of 8 values
   const uint32_t stride = ncta * NT;
   uint32_t hm = 0;
@@ -174,7 +186,14 @@ __device__ __forceinline__ void amax_plain_body(const uint16_t* __restrict__ x, 
   const uint32_t h = max(hm & 0xFFFFu, hm >> 16);
   uint32_t m = (h >= 0x7F80u) ? kNonFinite : (h << 16);
   m = block_max_u32<NT>(m, red);
-  if (threadIdx.x == 0) partial[cta] = m;
+  if (threadIdx.x == 0) {
+    if (atomic_out) {
+      atomicMax(atomic_out, m);
+      if (m == kNonFinite && status) *status = kStatusNonFinite;
+    } else {
+      partial[cta] = m;
+    }
+  }
 }
 
 // Rotated maxima: rows (16-element blocks along a row) and / or columns
@@ -182,11 +201,16 @@ __device__ __forceinline__ void amax_plain_body(const uint16_t* __restrict__ x, 
 // butterfly runs on two blocks at once (lane-paired) and without its final
 // 1/4: round-to-nearest multiplication is monotone, so the maximum of the
 // scaled magnitudes is the scaled maximum, applied once per CTA.
+// With atomic_out the CTA's maxima are folded into atomic_out[0] (plain
+// max |x|, from the same per-halfword maximum the Inf / NaN check keeps),
+// [1] (rotated rows) and [2] (rotated columns), zeroed by the launcher,
+// instead of being stored as partials.
 template <bool ROW, bool COL>
 __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, int64_t R, int64_t C, int64_t ld,
                                                FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
                                                uint32_t* __restrict__ part_r, uint32_t* __restrict__ part_c,
-                                               uint32_t cta, uint32_t ncta, uint8_t* ring, uint32_t* red) {
+                                               uint32_t cta, uint32_t ncta, uint8_t* ring, uint32_t* red,
+                                               uint32_t* atomic_out = nullptr, int32_t* status = nullptr) {
   auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);   // two tile buffers
   const SignMasks sm = sign_masks(sign_bits(philox_keys(seed)));
   const int t = threadIdx.x;
@@ -259,15 +283,28 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   }
   const uint32_t h = max(hin & 0xFFFFu, hin >> 16);
   const bool bad = h >= 0x7F80u;
+  if (atomic_out) {
+    const uint32_t mp = block_max_u32<TNT>(bad ? kNonFinite : (h << 16), red);
+    if (t == 0) {
+      atomicMax(atomic_out, mp);
+      if (mp == kNonFinite && status) *status = kStatusNonFinite;
+    }
+  }
   if constexpr (ROW) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mr, 0.25f));
     m = block_max_u32<TNT>(m, red);
-    if (t == 0) part_r[cta] = m;
+    if (t == 0) {
+      if (atomic_out) atomicMax(atomic_out + 1, m);
+      else part_r[cta] = m;
+    }
   }
   if constexpr (COL) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mc, 0.25f));
     m = block_max_u32<TNT>(m, red);
-    if (t == 0) part_c[cta] = m;
+    if (t == 0) {
+      if (atomic_out) atomicMax(atomic_out + 2, m);
+      else part_c[cta] = m;
+    }
   }
 }
 
@@ -974,6 +1011,28 @@ __global__ void __launch_bounds__(NT) amax_plain_kernel(const uint16_t* __restri
   amax_plain_body<NT>(x, R, ld, cpr, partial, blockIdx.x, gridDim.x, red);
 }
 
+// The amax pass of nvfp4_amax: maxima folded into out[0..2] (zeroed first).
+template <int NT>
+__global__ void __launch_bounds__(NT) amax_plain_atomic_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t ld,
+                                                               FastDiv cpr, uint32_t* __restrict__ out,
+                                                               int32_t* status) {
+  pdl_entry();
+  __shared__ uint32_t red[NT / 32];
+  amax_plain_body<NT>(x, R, ld, cpr, nullptr, blockIdx.x, gridDim.x, red, out, status);
+}
+
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(TNT) amax_tile_atomic_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                               int64_t ld, FastDiv tiles_c, uint32_t ntiles,
+                                                               uint64_t seed, uint32_t* __restrict__ out,
+                                                               int32_t* status) {
+  pdl_entry();
+  __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
+  __shared__ uint32_t red[TNT / 32];
+  amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, nullptr, nullptr, blockIdx.x, gridDim.x, ring, red,
+                           out, status);
+}
+
 template <bool ROW, bool COL>
 __global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
                                                         int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
@@ -1239,7 +1298,7 @@ size_t vec_workspace_bytes(int64_t R, int64_t C) {
 
 size_t quant_workspace_bytes(int64_t R, int64_t C, uint32_t flags) {
   if (flags & kVectorScales) return vec_workspace_bytes(R, C);
-  if (flags & kAlphaProvided) return 0;
+  if (flags & (kAlphaProvided | kAmaxProvided)) return 0;
   const size_t partials = static_cast<size_t>(2 * amax_partial_count()) * sizeof(uint32_t);
   return (flags & kSinglePass) ? partials + 16 : partials;
 }
@@ -1396,6 +1455,38 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
   return cudaGetLastError();
 }
 
+// nvfp4_amax: out[0..2] (plain, rotated rows, rotated columns) cleared, then
+// one pass folds every CTA's maxima into them.
+cudaError_t amax_launch(const void* x, int64_t R, int64_t C, int64_t ld, uint32_t flags, uint64_t seed,
+                        float* amax_out, int32_t* status, cudaStream_t st) {
+  uint32_t* out = reinterpret_cast<uint32_t*>(amax_out);
+  cudaError_t e = cudaMemsetAsync(out, 0, 3 * sizeof(uint32_t), st);
+  if (e != cudaSuccess || R == 0 || C == 0) return e;
+  const bool rot = (flags & kRht) != 0;
+  const bool row = rot && (flags & kRowwise), col = rot && (flags & kColwise);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  const int np = amax_partial_count();
+  if (!row && !col) {
+    launch_k(amax_plain_atomic_kernel<256>, dim3(np), dim3(256), 0, st, 1u, xs, R, ld,
+             make_fastdiv(static_cast<uint32_t>(C / 8)), out, status);
+  } else {
+    const int64_t tiles_r = (R + TR - 1) / TR, tiles_c = (C + TC - 1) / TC;
+    const uint32_t ntiles = static_cast<uint32_t>(tiles_r * tiles_c);
+    const FastDiv tcd = make_fastdiv(static_cast<uint32_t>(tiles_c));
+    if (row && col)
+      launch_k(amax_tile_atomic_kernel<true, true>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+               out, status);
+    else if (row)
+      launch_k(amax_tile_atomic_kernel<true, false>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+               out, status);
+    else
+      launch_k(amax_tile_atomic_kernel<false, true>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+               out, status);
+  }
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int mode, uint32_t flags,
                             uint64_t seed, uint32_t stream_id, const float* alpha_in,
                             const QuantOutputs& o, void* workspace, cudaStream_t st) {
@@ -1427,6 +1518,7 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
   const bool row = flags & kRowwise, col = flags & kColwise, two_d = flags & kBlock2D;
   const bool rot = (mode == kModeRhtSR || mode == kModeMsEden || mode == kModeRhtSRHw || (flags & kRht)) && !two_d;
   if (rot) a.partials_col = a.partials + a.npart;
+  a.amax_rot = rot ? 1 : 0;
   if (R == 0 || C == 0) return cudaSuccess;
   if (flags & kVectorScales) return quantize_vector_scales(a, mode, row, col, rot, st);
 
@@ -1457,7 +1549,7 @@ cudaError_t quantize_launch(const void* x, int64_t R, int64_t C, int64_t ld, int
     }
   }
 
-  if (!(flags & kAlphaProvided)) {
+  if (!(flags & (kAlphaProvided | kAmaxProvided))) {
     cudaError_t e = launch_amax(a, row || two_d, col && !two_d, rot, st);
     if (e != cudaSuccess) return e;
   }

@@ -40,6 +40,16 @@ int main(void) {
                    NVFP4_OUT_DTYPE_BF16, 128, NULL, 0, NULL) == NVFP4_ERR_SHAPE);
   CHECK(nvfp4_gemm_quantize(fb, fb, (const float*)fake, fb, fb, (const float*)fake, 256, 256, 128, NULL, 256,
                             NVFP4_MS_EDEN, 0, (const float*)fake, fb, fb, NULL, NULL, 0, NULL) == NVFP4_ERR_ARG);
+  /* amax pass: bad flags, missing output, shapes; AMAX_PROVIDED needs amax input and excludes ALPHA_PROVIDED */
+  CHECK(nvfp4_amax(fake, 16, 16, 16, NVFP4_BLOCK2D, 0, (float*)fake, NULL, NULL) == NVFP4_ERR_ARG);
+  CHECK(nvfp4_amax(fake, 16, 16, 16, 0, 0, NULL, NULL, NULL) == NVFP4_ERR_ARG);
+  CHECK(nvfp4_amax(fake, 16, 24, 24, 0, 0, (float*)fake, NULL, NULL) == NVFP4_ERR_SHAPE);
+  CHECK(nvfp4_amax(fake, 24, 16, 16, NVFP4_COLWISE | NVFP4_RHT, 0, (float*)fake, NULL, NULL) == NVFP4_ERR_SHAPE);
+  CHECK(nvfp4_workspace_size(16, 16, NVFP4_ROWWISE | NVFP4_AMAX_PROVIDED) == 0);
+  CHECK(nvfp4_quantize(fake, 16, 16, 16, NVFP4_RTN, NVFP4_ROWWISE | NVFP4_AMAX_PROVIDED, 0, 0, NULL, &out, NULL, 0,
+                       NULL) == NVFP4_ERR_ARG);
+  CHECK(nvfp4_quantize(fake, 16, 16, 16, NVFP4_RTN, NVFP4_ROWWISE | NVFP4_AMAX_PROVIDED | NVFP4_ALPHA_PROVIDED, 0, 0,
+                       (const float*)fake, &out, NULL, 0, NULL) == NVFP4_ERR_ARG);
   /* MXFP4 */
   CHECK(mxfp4_quantize(fake, 32, 48, 48, NVFP4_ROWWISE, 0, fb, fb, NULL, NULL, NULL, NULL) == NVFP4_ERR_SHAPE);
   CHECK(mxfp4_quantize(fake, 32, 32, 32, 0, 0, fb, fb, NULL, NULL, NULL, NULL) == NVFP4_ERR_ARG);

@@ -79,6 +79,23 @@ def test_host_argument_checks_need_no_gpu(lib):
                             None) == L.NVFP4_ERR_WORKSPACE
     # empty tensors are a no-op
     assert L.nvfp4_quantize(None, 0, 16, 16, 0, L.NVFP4_ROWWISE, 0, 0, None, out, None, 0, None) == L.NVFP4_OK
+    # amax pass: flags, output, shapes, alignment; AMAX_PROVIDED needs the amax
+    # input, excludes ALPHA_PROVIDED / SINGLE_PASS / VECTOR_SCALES, needs no workspace
+    assert L.nvfp4_amax(fake, 16, 16, 16, L.NVFP4_BLOCK2D, 0, fake, None, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_amax(fake, 16, 16, 16, 0, 0, None, None, None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_amax(fake, 16, 24, 24, 0, 0, fake, None, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_amax(fake, 24, 16, 16, L.NVFP4_COLWISE | L.NVFP4_RHT, 0, fake, None, None) == L.NVFP4_ERR_SHAPE
+    assert L.nvfp4_amax(fake + 8, 16, 16, 16, 0, 0, fake, None, None) == L.NVFP4_ERR_ALIGN
+    assert L.nvfp4_amax(fake, 16, 16, 16, 0, 0, fake + 2, None, None) == L.NVFP4_ERR_ALIGN
+    assert L.nvfp4_workspace_size(16, 16, L.NVFP4_ROWWISE | L.NVFP4_AMAX_PROVIDED) == 0
+    amax = L.NVFP4_AMAX_PROVIDED
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE | amax, 0, 0, None, out, None, 0,
+                            None) == L.NVFP4_ERR_ARG
+    for other in (L.NVFP4_ALPHA_PROVIDED, L.NVFP4_SINGLE_PASS, L.NVFP4_VECTOR_SCALES):
+        assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE | amax | other, 0, 0, fake, out, None, 0,
+                                None) == L.NVFP4_ERR_ARG
+    assert L.nvfp4_quantize(fake, 16, 16, 16, 0, L.NVFP4_ROWWISE | amax, 0, 0, fake + 2, out, None, 0,
+                            None) == L.NVFP4_ERR_ALIGN
     # dequantize / gemm checks
     assert L.nvfp4_dequantize(fake, fake, fake, 16, 24, 0, 0, fake, None) == L.NVFP4_ERR_SHAPE
     assert L.nvfp4_dequantize(fake, fake, fake, 16, 16, 0x8000, 0, fake, None) == L.NVFP4_ERR_ARG
