@@ -241,13 +241,13 @@ class LayerStep:
         with mark("q_dy"):
             self.quantize("dy", self.bwd, ROW | COL | GEMM, seed, 0)
         with mark("q_w_rot"):
-            self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1, amax=aw[1:] if sa else None)
+            self.quantize("w_rot", RTN, COL | RHT | GEMM, seed, 1, amax=aw if sa else None)
         qd, qwr = self.out["dy"], self.out["w_rot"]
         with mark("dgrad"):
             api.nvfp4_gemm(qd.codes_row, qd.scales_row, qd.alpha_row, qwr.codes_col, qwr.scales_col,
                            qwr.alpha_col, out=self.dx)
         with mark("q_x_rot"):
-            self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2, amax=ax[1:] if sa else None)
+            self.quantize("x_rot", RTN, COL | RHT | GEMM, seed, 2, amax=ax if sa else None)
         qxr = self.out["x_rot"]
         with mark("wgrad"):
             api.nvfp4_gemm(qd.codes_col, qd.scales_col, qd.alpha_col, qxr.codes_col, qxr.scales_col,

@@ -122,13 +122,12 @@ typedef enum {
                                      * SINGLE_PASS or ALPHA_PROVIDED).  The
                                      * workspace holds the R + C vector maxima. */
 #define NVFP4_AMAX_PROVIDED 0x800u  /* skip the amax pass: alpha_in points to
-                                     * device float amax values (as written by
-                                     * nvfp4_amax), from which alpha follows by
-                                     * Eq. 1 exactly as in the two-pass path.
-                                     * Without rotation alpha_in[0] serves both
-                                     * orientations; with rotation alpha_in[0]
-                                     * is the row orientation's amax and
-                                     * alpha_in[1] the column orientation's.  A
+                                     * the three device floats nvfp4_amax
+                                     * writes (plain, rotated rows, rotated
+                                     * columns), from which alpha follows by
+                                     * Eq. 1 exactly as in the two-pass path:
+                                     * [0] without rotation, [1] for rotated
+                                     * rows, [2] for rotated columns.  A
                                      * non-finite marker (0xFFFFFFFF) sets
                                      * NVFP4_ERR_NONFINITE.  Not with
                                      * ALPHA_PROVIDED, SINGLE_PASS or
@@ -220,8 +219,8 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t R, int64_t C, int
  *                 (with NVFP4_COLWISE | NVFP4_RHT; R % 16 == 0)
  * with D the sign diagonal drawn from `seed` (as nvfp4_quantize rotates).
  * A tensor whose plain, row or column maxima several quantize calls need is
- * read once instead of once per call: pass amax_out to a call without
- * rotation and amax_out + 1 to a rotating one.  Entries not requested are 0.
+ * read once instead of once per call: pass amax_out as each call's alpha_in
+ * with NVFP4_AMAX_PROVIDED.  Entries not requested are 0.
  * Each value is a device float (bit pattern 0xFFFFFFFF if a NaN or Inf was
  * read, and then NVFP4_ERR_NONFINITE in *status when status is not NULL).
  * x 16-byte aligned, ld % 8 == 0, C % 16 == 0; amax_out 4-byte aligned (3

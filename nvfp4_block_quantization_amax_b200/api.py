@@ -146,10 +146,9 @@ def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream
                    status: Optional[torch.Tensor] = None, amax: Optional[torch.Tensor] = None) -> QTensor:
     """Quantize a 2D bf16 CUDA tensor (unit column stride) with the C ABI's
     nvfp4_quantize; allocates outputs and workspace when not given.  alpha
-    (a device float) replaces Eq. 1 (NVFP4_ALPHA_PROVIDED); amax (device
-    floats from nvfp4_amax: the plain entry for a call without rotation, the
-    slice from the rotated-rows entry on for a rotating one) replaces the
-    amax pass (NVFP4_AMAX_PROVIDED)."""
+    (a device float) replaces Eq. 1 (NVFP4_ALPHA_PROVIDED); amax (the three
+    device floats nvfp4_amax writes) replaces the amax pass
+    (NVFP4_AMAX_PROVIDED)."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
         raise TypeError("x must be a 2D bfloat16 CUDA tensor")
     if x.numel() and x.stride(1) != 1:
@@ -161,7 +160,7 @@ def nvfp4_quantize(x: torch.Tensor, mode: int, flags: int, seed: int = 0, stream
     if alpha is not None:
         flags |= NVFP4_ALPHA_PROVIDED
     if amax is not None:
-        if amax.dtype != torch.float32 or not amax.is_cuda or amax.device != x.device or amax.numel() < 1 \
+        if amax.dtype != torch.float32 or not amax.is_cuda or amax.device != x.device or amax.numel() < 3 \
                 or not amax.is_contiguous():
             raise ValueError("amax must be a contiguous float32 tensor on x's device")
         flags |= NVFP4_AMAX_PROVIDED

@@ -111,11 +111,11 @@ __device__ __forceinline__ void resolve_alpha(const QuantArgs& a, bool need_r, b
   }
   uint32_t mr = 0, mc = 0;
   if (a.flags & kAmaxProvided) {
-    // amax values from an earlier amax pass (nvfp4_amax): [0] for the row
-    // orientation (both without rotation), [1] for the columns when rotated
+    // amax values of an earlier amax pass (nvfp4_amax's [plain, rotated
+    // rows, rotated columns]): the plain one without rotation
     const uint32_t* am = reinterpret_cast<const uint32_t*>(a.alpha_in);
-    if (need_r) mr = __ldg(am);
-    if (need_c) mc = __ldg(am + (a.amax_rot ? 1 : 0));
+    if (need_r) mr = __ldg(am + (a.amax_rot ? 1 : 0));
+    if (need_c) mc = __ldg(am + (a.amax_rot ? 2 : 0));
   } else {
     if (need_r) mr = reduce_partials<NT>(a.partials, a.npart, red);
     if (need_c) mc = reduce_partials<NT>(a.partials_col, a.npart, red);
