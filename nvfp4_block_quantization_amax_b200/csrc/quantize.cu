@@ -588,44 +588,54 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   // (R % 64 == 0 keeps both aligned)
   const bool col_words = R % 64 == 0 && (reinterpret_cast<uintptr_t>(a.scales_col) & 3u) == 0;
 
+  // Per-thread parts of the block indices and offsets, fixed for the whole
+  // kernel: rows t/8 and t/8 + 32 of block column t%8 (row orientation);
+  // columns 2 (t/4), +1 of row block t%4 and, in the write-out, column t/2
+  // (column orientation).  A tile adds its own part once.
+  const int64_t nbr = C / 16, nbc = R / 16;
+  const int trow = t >> 3, tcb = t & 7, tcp = t >> 2, trb = t & 3;
+  const int64_t rblk_thr = trow * nbr + tcb, rcode_thr = trow * (C / 2) + 8 * tcb;
+  const int64_t cblk_thr = 2 * tcp * nbc + trb, ccode_thr = (t >> 1) * (R / 2) + 16 * (t & 1);
+  const int64_t share_thr = (j4 < 2) ? (trow + 32 * j4) * nbr + (tcb & ~3) : (2 * tcp + (j4 - 2)) * nbc;
+  // this tile and the one kTileStages - 1 iterations ahead, walked without
+  // divisions
+  TileWalk cur(cta, ncta, static_cast<uint32_t>(a.tiles_c)), ahd = cur;
+
   // prologue: the first kTileStages - 1 tiles (an empty copy group when a
   // tile does not exist keeps the group count in step)
   uint32_t tile = cta;
 #pragma unroll
   for (int k = 0; k < kTileStages - 1; ++k) {
     const uint32_t tk = tile + k * ncta;
-    if (tk < ntiles) load_tile_async(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
+    if (tk < ntiles) load_tile_at(tiles[k], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
+    ahd.advance();
   }
   int buf = 0;
   for (; tile < ntiles; tile += ncta, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
     const uint32_t ahead = tile + (kTileStages - 1) * ncta;
     const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;   // (buf + kTileStages - 1) % kTileStages
-    if (ahead < ntiles) load_tile_async(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
+    if (ahead < ntiles) load_tile_at(tiles[abuf], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
+    ahd.advance();
     cp_async_wait<kTileStages - 1>();   // this tile's group has landed
     __syncthreads();
     const uint4 (*s)[TC / 8] = tiles[buf];
-    int64_t tr, tc;
-    tile_coords(tile, a.tiles_c_div, tr, tc);
-    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const uint32_t tr = cur.tr, tc = cur.tc;
+    cur.advance();
+    const int64_t r0 = static_cast<int64_t>(tr) * TR, c0 = static_cast<int64_t>(tc) * TC;
     const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
     const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
+    const int64_t rblk_tile = r0 * nbr + c0 / 16;   // first row block of the tile
+    const int64_t cblk_tile = c0 * nbc + r0 / 16;   // first column block of the tile
 
     // scale-SR words of this thread's blocks: row a, row b, column 2cp, 2cp+1
     uint32_t w_ra = 0u, w_rb = 0u, w_ca = 0u, w_cb = 0u;
     if (share) {
-      uint64_t unit;
-      uint32_t c2;
-      if (j4 < 2) {   // row block units: row (t / 8) + 32 j4, blocks (t % 8) & ~3 ..
-        const int64_t grow = r0 + (t >> 3) + 32 * j4;
-        unit = (static_cast<uint64_t>(grow) * (C / 16) + c0 / 16 + ((t & 7) & ~3)) >> 2;
-        c2 = c2r;
-      } else {        // column units: column 2 (t / 4) + (j4 - 2), row blocks r0/16 ..
-        const int64_t gcol = c0 + 2 * (t >> 2) + (j4 - 2);
-        unit = (static_cast<uint64_t>(gcol) * (R / 16) + r0 / 16) >> 2;
-        c2 = c2c;
-      }
+      // row block units: row (t / 8) + 32 j4, blocks (t % 8) & ~3 ..; column
+      // units: column 2 (t / 4) + (j4 - 2), row blocks r0/16 ..
+      const uint64_t unit = static_cast<uint64_t>((j4 < 2 ? rblk_tile : cblk_tile) + share_thr) >> 2;
+      const uint32_t c2 = (j4 < 2) ? c2r : c2c;
       const uint4 d = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
       uint32_t got[4];   // got[r] = word j4 of the draw of lane (j4 + r) % 4
 #pragma unroll
@@ -671,9 +681,9 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         float2 v[16];
         unpack16x2_signed(a0, a1, b0, b1, sm, v);
         if constexpr (ROT) rht16x2_presigned(v);
-        const int64_t gra = r0 + row, grb = gra + 32, gcb = c0 / 16 + cb;
-        const uint64_t blka = static_cast<uint64_t>(gra) * (C / 16) + gcb;
-        const uint64_t blkb = static_cast<uint64_t>(grb) * (C / 16) + gcb;
+        const int64_t gra = r0 + row, grb = gra + 32;
+        const uint64_t blka = static_cast<uint64_t>(rblk_tile + rblk_thr);
+        const uint64_t blkb = blka + static_cast<uint64_t>(32 * nbr);
         Packed16 pa, pb;
         uint32_t sa, sb;
         if constexpr (VEC) {
@@ -691,14 +701,14 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         }
         // row gra's 8 code bytes, row grb's 32 rows further on; the scale
         // offsets split into a tile part and a thread part
-        uint8_t* crow = a.codes_row + gra * (C / 2) + 8 * gcb;
+        uint8_t* crow = a.codes_row + (r0 * (C / 2) + c0 / 2) + rcode_thr;
         if (va) *reinterpret_cast<uint2*>(crow) = make_uint2(pa.lo, pa.hi);
         if (vb) *reinterpret_cast<uint2*>(crow + 32 * (C / 2)) = make_uint2(pb.lo, pb.hi);
         if (a.scales_row) {
           uint8_t* srow = a.scales_row + (gemm ? gemm_scale_tile_row(tr, tc, C / 16) + gemm_scale_thread_row(row, cb)
                                                : static_cast<int64_t>(blka));
           if (va) srow[0] = static_cast<uint8_t>(sa);
-          if (vb) srow[gemm ? 4 : 32 * (C / 16)] = static_cast<uint8_t>(sb);
+          if (vb) srow[gemm ? 4 : 32 * nbr] = static_cast<uint8_t>(sb);
         }
       }
     }
@@ -715,22 +725,20 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
           v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
         }
         if constexpr (ROT) rht16x2_presigned(v);
-        const int64_t nbc = R / 16;
-        const int64_t gc = c0 + 2 * cp, grb = r0 / 16 + rb;
+        const int64_t gc = c0 + 2 * cp;
+        const uint64_t blka = static_cast<uint64_t>(cblk_tile + cblk_thr), blkb = blka + static_cast<uint64_t>(nbc);
         Packed16 qa, qb;
         uint32_t sa, sb;
         if constexpr (VEC) {
           // tensor scales of columns gc, gc + 1; the first tile row publishes them
           const float aa = vector_alpha(a, a.vmax_c, gc), ab = vector_alpha(a, a.vmax_c, gc + 1);
-          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
-                              static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca, w_cb);
           if (tr == 0 && rb == 0) {
             a.alpha_col[gc] = aa;
             a.alpha_col[gc + 1] = ab;
           }
         } else {
-          quantize_pair<MODE>(v, scc, K, c2c, static_cast<uint64_t>(gc) * nbc + grb,
-                              static_cast<uint64_t>(gc + 1) * nbc + grb, qa, qb, sa, sb, share, w_ca, w_cb);
+          quantize_pair<MODE>(v, scc, K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca, w_cb);
         }
         *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
@@ -742,11 +750,11 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         // whole tile: thread t copies 16 code bytes of column t / 2 and
         // threads 0..127 the 4-byte word of column t's four scales
         const int c = t >> 1, h = t & 1;
-        *reinterpret_cast<uint4*>(a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h) =
+        *reinterpret_cast<uint4*>(a.codes_col + (c0 * (R / 2) + r0 / 2) + ccode_thr) =
             *reinterpret_cast<const uint4*>(&colcodes[c][16 * h]);
         if (a.scales_col && t < TC) {
-          const int64_t off = gemm ? gemm_scale_tile_col(tr, tc, R / 16) + gemm_scale_thread_col(t)
-                                   : (c0 + t) * (R / 16) + r0 / 16;
+          const int64_t off = gemm ? gemm_scale_tile_col(tr, tc, nbc) + gemm_scale_thread_col(t)
+                                   : cblk_tile + t * nbc;
           *reinterpret_cast<uint32_t*>(a.scales_col + off) = *reinterpret_cast<const uint32_t*>(&colscale[t][0]);
         }
       } else {

@@ -46,11 +46,9 @@ __device__ __forceinline__ int tile_word_2d(int r, int w) { return (tile_chunk_2
 // Thread t copies chunk cc = t % 16 of rows t / 16 + 16 i (i < 4): one
 // 64-bit address for the first row, the others 16 rows apart.
 template <bool SW2D = false>
-__device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
-                                                int64_t ld, const FastDiv& tiles_c, uint32_t tile) {
-  int64_t tr, tc;
-  tile_coords(tile, tiles_c, tr, tc);
-  const int64_t r0 = tr * TR, c0 = tc * TC;
+__device__ __forceinline__ void load_tile_at(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
+                                             int64_t ld, uint32_t tr, uint32_t tc) {
+  const int64_t r0 = static_cast<int64_t>(tr) * TR, c0 = static_cast<int64_t>(tc) * TC;
   const int row0 = static_cast<int>(threadIdx.x) >> 4, cc = static_cast<int>(threadIdx.x) & 15;
   const uint16_t* src = x + (r0 + row0) * ld + c0 + 8 * cc;
   const int64_t step = 16 * ld;
@@ -72,5 +70,30 @@ __device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint
   }
   cp_async_commit();
 }
+
+template <bool SW2D = false>
+__device__ __forceinline__ void load_tile_async(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
+                                                int64_t ld, const FastDiv& tiles_c, uint32_t tile) {
+  int64_t tr, tc;
+  tile_coords(tile, tiles_c, tr, tc);
+  load_tile_at<SW2D>(buf, x, R, C, ld, static_cast<uint32_t>(tr), static_cast<uint32_t>(tc));
+}
+
+// Coordinates of the tiles a CTA visits (tile, tile + step, ...) in the
+// row-major grid of `tiles_c` tile columns, advanced without a division.
+struct TileWalk {
+  uint32_t tr, tc, dtr, dtc, tiles_c;
+  __device__ __forceinline__ TileWalk(uint32_t tile, uint32_t step, uint32_t cols)
+      : tr(tile / cols), tc(tile - (tile / cols) * cols), dtr(step / cols), dtc(step - (step / cols) * cols),
+        tiles_c(cols) {}
+  __device__ __forceinline__ void advance() {
+    tc += dtc;
+    tr += dtr;
+    if (tc >= tiles_c) {
+      tc -= tiles_c;
+      ++tr;
+    }
+  }
+};
 
 }  // namespace nvfp4
