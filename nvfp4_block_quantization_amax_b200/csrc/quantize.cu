@@ -218,21 +218,24 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   uint32_t hin = 0;   // per-halfword max of the input magnitudes (Inf / NaN check)
   uint32_t tile = cta;
   int buf = 0;
-  if (tile < ntiles) load_tile_async(tiles[0], x, R, C, ld, tiles_c, tile);
+  TileWalk cur(cta, ncta, tiles_c.d), nxt = cur;   // this tile and the next, without divisions
+  if (tile < ntiles) load_tile_at(tiles[0], x, R, C, ld, nxt.tr, nxt.tc);
+  nxt.advance();
   for (; tile < ntiles; tile += ncta, buf ^= 1) {
     const uint32_t next = tile + ncta;
     if (next < ntiles) {
-      load_tile_async(tiles[buf ^ 1], x, R, C, ld, tiles_c, next);
+      load_tile_at(tiles[buf ^ 1], x, R, C, ld, nxt.tr, nxt.tc);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
+    nxt.advance();
     __syncthreads();
     const uint4 (*s)[TC / 8] = tiles[buf];
-    int64_t tr, tc;
-    tile_coords(tile, tiles_c, tr, tc);
-    const int rows = static_cast<int>(R - tr * TR < TR ? R - tr * TR : TR);
-    const int cols = static_cast<int>(C - tc * TC < TC ? C - tc * TC : TC);
+    const int64_t r0 = static_cast<int64_t>(cur.tr) * TR, c0 = static_cast<int64_t>(cur.tc) * TC;
+    cur.advance();
+    const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
+    const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
     if constexpr (ROW) {
       // blocks (row, cb) and (row + 32, cb)
       const int row = t >> 3, cb = t & 7;
@@ -819,25 +822,30 @@ __device__ __forceinline__ void quant_tile_2d_body(const QuantArgs& a, uint32_t 
   // whole tiles write columns as 16-byte code pieces and 4-byte scale words
   const bool col_words = R % 64 == 0 && (reinterpret_cast<uintptr_t>(a.scales_col) & 3u) == 0;
 
+  // this tile and the one kTileStages - 1 iterations ahead, walked without
+  // divisions
+  TileWalk cur(cta, ncta, static_cast<uint32_t>(a.tiles_c)), ahd = cur;
   uint32_t tile = cta;
 #pragma unroll
   for (int k = 0; k < kTileStages - 1; ++k) {
     const uint32_t tk = tile + k * ncta;
-    if (tk < ntiles) load_tile_async<true>(tiles[k], a.x, R, C, a.ld, a.tiles_c_div, tk);
+    if (tk < ntiles) load_tile_at<true>(tiles[k], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
+    ahd.advance();
   }
   int buf = 0;
   for (; tile < ntiles; tile += ncta, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
     const uint32_t ahead = tile + (kTileStages - 1) * ncta;
     const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;
-    if (ahead < ntiles) load_tile_async<true>(tiles[abuf], a.x, R, C, a.ld, a.tiles_c_div, ahead);
+    if (ahead < ntiles) load_tile_at<true>(tiles[abuf], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
+    ahd.advance();
     cp_async_wait<kTileStages - 1>();
     __syncthreads();
     const uint4 (*s)[TC / 8] = tiles[buf];
-    int64_t tr, tc;
-    tile_coords(tile, a.tiles_c_div, tr, tc);
-    const int64_t r0 = tr * TR, c0 = tc * TC;
+    const uint32_t tr = cur.tr, tc = cur.tc;
+    cur.advance();
+    const int64_t r0 = static_cast<int64_t>(tr) * TR, c0 = static_cast<int64_t>(tc) * TC;
     const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);   // multiple of 16
     const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);   // multiple of 16
 
