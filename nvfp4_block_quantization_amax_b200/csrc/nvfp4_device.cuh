@@ -112,14 +112,15 @@ __device__ __forceinline__ uint32_t e4m3_ceil(float v) {
 //   Subnormal range [0, 2^-6): the grid step is 2^-9, so with t = 512 v
 //   (exact) lo = floor(t) and f = t - lo, both exact.
 __device__ __forceinline__ uint32_t e4m3_sr(float v, uint32_t u24) {
-  if (!(v < 448.0f)) return 0x7Eu;
   const uint32_t b = __float_as_uint(v);
   const uint32_t lo_n = (b >> 20) - (120u << 3);
   const uint32_t up_n = (u24 < ((b & 0xFFFFFu) << 4)) ? 1u : 0u;
   const float t = __fmul_rn(v, 512.0f);
   const float fl = floorf(t);
   const uint32_t up_s = (static_cast<float>(u24) < __fmul_rn(__fsub_rn(t, fl), 16777216.0f)) ? 1u : 0u;
-  return (v >= 0.015625f) ? lo_n + up_n : static_cast<uint32_t>(fl) + up_s;
+  // selects rather than early returns: no divergent branch per block
+  const uint32_t r = (v >= 0.015625f) ? lo_n + up_n : static_cast<uint32_t>(fl) + up_s;
+  return (v < 448.0f) ? r : 0x7Eu;
 }
 
 // ---------------------------------------------------------------------------
@@ -625,7 +626,8 @@ __device__ __forceinline__ VecScales make_vec_scales(float alpha_a, float alpha_
 
 // Eq. 2's quotient amax_b / den (0 when den is 0).
 __device__ __forceinline__ float scale_quot(float amax_b, float den) {
-  return (den == 0.0f) ? 0.0f : __fdiv_rn(amax_b, den);
+  const float q = __fdiv_rn(amax_b, den);   // computed either way: a select, not a branch
+  return (den == 0.0f) ? 0.0f : q;
 }
 
 // Codes of the two lane-paired blocks v * rinv (Eq. 3 as a reciprocal

@@ -321,8 +321,8 @@ constexpr int kColPitch = 48;   // bytes per staged column of codes (32 used; ro
 // ---------------------------------------------------------------------------
 // MS-EDEN scale of one block from its sums and its random word.
 __device__ __forceinline__ uint32_t eden_scale(float num, float den, uint32_t word) {
-  if (den == 0.0f) return 0u;
-  return e4m3_sr(__fdiv_rn(num, den), word >> 8);
+  const uint32_t sc = e4m3_sr(__fdiv_rn(num, den), word >> 8);   // a select, not a branch, on den == 0
+  return (den == 0.0f) ? 0u : sc;
 }
 
 // have_words: MS-EDEN only - wa / wb already hold the blocks' scale-SR words.
