@@ -68,6 +68,12 @@ constexpr uint32_t kTagValueSRHw = 4u; // one word per 4 elements for the hardwa
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// The same with the sign flipped where m = 0x80000000 (m is 0 or bit 31).
+// Adding bit 31 modulo 2^32 flips it exactly as an exclusive or does, and a
+// shift followed by an add is one instruction; the high half masks and
+// flips in one three-input logic operation.
+__device__ __forceinline__ float bf16lo_flip(uint32_t w, uint32_t m) { return __uint_as_float((w << 16) + m); }
+__device__ __forceinline__ float bf16hi_flip(uint32_t w, uint32_t m) { return __uint_as_float((w & 0xFFFF0000u) ^ m); }
 
 // 8 bf16 packed in a uint4 -> 8 floats
 __device__ __forceinline__ void unpack8(const uint4 u, float* v) {
@@ -203,13 +209,16 @@ __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
 // are sums (the butterflies): when b is itself a product, the compiler may
 // fold the two into one fma and drop the product's rounding, so a - RN(p)
 // uses sub2_exact (two scalar subtractions, which are never merged).
+// Measured on sm_100a: the code generator merges a packed product into a
+// packed add or subtract even when both are written in PTX with an explicit
+// .rn, so naming the rounding mode does not keep a packed pair apart.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 sub2_exact(float2 a, float2 b) {
   return make_float2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y));
 }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // Sign masks of the rotation's diagonal: bit 31 set where element i flips.
 struct SignMasks {
@@ -230,9 +239,8 @@ __device__ __forceinline__ void unpack16x2_signed(const uint4 a0, const uint4 a1
   const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    v[2 * j] = make_float2(__uint_as_float((wa[j] << 16) ^ sm.m[2 * j]), __uint_as_float((wb[j] << 16) ^ sm.m[2 * j]));
-    v[2 * j + 1] = make_float2(__uint_as_float((wa[j] & 0xFFFF0000u) ^ sm.m[2 * j + 1]),
-                               __uint_as_float((wb[j] & 0xFFFF0000u) ^ sm.m[2 * j + 1]));
+    v[2 * j] = make_float2(bf16lo_flip(wa[j], sm.m[2 * j]), bf16lo_flip(wb[j], sm.m[2 * j]));
+    v[2 * j + 1] = make_float2(bf16hi_flip(wa[j], sm.m[2 * j + 1]), bf16hi_flip(wb[j], sm.m[2 * j + 1]));
   }
 }
 

@@ -274,7 +274,7 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
         for (int i = 0; i < 16; ++i) {
           const uint32_t w = base[i * (TC / 2) + wofs];
           if constexpr (!ROW) hin = __vmaxu2(hin, w & 0x7FFF7FFFu);
-          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+          v[i] = make_float2(bf16lo_flip(w, sm.m[i]), bf16hi_flip(w, sm.m[i]));
         }
         hadamard16x2(v);
         float ma, mb;
@@ -725,7 +725,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint32_t w = base[i * (TC / 2) + wofs];
-          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+          v[i] = make_float2(bf16lo_flip(w, sm.m[i]), bf16hi_flip(w, sm.m[i]));
         }
         if constexpr (ROT) rht16x2_presigned(v);
         const int64_t gc = c0 + 2 * cp;
@@ -1165,7 +1165,7 @@ __global__ void __launch_bounds__(TNT) amax_vec_kernel(const QuantArgs a) {
         for (int i = 0; i < 16; ++i) {
           const uint32_t w = base[i * (TC / 2) + wofs];
           if constexpr (!ROW) hin = __vmaxu2(hin, w & 0x7FFF7FFFu);
-          v[i] = make_float2(__uint_as_float((w << 16) ^ sm.m[i]), __uint_as_float((w & 0xFFFF0000u) ^ sm.m[i]));
+          v[i] = make_float2(bf16lo_flip(w, sm.m[i]), bf16hi_flip(w, sm.m[i]));
         }
         if constexpr (ROT) hadamard16x2(v);
         float mx = 0.0f, my = 0.0f;
