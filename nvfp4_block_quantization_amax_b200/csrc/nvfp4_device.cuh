@@ -209,13 +209,35 @@ __device__ __forceinline__ void irht16(float* v, uint32_t signs) {
 // are sums (the butterflies): when b is itself a product, the compiler may
 // fold the two into one fma and drop the product's rounding, so a - RN(p)
 // uses sub2_exact (two scalar subtractions, which are never merged).
-// Measured on sm_100a: the code generator merges a packed product into a
-// packed add or subtract even when both are written in PTX with an explicit
-// .rn, so naming the rounding mode does not keep a packed pair apart.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// 1.0f that the code generator cannot treat as a constant: its sign and
+// exponent bits are ORed with %nsmid >> 31 (the SM count is a launch-time
+// value below 2^31, so the bit is always 0).  Hoisted: one read per kernel.
+__device__ __forceinline__ float opaque_one() {
+  uint32_t n;
+  asm("mov.u32 %0, %%nsmid;" : "=r"(n));
+  return __uint_as_float(0x3F800000u | (n >> 31));
+}
+__device__ __forceinline__ float2 fma2_ptx(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+// a + p, packed, for a product p that must keep its own rounding:
+// fma(p, 1, a) adds exactly (p * 1 is exact) with one rounding, and with the
+// factor opaque the code generator can neither drop it nor merge p's
+// multiply into the fma (measured on sm_100a: with a literal 1.0 it does
+// both, and it also merges into add.rn.f32x2 / sub.rn.f32x2).
+__device__ __forceinline__ float2 add2_prod(float2 a, float2 p) {
+  const float u = opaque_one();
+  return fma2_ptx(p, make_float2(u, u), a);
+}
 __device__ __forceinline__ float2 sub2_exact(float2 a, float2 b) {
   return make_float2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y));
 }
@@ -467,11 +489,17 @@ __device__ __forceinline__ void decode16x2(const Packed16& pa, const Packed16& p
 // made e[] may be contracted with a packed add into one fma (measured: the
 // rounding of d * d vanished from 4/6 errors), so the first level, which
 // consumes the products, adds with the scalar __fadd_rn, which is never
-// merged; the later levels add sums only.
+// merged (or, with PACKED, with add2_prod); the later levels add sums only.
+// PACKED measured faster for the MS-EDEN sums (225 vs 229 us for the dY
+// rows + columns kernel) and slower for the 4/6 errors (the packed fma
+// loads the busier FMA pipe).
+template <bool PACKED = false>
 __device__ __forceinline__ float2 sum16x2(const float2* e) {
   float2 t[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = make_float2(__fadd_rn(e[i].x, e[i + 8].x), __fadd_rn(e[i].y, e[i + 8].y));
+  for (int i = 0; i < 8; ++i)
+    t[i] = PACKED ? add2_prod(e[i + 8], e[i])
+                  : make_float2(__fadd_rn(e[i].x, e[i + 8].x), __fadd_rn(e[i].y, e[i + 8].y));
 #pragma unroll
   for (int i = 0; i < 4; ++i) t[i] = add2(t[i], t[i + 4]);
 #pragma unroll

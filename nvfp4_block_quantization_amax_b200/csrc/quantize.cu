@@ -350,8 +350,8 @@ __device__ __forceinline__ void quantize_pair(const float2* v, const S& c, const
       rr[i] = mul2(v[i], v[i]);
       rq[i] = mul2(v[i], q[i]);
     }
-    const float2 num = sum16x2(rr);
-    const float2 den = mul2(c.alpha2(), sum16x2(rq));
+    const float2 num = sum16x2<true>(rr);
+    const float2 den = mul2(c.alpha2(), sum16x2<true>(rq));
     if (!have_words) {
       const uint64_t ua = blka >> 2, ub = blkb >> 2;
       const uint4 da = philox(K, static_cast<uint32_t>(ua), static_cast<uint32_t>(ua >> 32), c2, kTagScaleSR);
@@ -583,8 +583,8 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   // 4k .. 4k+3 of a warp hold the same two row-block units and the same two
   // column-block units of a tile (when C and R are multiples of 64, so units
   // never straddle a row or a column), each lane needing word (lane % 4) of
-  // all four draws: each lane computes one draw and a 4 x 4 shuffle
-  // transpose hands the words out.
+  // all four draws: each lane computes one draw, stores it in its warp's
+  // slice of the column staging and reads its words back.
   const bool share = MODE == kModeMsEden && (!ROW || C % 64 == 0) && (!COL || R % 64 == 0);
   const int lane = t & 31, j4 = t & 3;
   // whole tiles write columns as 16-byte code pieces and 4-byte scale words
@@ -640,21 +640,20 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
       const uint64_t unit = static_cast<uint64_t>((j4 < 2 ? rblk_tile : cblk_tile) + share_thr) >> 2;
       const uint32_t c2 = (j4 < 2) ? c2r : c2c;
       const uint4 d = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
-      uint32_t got[4];   // got[r] = word j4 of the draw of lane (j4 + r) % 4
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int wi = (j4 - r) & 3;
-        const uint32_t send = wi == 0 ? d.x : (wi == 1 ? d.y : (wi == 2 ? d.z : d.w));
-        got[r] = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((j4 + r) & 3));
-      }
-      auto pick = [&](int dj) {
-        const int r = (dj - j4) & 3;
-        return r == 0 ? got[0] : (r == 1 ? got[1] : (r == 2 ? got[2] : got[3]));
-      };
-      w_ra = pick(0);
-      w_rb = pick(1);
-      w_ca = pick(2);
-      w_cb = pick(3);
+      // warp w's slice: 512 bytes at the start of colcodes rows 16 w .., the
+      // rows only warp w writes (column pass) and reads (write-out) in this
+      // tile, free until its column pass; the previous tile's write-out read
+      // them before the barrier at the top of this iteration
+      uint4* xs = reinterpret_cast<uint4*>(&colcodes[16 * (t >> 5)][0]);
+      xs[lane] = d;
+      __syncwarp();
+      // word j4 of the draws of quad lanes 0..3
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(xs + (lane & ~3)) + j4;
+      w_ra = xw[0];
+      w_rb = xw[4];
+      w_ca = xw[8];
+      w_cb = xw[12];
+      __syncwarp();   // every lane has read before the column pass rewrites the rows
     }
 
     if (check) {
