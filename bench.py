@@ -178,10 +178,19 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # the step
 # --------------------------------------------------------------------------
+def carve(buf, shapes):
+    """Consecutive row-major views of the given shapes in a 1-D buffer."""
+    views, o = [], 0
+    for r, c in shapes:
+        views.append(buf[o:o + r * c].view(r, c))
+        o += r * c
+    return views
+
+
 class LayerStep:
     """Pre-allocated buffers and the C-ABI call sequence of one step."""
 
-    def __init__(self, x, w, dy, bwd_mode, device, shared_amax=True):
+    def __init__(self, x, w, dy, bwd_mode, device, shared_amax=True, results=None):
         import torch
         from nvfp4_block_quantization_amax_b200 import api
         self.api = api
@@ -209,9 +218,11 @@ class LayerStep:
             t = src[name]
             self.out[name] = api.alloc_outputs(t.shape[0], t.shape[1], flags, device)
             self.ws[name] = api.workspace_for(t.shape[0], t.shape[1], flags, device)
-        self.y = torch.empty((T, O), dtype=torch.bfloat16, device=device)
-        self.dx = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-        self.dw = torch.empty((O, H), dtype=torch.bfloat16, device=device)
+        # results: optionally one contiguous bf16 buffer holding Y, dX, dW
+        if results is None:
+            results = torch.empty(T * O + T * H + O * H, dtype=torch.bfloat16, device=device)
+        self.y, self.dx, self.dw = carve(results, [(T, O), (T, H), (O, H)])
+        self.results = results
         self.ev = None
 
     def quantize(self, name, mode, flags, seed, sid, amax=None):
@@ -515,14 +526,25 @@ def run_device(args, rank, world, local_rank):
     # --- end to end: pinned host inputs in, results back to pinned host ---
     # Every step copies its inputs in and its results out; the copies run on
     # their own streams (one per direction) and overlap the compute of the
-    # neighbouring steps, two sets of device buffers taking turns.
-    hx, hw, hdy = (t.cpu().pin_memory() for t in (x, w, dy))
-    hy = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
-    hdx = torch.empty(step.dx.shape, dtype=torch.bfloat16).pin_memory()
-    hdw = torch.empty(step.dw.shape, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(4, min(args.steps, 12))
-    sets = [step, LayerStep(torch.empty_like(x), torch.empty_like(w), torch.empty_like(dy), bwd, device,
-                            shared_amax=not args.amax_per_call)]
+    # neighbouring steps, two sets of device buffers taking turns.  A step's
+    # inputs X, W, dY sit in one buffer and its results Y, dX, dW in another,
+    # so each direction is one copy per step (measured about 2% faster than
+    # three copies each way).
+    T_, H_ = x.shape
+    O_ = w.shape[0]
+    in_shapes, out_shapes = [(T_, H_), (O_, H_), (T_, O_)], [(T_, O_), (T_, H_), (O_, H_)]
+    n_in, n_out = sum(r * c for r, c in in_shapes), sum(r * c for r, c in out_shapes)
+    h_in = torch.empty(n_in, dtype=torch.bfloat16).pin_memory()
+    for v, t in zip(carve(h_in, in_shapes), (x, w, dy)):
+        v.copy_(t.cpu())
+    h_out = torch.empty(n_out, dtype=torch.bfloat16).pin_memory()
+    # 32 steps: the one pipeline fill and drain in the timed region weighs 1/32
+    e2e_steps = max(4, min(args.steps, 32))
+    sets = []
+    for _ in range(2):
+        d_in = torch.empty(n_in, dtype=torch.bfloat16, device=device)
+        sets.append((LayerStep(*carve(d_in, in_shapes), bwd, device, shared_amax=not args.amax_per_call,
+                               results=torch.empty(n_out, dtype=torch.bfloat16, device=device)), d_in))
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     comp = torch.cuda.current_stream(device)
 
@@ -530,13 +552,11 @@ def run_device(args, rank, world, local_rank):
         done_compute, done_out = [None, None], [None, None]
         for i in range(n):
             k = i % 2
-            b = sets[k]
+            b, d_in = sets[k]
             with torch.cuda.stream(s_in):
                 if done_compute[k] is not None:   # the set's previous step has read its inputs
                     s_in.wait_event(done_compute[k])
-                b.x.copy_(hx, non_blocking=True)
-                b.w.copy_(hw, non_blocking=True)
-                b.dy.copy_(hdy, non_blocking=True)
+                d_in.copy_(h_in, non_blocking=True)
                 e_in = torch.cuda.Event()
                 e_in.record(s_in)
             comp.wait_event(e_in)
@@ -548,9 +568,7 @@ def run_device(args, rank, world, local_rank):
             done_compute[k] = e_c
             with torch.cuda.stream(s_out):
                 s_out.wait_event(e_c)
-                hy.copy_(b.y, non_blocking=True)
-                hdx.copy_(b.dx, non_blocking=True)
-                hdw.copy_(b.dw, non_blocking=True)
+                h_out.copy_(b.results, non_blocking=True)
                 e_o = torch.cuda.Event()
                 e_o.record(s_out)
                 done_out[k] = e_o
@@ -583,8 +601,8 @@ def run_device(args, rank, world, local_rank):
     q_gelem = q_elems / (quant_ms * 1e-3) / 1e9
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
     traffic = gemm_traffic_record()
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
-    d2h = sum(t.numel() * t.element_size() for t in (hy, hdx, hdw))
+    h2d = h_in.numel() * h_in.element_size()
+    d2h = h_out.numel() * h_out.element_size()
     per_call = {k: round(1e3 * sum(s.elapsed_time(e) for s, e in timers[k]) / args.steps, 2)
                 for k in QUANT_CALLS + GEMM_CALLS}
     result = {
@@ -632,7 +650,7 @@ def run_device(args, rank, world, local_rank):
         result["quantize_roofline"] = quantize_roofline(qrec, quant_ms, clocks["sm_mhz"], n_sm, hbm)
     else:
         result["quantize_roofline"] = None
-    del hx, hw, hdy, hy, hdx, hdw
+    del h_in, h_out
     if not args.no_extras:
         result.update(run_extras(args, step, x, w, dy, device, hbm, fp4_peak))
     return result
