@@ -205,7 +205,10 @@ __device__ __forceinline__ void amax_plain_body(const uint16_t* __restrict__ x, 
 // max |x|, from the same per-halfword maximum the Inf / NaN check keeps),
 // [1] (rotated rows) and [2] (rotated columns), zeroed by the launcher,
 // instead of being stored as partials.
-template <bool ROW, bool COL>
+// NT threads per CTA (256 or 128): with 128 each thread takes two row pairs
+// and two column units of every tile, so the per-tile work (tile walk,
+// copies, barrier) is spread over twice the elements.
+template <bool ROW, bool COL, int NT = TNT>
 __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, int64_t R, int64_t C, int64_t ld,
                                                FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
                                                uint32_t* __restrict__ part_r, uint32_t* __restrict__ part_c,
@@ -219,12 +222,14 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   uint32_t tile = cta;
   int buf = 0;
   TileWalk cur(cta, ncta, tiles_c.d), nxt = cur;   // this tile and the next, without divisions
-  if (tile < ntiles) load_tile_at(tiles[0], x, R, C, ld, nxt.tr, nxt.tc);
+  static_assert(NT == 256 || NT == 128, "256 or 128 threads");
+  constexpr int kReps = 256 / NT;   // row pairs and column units per thread and tile
+  if (tile < ntiles) load_tile_at<false, NT>(tiles[0], x, R, C, ld, nxt.tr, nxt.tc);
   nxt.advance();
   for (; tile < ntiles; tile += ncta, buf ^= 1) {
     const uint32_t next = tile + ncta;
     if (next < ntiles) {
-      load_tile_at(tiles[buf ^ 1], x, R, C, ld, nxt.tr, nxt.tc);
+      load_tile_at<false, NT>(tiles[buf ^ 1], x, R, C, ld, nxt.tr, nxt.tc);
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
@@ -237,8 +242,10 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
     const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
     const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
     if constexpr (ROW) {
+#pragma unroll
+      for (int rep = 0; rep < kReps; ++rep) {
       // blocks (row, cb) and (row + 32, cb)
-      const int row = t >> 3, cb = t & 7;
+      const int row = (t >> 3) + (NT / 8) * rep, cb = t & 7;
       const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
       const uint4 a0 = s[row][tile_chunk(row, 2 * cb)], a1 = s[row][tile_chunk(row, 2 * cb + 1)];
       const uint4 b0 = s[row + 32][tile_chunk(row + 32, 2 * cb)];
@@ -262,10 +269,13 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
       max_abs16x2(v, ma, mb);
       if (va) mr = fmaxf(mr, ma);
       if (vb) mr = fmaxf(mr, mb);
+      }
     }
     if constexpr (COL) {
+#pragma unroll
+      for (int rep = 0; rep < kReps; ++rep) {
       // columns (2 cp, 2 cp + 1) of row block rb: one 32-bit word per row
-      const int cp = t & 63, rb = t >> 6;
+      const int cp = t & 63, rb = (t >> 6) + (NT / 64) * rep;
       if (16 * rb < rows && 2 * cp < cols) {
         const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
         const int wofs = tile_word(16 * rb, cp);   // the same for all 16 rows of the block
@@ -281,13 +291,14 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
         max_abs16x2(v, ma, mb);
         mc = max3(mc, ma, mb);
       }
+      }
     }
     __syncthreads();   // buf is refilled two iterations from now
   }
   const uint32_t h = max(hin & 0xFFFFu, hin >> 16);
   const bool bad = h >= 0x7F80u;
   if (atomic_out) {
-    const uint32_t mp = block_max_u32<TNT>(bad ? kNonFinite : (h << 16), red);
+    const uint32_t mp = block_max_u32<NT>(bad ? kNonFinite : (h << 16), red);
     if (t == 0) {
       atomicMax(atomic_out, mp);
       if (mp == kNonFinite && status) *status = kStatusNonFinite;
@@ -295,7 +306,7 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   }
   if constexpr (ROW) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mr, 0.25f));
-    m = block_max_u32<TNT>(m, red);
+    m = block_max_u32<NT>(m, red);
     if (t == 0) {
       if (atomic_out) atomicMax(atomic_out + 1, m);
       else part_r[cta] = m;
@@ -303,7 +314,7 @@ __device__ __forceinline__ void amax_tile_body(const uint16_t* __restrict__ x, i
   }
   if constexpr (COL) {
     uint32_t m = bad ? kNonFinite : __float_as_uint(__fmul_rn(mc, 0.25f));
-    m = block_max_u32<TNT>(m, red);
+    m = block_max_u32<NT>(m, red);
     if (t == 0) {
       if (atomic_out) atomicMax(atomic_out + 2, m);
       else part_c[cta] = m;
@@ -1036,27 +1047,30 @@ __global__ void __launch_bounds__(NT) amax_plain_atomic_kernel(const uint16_t* _
   amax_plain_body<NT>(x, R, ld, cpr, nullptr, blockIdx.x, gridDim.x, red, out, status);
 }
 
+// Threads per CTA of the rotated amax kernels (two units per thread and tile).
+constexpr int kAmaxNT = 128;
+
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT) amax_tile_atomic_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                               int64_t ld, FastDiv tiles_c, uint32_t ntiles,
-                                                               uint64_t seed, uint32_t* __restrict__ out,
-                                                               int32_t* status) {
+__global__ void __launch_bounds__(kAmaxNT) amax_tile_atomic_kernel(const uint16_t* __restrict__ x, int64_t R,
+                                                                   int64_t C, int64_t ld, FastDiv tiles_c,
+                                                                   uint32_t ntiles, uint64_t seed,
+                                                                   uint32_t* __restrict__ out, int32_t* status) {
   pdl_entry();
   __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
-  __shared__ uint32_t red[TNT / 32];
-  amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, nullptr, nullptr, blockIdx.x, gridDim.x, ring, red,
+  __shared__ uint32_t red[kAmaxNT / 32];
+  amax_tile_body<ROW, COL, kAmaxNT>(x, R, C, ld, tiles_c, ntiles, seed, nullptr, nullptr, blockIdx.x, gridDim.x, ring, red,
                            out, status);
 }
 
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(TNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
-                                                        int64_t ld, FastDiv tiles_c, uint32_t ntiles, uint64_t seed,
-                                                        uint32_t* __restrict__ part_r,
-                                                        uint32_t* __restrict__ part_c) {
+__global__ void __launch_bounds__(kAmaxNT) amax_tile_kernel(const uint16_t* __restrict__ x, int64_t R, int64_t C,
+                                                            int64_t ld, FastDiv tiles_c, uint32_t ntiles,
+                                                            uint64_t seed, uint32_t* __restrict__ part_r,
+                                                            uint32_t* __restrict__ part_c) {
   pdl_entry();
   __shared__ __align__(16) uint8_t ring[2 * kTileBytes];
-  __shared__ uint32_t red[TNT / 32];
-  amax_tile_body<ROW, COL>(x, R, C, ld, tiles_c, ntiles, seed, part_r, part_c, blockIdx.x, gridDim.x, ring, red);
+  __shared__ uint32_t red[kAmaxNT / 32];
+  amax_tile_body<ROW, COL, kAmaxNT>(x, R, C, ld, tiles_c, ntiles, seed, part_r, part_c, blockIdx.x, gridDim.x, ring, red);
 }
 
 template <int MODE, bool ROT, int NT, bool VEC>
@@ -1460,11 +1474,11 @@ static cudaError_t launch_amax(const QuantArgs& a, bool row, bool col, bool rot,
     const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
     const FastDiv tcd = a.tiles_c_div;
     if (row && col)
-      launch_k(amax_tile_kernel<true, true>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<true, true>, dim3(np), dim3(kAmaxNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else if (row)
-      launch_k(amax_tile_kernel<true, false>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<true, false>, dim3(np), dim3(kAmaxNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
     else
-      launch_k(amax_tile_kernel<false, true>, dim3(np), dim3(TNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
+      launch_k(amax_tile_kernel<false, true>, dim3(np), dim3(kAmaxNT), 0, st, 1u, a.x, a.R, a.C, a.ld, tcd, ntiles, a.seed, pr, pc);
   }
   note_launch();
   return cudaGetLastError();
@@ -1489,13 +1503,13 @@ cudaError_t amax_launch(const void* x, int64_t R, int64_t C, int64_t ld, uint32_
     const uint32_t ntiles = static_cast<uint32_t>(tiles_r * tiles_c);
     const FastDiv tcd = make_fastdiv(static_cast<uint32_t>(tiles_c));
     if (row && col)
-      launch_k(amax_tile_atomic_kernel<true, true>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+      launch_k(amax_tile_atomic_kernel<true, true>, dim3(np), dim3(kAmaxNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
                out, status);
     else if (row)
-      launch_k(amax_tile_atomic_kernel<true, false>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+      launch_k(amax_tile_atomic_kernel<true, false>, dim3(np), dim3(kAmaxNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
                out, status);
     else
-      launch_k(amax_tile_atomic_kernel<false, true>, dim3(np), dim3(TNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
+      launch_k(amax_tile_atomic_kernel<false, true>, dim3(np), dim3(kAmaxNT), 0, st, 1u, xs, R, C, ld, tcd, ntiles, seed,
                out, status);
   }
   note_launch();

@@ -42,28 +42,30 @@ __device__ __forceinline__ int tile_chunk_2d(int r, int c) { return c ^ (r & 7);
 __device__ __forceinline__ int tile_word_2d(int r, int w) { return (tile_chunk_2d(r, w >> 2) << 2) | (w & 3); }
 
 // Issue the copies of tile `tile` (row-major tile grid) into buf, in the
-// 1D (SW2D = false) or the 2D-block (SW2D = true) layout.
-// Thread t copies chunk cc = t % 16 of rows t / 16 + 16 i (i < 4): one
-// 64-bit address for the first row, the others 16 rows apart.
-template <bool SW2D = false>
+// 1D (SW2D = false) or the 2D-block (SW2D = true) layout, by NT threads.
+// Thread t copies chunk cc = t % 16 of rows t / 16 + (NT / 16) i
+// (i < 16 TR / NT): one 64-bit address for the first row, the others NT / 16
+// rows apart.
+template <bool SW2D = false, int NT = TNT>
 __device__ __forceinline__ void load_tile_at(uint4 (*buf)[TC / 8], const uint16_t* x, int64_t R, int64_t C,
                                              int64_t ld, uint32_t tr, uint32_t tc) {
+  constexpr int kRowStep = NT / 16, kPasses = TR / kRowStep;
   const int64_t r0 = static_cast<int64_t>(tr) * TR, c0 = static_cast<int64_t>(tc) * TC;
   const int row0 = static_cast<int>(threadIdx.x) >> 4, cc = static_cast<int>(threadIdx.x) & 15;
   const uint16_t* src = x + (r0 + row0) * ld + c0 + 8 * cc;
-  const int64_t step = 16 * ld;
+  const int64_t step = kRowStep * ld;
   if (R - r0 >= TR && C - c0 >= TC) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = row0 + 16 * i;
+    for (int i = 0; i < kPasses; ++i) {
+      const int row = row0 + kRowStep * i;
       cp_async16(&buf[row][SW2D ? tile_chunk_2d(row, cc) : tile_chunk(row, cc)], src + i * step);
     }
   } else {
     const int rows = static_cast<int>(R - r0 < TR ? R - r0 : TR);
     const int cols = static_cast<int>(C - c0 < TC ? C - c0 : TC);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int row = row0 + 16 * i;
+    for (int i = 0; i < kPasses; ++i) {
+      const int row = row0 + kRowStep * i;
       if (row < rows && 8 * cc < cols)
         cp_async16(&buf[row][SW2D ? tile_chunk_2d(row, cc) : tile_chunk(row, cc)], src + i * step);
     }
