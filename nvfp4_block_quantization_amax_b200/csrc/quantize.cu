@@ -548,8 +548,16 @@ constexpr int kTileBytes = TR * TC * 2;
 
 // Resident CTAs per SM the register budget is sized for: the kernels are
 // bound by the latency of dependent arithmetic, so more warps help.
+// Threads per CTA of the 1D tile kernels: RTN and hardware-SR run 128-thread
+// CTAs (two units of each orientation per thread and tile, five CTAs per SM
+// by shared memory), measured 3-4% faster; the modes with more arithmetic
+// per block keep 256 threads, where the extra registers of two units cost
+// more than the shared per-tile work saves (4/6 rows + columns +13%, RHT + SR
+// +26% at 128).
 template <int MODE>
-constexpr int tile_1d_min_blocks() { return (MODE == kModeRTN) ? 4 : 3; }
+constexpr int tile_1d_threads() { return (MODE == kModeRTN || MODE == kModeRhtSRHw) ? 128 : 256; }
+template <int MODE>
+constexpr int tile_1d_min_blocks() { return tile_1d_threads<MODE>() == 128 ? 5 : 3; }
 
 // Shared memory of the tile kernels besides the tile ring.
 struct TileStaging {
@@ -561,7 +569,9 @@ struct TileStaging {
   float2 tab_c[kScaleTab];           // the same for the column orientation
 };
 
-template <int MODE, bool ROT, bool ROW, bool COL, bool VEC = false>
+// NT threads per CTA (256 or 128): with 128 each thread takes two row pairs
+// and two column pairs of every tile (kReps units of each).
+template <int MODE, bool ROT, bool ROW, bool COL, bool VEC = false, int NT = TNT>
 __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t cta, uint32_t ncta, uint8_t* ring,
                                                    TileStaging& stg) {
   auto tiles = reinterpret_cast<uint4(*)[TR][TC / 8]>(ring);
@@ -570,9 +580,9 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   uint32_t* red = stg.red;
   float alpha_r = 0.0f, alpha_c = 0.0f;
   if constexpr (!VEC) {
-    resolve_alpha<TNT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
-    if constexpr (ROW) build_scale_tab<TNT>(stg.tab_r, alpha_r);
-    if constexpr (COL) build_scale_tab<TNT>(stg.tab_c, alpha_c);
+    resolve_alpha<NT>(a, ROW, COL, ROW, COL, alpha_r, alpha_c, red, cta);
+    if constexpr (ROW) build_scale_tab<NT>(stg.tab_r, alpha_r);
+    if constexpr (COL) build_scale_tab<NT>(stg.tab_c, alpha_c);
     __syncthreads();
   }
   const TabScales scr = make_scale_ctx(stg.tab_r, alpha_r), scc = make_scale_ctx(stg.tab_c, alpha_c);
@@ -598,6 +608,8 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   // slice of the column staging and reads its words back.
   const bool share = MODE == kModeMsEden && (!ROW || C % 64 == 0) && (!COL || R % 64 == 0);
   const int lane = t & 31, j4 = t & 3;
+  static_assert(NT == 256 || NT == 128, "256 or 128 threads");
+  constexpr int kReps = 256 / NT;
   // whole tiles write columns as 16-byte code pieces and 4-byte scale words
   // (R % 64 == 0 keeps both aligned)
   const bool col_words = R % 64 == 0 && (reinterpret_cast<uintptr_t>(a.scales_col) & 3u) == 0;
@@ -605,12 +617,15 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   // Per-thread parts of the block indices and offsets, fixed for the whole
   // kernel: rows t/8 and t/8 + 32 of block column t%8 (row orientation);
   // columns 2 (t/4), +1 of row block t%4 and, in the write-out, column t/2
-  // (column orientation).  A tile adds its own part once.
+  // (column orientation); unit k of kReps adds NT/8 rows, NT/4 column pairs
+  // and NT/2 write-out columns.  A tile adds its own part once.
   const int64_t nbr = C / 16, nbc = R / 16;
   const int trow = t >> 3, tcb = t & 7, tcp = t >> 2, trb = t & 3;
   const int64_t rblk_thr = trow * nbr + tcb, rcode_thr = trow * (C / 2) + 8 * tcb;
   const int64_t cblk_thr = 2 * tcp * nbc + trb, ccode_thr = (t >> 1) * (R / 2) + 16 * (t & 1);
   const int64_t share_thr = (j4 < 2) ? (trow + 32 * j4) * nbr + (tcb & ~3) : (2 * tcp + (j4 - 2)) * nbc;
+  const int64_t rep_rblk = (NT / 8) * nbr, rep_rcode = (NT / 8) * (C / 2), rep_cblk = 2 * (NT / 4) * nbc;
+  const int64_t rep_share = (j4 < 2) ? rep_rblk : rep_cblk, rep_ccode = (NT / 2) * (R / 2);
   // this tile and the one kTileStages - 1 iterations ahead, walked without
   // divisions
   TileWalk cur(cta, ncta, static_cast<uint32_t>(a.tiles_c)), ahd = cur;
@@ -621,7 +636,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
 #pragma unroll
   for (int k = 0; k < kTileStages - 1; ++k) {
     const uint32_t tk = tile + k * ncta;
-    if (tk < ntiles) load_tile_at(tiles[k], a.x, R, C, a.ld, ahd.tr, ahd.tc);
+    if (tk < ntiles) load_tile_at<false, NT>(tiles[k], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
     ahd.advance();
   }
@@ -629,7 +644,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
   for (; tile < ntiles; tile += ncta, buf = (buf + 1 == kTileStages) ? 0 : buf + 1) {
     const uint32_t ahead = tile + (kTileStages - 1) * ncta;
     const int abuf = (buf == 0) ? kTileStages - 1 : buf - 1;   // (buf + kTileStages - 1) % kTileStages
-    if (ahead < ntiles) load_tile_at(tiles[abuf], a.x, R, C, a.ld, ahd.tr, ahd.tc);
+    if (ahead < ntiles) load_tile_at<false, NT>(tiles[abuf], a.x, R, C, a.ld, ahd.tr, ahd.tc);
     else cp_async_commit();
     ahd.advance();
     cp_async_wait<kTileStages - 1>();   // this tile's group has landed
@@ -644,34 +659,39 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
     const int64_t cblk_tile = c0 * nbc + r0 / 16;   // first column block of the tile
 
     // scale-SR words of this thread's blocks: row a, row b, column 2cp, 2cp+1
-    uint32_t w_ra = 0u, w_rb = 0u, w_ca = 0u, w_cb = 0u;
+    // (per unit)
+    uint32_t w_ra[kReps] = {}, w_rb[kReps] = {}, w_ca[kReps] = {}, w_cb[kReps] = {};
     if (share) {
-      // row block units: row (t / 8) + 32 j4, blocks (t % 8) & ~3 ..; column
-      // units: column 2 (t / 4) + (j4 - 2), row blocks r0/16 ..
-      const uint64_t unit = static_cast<uint64_t>((j4 < 2 ? rblk_tile : cblk_tile) + share_thr) >> 2;
-      const uint32_t c2 = (j4 < 2) ? c2r : c2c;
-      const uint4 d = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
-      // warp w's slice: 512 bytes at the start of colcodes rows 16 w .., the
-      // rows only warp w writes (column pass) and reads (write-out) in this
-      // tile, free until its column pass; the previous tile's write-out read
-      // them before the barrier at the top of this iteration
-      uint4* xs = reinterpret_cast<uint4*>(&colcodes[16 * (t >> 5)][0]);
-      xs[lane] = d;
-      __syncwarp();
-      // word j4 of the draws of quad lanes 0..3
-      const uint32_t* xw = reinterpret_cast<const uint32_t*>(xs + (lane & ~3)) + j4;
-      w_ra = xw[0];
-      w_rb = xw[4];
-      w_ca = xw[8];
-      w_cb = xw[12];
+#pragma unroll
+      for (int k = 0; k < kReps; ++k) {
+        // row block units: row (t / 8) + 32 j4, blocks (t % 8) & ~3 ..;
+        // column units: column 2 (t / 4) + (j4 - 2), row blocks r0/16 ..
+        const uint64_t unit = static_cast<uint64_t>((j4 < 2 ? rblk_tile : cblk_tile) + share_thr + k * rep_share) >> 2;
+        const uint32_t c2 = (j4 < 2) ? c2r : c2c;
+        const uint4 d = philox(K, static_cast<uint32_t>(unit), static_cast<uint32_t>(unit >> 32), c2, kTagScaleSR);
+        // warp w's slice for unit k: 512 bytes at the start of colcodes rows
+        // 16 w + (NT / 2) k .., rows only warp w writes (column pass) and
+        // reads (write-out) in this tile, free until its column pass; the
+        // previous tile's write-out read them before the barrier at the top
+        // of this iteration
+        uint4* xs = reinterpret_cast<uint4*>(&colcodes[16 * (t >> 5) + (NT / 2) * k][0]);
+        xs[lane] = d;
+        __syncwarp();
+        // word j4 of the draws of quad lanes 0..3
+        const uint32_t* xw = reinterpret_cast<const uint32_t*>(xs + (lane & ~3)) + j4;
+        w_ra[k] = xw[0];
+        w_rb[k] = xw[4];
+        w_ca[k] = xw[8];
+        w_cb[k] = xw[12];
+      }
       __syncwarp();   // every lane has read before the column pass rewrites the rows
     }
 
     if (check) {
       uint32_t hin = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int ch = t + TNT * i;
+      for (int i = 0; i < (TR * TC / 8) / NT; ++i) {
+        const int ch = t + NT * i;
         const int row = ch >> 4, cc = ch & 15;
         if (row < rows && 8 * cc < cols) {
           const uint4 u = s[row][tile_chunk(row, cc)];
@@ -685,7 +705,9 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
     }
 
     if constexpr (ROW) {
-      const int row = t >> 3, cb = t & 7;
+#pragma unroll
+      for (int k = 0; k < kReps; ++k) {
+      const int row = trow + (NT / 8) * k, cb = tcb;
       const bool va = row < rows && 16 * cb < cols, vb = row + 32 < rows && 16 * cb < cols;
       if (va || vb) {
         const uint4 a0 = s[row][tile_chunk(row, 2 * cb)], a1 = s[row][tile_chunk(row, 2 * cb + 1)];
@@ -695,7 +717,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         unpack16x2_signed(a0, a1, b0, b1, sm, v);
         if constexpr (ROT) rht16x2_presigned(v);
         const int64_t gra = r0 + row, grb = gra + 32;
-        const uint64_t blka = static_cast<uint64_t>(rblk_tile + rblk_thr);
+        const uint64_t blka = static_cast<uint64_t>(rblk_tile + rblk_thr + k * rep_rblk);
         const uint64_t blkb = blka + static_cast<uint64_t>(32 * nbr);
         Packed16 pa, pb;
         uint32_t sa, sb;
@@ -704,17 +726,17 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
           // column publish them
           const float aa = va ? vector_alpha(a, a.vmax_r, gra) : 0.0f;
           const float ab = vb ? vector_alpha(a, a.vmax_r, grb) : aa;
-          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra[k], w_rb[k]);
           if (tc == 0 && cb == 0) {
             if (va) a.alpha_row[gra] = aa;
             if (vb) a.alpha_row[grb] = ab;
           }
         } else {
-          quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra, w_rb);
+          quantize_pair<MODE>(v, scr, K, c2r, blka, blkb, pa, pb, sa, sb, share, w_ra[k], w_rb[k]);
         }
         // row gra's 8 code bytes, row grb's 32 rows further on; the scale
         // offsets split into a tile part and a thread part
-        uint8_t* crow = a.codes_row + (r0 * (C / 2) + c0 / 2) + rcode_thr;
+        uint8_t* crow = a.codes_row + (r0 * (C / 2) + c0 / 2) + rcode_thr + k * rep_rcode;
         if (va) *reinterpret_cast<uint2*>(crow) = make_uint2(pa.lo, pa.hi);
         if (vb) *reinterpret_cast<uint2*>(crow + 32 * (C / 2)) = make_uint2(pb.lo, pb.hi);
         if (a.scales_row) {
@@ -724,10 +746,13 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
           if (vb) srow[gemm ? 4 : 32 * nbr] = static_cast<uint8_t>(sb);
         }
       }
+      }
     }
 
     if constexpr (COL) {
-      const int cp = t >> 2, rb = t & 3;
+#pragma unroll
+      for (int k = 0; k < kReps; ++k) {
+      const int cp = tcp + (NT / 4) * k, rb = trb;
       if (16 * rb < rows && 2 * cp < cols) {
         const uint32_t* base = reinterpret_cast<const uint32_t*>(&s[16 * rb][0]);
         const int wofs = tile_word(16 * rb, cp);   // the same for all 16 rows of the block
@@ -739,40 +764,48 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
         }
         if constexpr (ROT) rht16x2_presigned(v);
         const int64_t gc = c0 + 2 * cp;
-        const uint64_t blka = static_cast<uint64_t>(cblk_tile + cblk_thr), blkb = blka + static_cast<uint64_t>(nbc);
+        const uint64_t blka = static_cast<uint64_t>(cblk_tile + cblk_thr + k * rep_cblk);
+        const uint64_t blkb = blka + static_cast<uint64_t>(nbc);
         Packed16 qa, qb;
         uint32_t sa, sb;
         if constexpr (VEC) {
           // tensor scales of columns gc, gc + 1; the first tile row publishes them
           const float aa = vector_alpha(a, a.vmax_c, gc), ab = vector_alpha(a, a.vmax_c, gc + 1);
-          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca, w_cb);
+          quantize_pair<MODE>(v, make_vec_scales(aa, ab), K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca[k], w_cb[k]);
           if (tr == 0 && rb == 0) {
             a.alpha_col[gc] = aa;
             a.alpha_col[gc + 1] = ab;
           }
         } else {
-          quantize_pair<MODE>(v, scc, K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca, w_cb);
+          quantize_pair<MODE>(v, scc, K, c2c, blka, blkb, qa, qb, sa, sb, share, w_ca[k], w_cb[k]);
         }
         *reinterpret_cast<uint2*>(&colcodes[2 * cp][8 * rb]) = make_uint2(qa.lo, qa.hi);
         *reinterpret_cast<uint2*>(&colcodes[2 * cp + 1][8 * rb]) = make_uint2(qb.lo, qb.hi);
         colscale[2 * cp][rb] = static_cast<uint8_t>(sa);
         colscale[2 * cp + 1][rb] = static_cast<uint8_t>(sb);
       }
+      }
       __syncthreads();
       if (rows == TR && cols == TC && col_words) {
-        // whole tile: thread t copies 16 code bytes of column t / 2 and
-        // threads 0..127 the 4-byte word of column t's four scales
-        const int c = t >> 1, h = t & 1;
-        *reinterpret_cast<uint4*>(a.codes_col + (c0 * (R / 2) + r0 / 2) + ccode_thr) =
-            *reinterpret_cast<const uint4*>(&colcodes[c][16 * h]);
-        if (a.scales_col && t < TC) {
-          const int64_t off = gemm ? gemm_scale_tile_col(tr, tc, nbc) + gemm_scale_thread_col(t)
-                                   : cblk_tile + t * nbc;
-          *reinterpret_cast<uint32_t*>(a.scales_col + off) = *reinterpret_cast<const uint32_t*>(&colscale[t][0]);
+        // whole tile: thread t copies 16 code bytes of column t / 2 (+ NT / 2
+        // per unit) and the 4-byte word of column t's (t + NT ..) four scales
+#pragma unroll
+        for (int k = 0; k < kReps; ++k) {
+          const int c = (t >> 1) + (NT / 2) * k, h = t & 1;
+          *reinterpret_cast<uint4*>(a.codes_col + (c0 * (R / 2) + r0 / 2) + ccode_thr + k * rep_ccode) =
+              *reinterpret_cast<const uint4*>(&colcodes[c][16 * h]);
+        }
+        if (a.scales_col) {
+          for (int c = t; c < TC; c += NT) {
+            const int64_t off = gemm ? gemm_scale_tile_col(tr, tc, nbc) + gemm_scale_thread_col(c)
+                                     : cblk_tile + c * nbc;
+            *reinterpret_cast<uint32_t*>(a.scales_col + off) = *reinterpret_cast<const uint32_t*>(&colscale[c][0]);
+          }
         }
       } else {
-        {
-          const int c = t >> 1, h = t & 1;
+#pragma unroll
+        for (int k = 0; k < kReps; ++k) {
+          const int c = (t >> 1) + (NT / 2) * k, h = t & 1;
           const int nbytes = rows / 2;
           if (c < cols && 16 * h < nbytes) {
             uint8_t* dst = a.codes_col + (c0 + c) * (R / 2) + r0 / 2 + 16 * h;
@@ -782,8 +815,7 @@ __device__ __forceinline__ void quant_tile_1d_body(const QuantArgs& a, uint32_t 
           }
         }
         if (a.scales_col) {
-          const int c = t >> 1;
-          if (c < cols) {
+          for (int c = t >> 1; c < cols; c += NT / 2) {
             for (int rb2 = (t & 1); rb2 < rows / 16; rb2 += 2) {
               const int64_t gc = c0 + c, grb = r0 / 16 + rb2;
               const uint8_t sbyte = colscale[c][rb2];
@@ -1082,11 +1114,12 @@ __global__ void __launch_bounds__(NT) quant_rows_kernel(const QuantArgs a) {
 }
 
 template <int MODE, bool ROT, bool ROW, bool COL, bool VEC>
-__global__ void __launch_bounds__(TNT, tile_1d_min_blocks<MODE>()) quant_tile_1d_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(tile_1d_threads<MODE>(), tile_1d_min_blocks<MODE>())
+    quant_tile_1d_kernel(const QuantArgs a) {
   pdl_entry();
   extern __shared__ __align__(16) uint8_t tile_ring[];
   __shared__ __align__(16) TileStaging stg;
-  quant_tile_1d_body<MODE, ROT, ROW, COL, VEC>(a, blockIdx.x, gridDim.x, tile_ring, stg);
+  quant_tile_1d_body<MODE, ROT, ROW, COL, VEC, tile_1d_threads<MODE>()>(a, blockIdx.x, gridDim.x, tile_ring, stg);
 }
 
 // Per-vector maxima for NVFP4_VECTOR_SCALES: max |x| (over rotated 16-blocks
@@ -1369,12 +1402,12 @@ static cudaError_t launch_tile_1d(const QuantArgs& a, cudaStream_t st) {
   if (per_sm == 0) {
     int n = 0;
     cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, TNT, smem) != cudaSuccess || n <= 0) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, tile_1d_threads<MODE>(), smem) != cudaSuccess || n <= 0) n = 1;
     per_sm = n;
   }
   const uint32_t ntiles = static_cast<uint32_t>(a.tiles_r * a.tiles_c);
   const int blocks = static_cast<int>(std::min<int64_t>(ntiles, static_cast<int64_t>(sm_count()) * per_sm));
-  launch_k(fn, dim3(std::max(blocks, 1)), dim3(TNT), smem, st, 1u, a);
+  launch_k(fn, dim3(std::max(blocks, 1)), dim3(tile_1d_threads<MODE>()), smem, st, 1u, a);
   note_launch();
   return cudaGetLastError();
 }
