@@ -431,7 +431,7 @@ def quantize_modes_table(api, tensors, hbm, flush, iters=7):
 
 
 def sweep_table(api, hbm, flush, device):
-    """BASELINE config 4: bf16 4096 x N, every mode, rows and rows + columns,
+    """The size sweep: bf16 4096 x N, every mode, rows and rows + columns,
     two-pass vs single-pass amax; Gelem/s and fraction of HBM bandwidth."""
     import torch
     from nvfp4_block_quantization_amax_b200 import synthetic
@@ -688,7 +688,7 @@ def run_extras(args, step, x, w, dy, device, hbm, fp4_peak):
                             "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / fp4_peak,
                             "frac_datasheet": fl / (ms * 1e-3) / 1e12 / FP4_DATASHEET_TFLOPS}
     del mx_x, mx_w
-    # the 12B-hybrid-shaped step (BASELINE config 5): tokens 16384, hidden 5120, FFN 20480
+    # the 12B-hybrid-shaped step: tokens 16384, hidden 5120, FFN 20480
     s = synthetic.STEP_12B
     lay = synthetic.device_layer(s["tokens"], s["hidden"], s["ffn"], seed=12, device=device)
     st12 = LayerStep(lay["x"], lay["w"], lay["dy"], BWD_MODES[args.bwd_mode], device,
