@@ -115,3 +115,17 @@ def test_quantizer_issue_record_checks_the_sources(tmp_path, monkeypatch):
     h = hashlib.sha256(b"".join(f.encode() for f in bench.QUANT_SOURCES)).hexdigest()[:16]
     (prof / "quantizer_issue.json").write_text(json.dumps({"source_sha256_16": h, "kernels": []}))
     assert bench.quantizer_issue_record() == {"source_sha256_16": h, "kernels": []}
+
+
+def test_carve_lays_shapes_end_to_end():
+    # the e2e buffers: X, W, dY (and Y, dX, dW) as consecutive row-major views
+    # of one buffer, so each direction is a single copy of all of them
+    import torch
+    shapes = [(3, 4), (5, 4), (3, 5)]
+    buf = torch.arange(sum(r * c for r, c in shapes), dtype=torch.float32)
+    views = bench.carve(buf, shapes)
+    assert [tuple(v.shape) for v in views] == shapes
+    assert all(v.is_contiguous() for v in views)
+    assert torch.equal(torch.cat([v.reshape(-1) for v in views]), buf)
+    views[1][0, 0] = -1.0   # views, not copies
+    assert buf[12].item() == -1.0
